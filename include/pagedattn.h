@@ -1,0 +1,217 @@
+/*
+ * pagedattn.h — C ABI of libpagedattn.so, paged decode attention for NVIDIA B200 (sm_100a).
+ *
+ * Scope: the decode-step hot path of PagedAttention. The KV cache is cut into fixed
+ * 16-token blocks scattered through a physical block pool; a per-sequence block table maps
+ * logical blocks to physical ones; sequences with a common prefix share physical blocks,
+ * counted by ref_count, and a shared block is copied before it is written (copy-on-write).
+ * Sources (page title, section):
+ *   [KVPaged] "KV cache and paged attention" (youngju.dev)
+ *   [Ch4PA]   "Why PagedAttention cuts GPU memory waste by up to 95%" (iq-universe.github.io,
+ *             ch4-paged-attention)
+ *   [OpsVLLM] "How does vLLM PagedAttention manage the KV cache" (opsoai.com)
+ *   [KVFail]  "Transformer inference KV-cache memory-management failure modes"
+ *             (knowledge.openakashic.com)
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named *_cache, q, out, k, v, block_tables, context_lens, slot_mapping, pairs,
+ *   *_scales, lse_out and workspace are DEVICE pointers; the caller owns them. The library
+ *   allocates no device memory.
+ * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device
+ *   work is enqueued asynchronously on it; a PA_OK return means "enqueued".
+ * - Every call validates its host-side arguments first and returns an error without
+ *   enqueuing anything when they are wrong. Faults of asynchronous work show up at the next
+ *   synchronisation, as with any CUDA launch.
+ * - Data that lives on the device cannot be validated by the host. Kernels bounds-check
+ *   every block id, slot and copy pair they read; an out-of-range value is skipped (the
+ *   access is not made) and recorded in a device error word, see pa_device_error().
+ * - Cache layout: cache[num_blocks][num_kv_heads][block_size][head_dim], row-major, so each
+ *   (physical block, kv head) tile is contiguous (the pages give no layout; this is the
+ *   library's choice). fp8 caches carry float32 scales[num_blocks][num_kv_heads], one per
+ *   (block, kv head), separately for K and V: stored value = E4M3(x / scale).
+ * - q and out: [num_seqs][num_q_heads][head_dim] row-major. Query head h reads kv head
+ *   h / (num_q_heads / num_kv_heads) ([KVPaged] "GQA and MQA": query heads are grouped and
+ *   each group shares one KV head).
+ * - block_tables: int32 [num_seqs][max_blocks_per_seq]; entry b of row s is the physical
+ *   block holding logical tokens [16b, 16b+16) of sequence s; entries at or beyond
+ *   ceil(context_lens[s] / block_size) are never read ([Ch4PA] "PagedAttention algorithm":
+ *   the block table maps logical block ids to physical blocks that need not be contiguous).
+ * - context_lens[s] counts every cached token of sequence s, including the token being
+ *   decoded (whose K/V must have been written by reshape_and_cache first).
+ *
+ * Supported today: block_size 16; head_dim 64, 128 or 256; num_q_heads a multiple of
+ * num_kv_heads with a group of at most 16; (q, kv, out) dtypes (f32, f32, f32),
+ * (bf16, bf16, bf16) and (bf16, fp8_e4m3, bf16). Anything else returns PA_ERR_UNSUPPORTED.
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
+
+typedef enum {
+  PA_OK = 0,
+  PA_ERR_INVALID = -1,      /* bad argument: null pointer, size out of range, bad id      */
+  PA_ERR_UNSUPPORTED = -2,  /* valid but not implemented (dtype combination, head_dim...) */
+  PA_ERR_CUDA = -3,         /* a CUDA runtime call or launch failed                       */
+  PA_ERR_NO_BLOCKS = -4,    /* allocator: not enough free blocks; nothing was changed     */
+  PA_ERR_WORKSPACE = -5,    /* workspace missing or smaller than paged_attn_workspace_size */
+  PA_ERR_DEVICE = -6        /* a kernel recorded a bad block id / slot / pair, see below  */
+} pa_status;
+
+/* Bits of the device error word (pa_device_error). */
+#define PA_DEVERR_BLOCK_ID 0x1   /* block table entry outside [0, num_blocks)          */
+#define PA_DEVERR_SLOT 0x2       /* slot_mapping entry outside [-inf, num_blocks*bs)    */
+#define PA_DEVERR_PAIR 0x4       /* copy_blocks pair outside [0, num_blocks)            */
+#define PA_DEVERR_CONTEXT 0x8    /* context_lens entry < 0 or > max_context_len         */
+#define PA_DEVERR_TIMEOUT 0x10   /* a bounded wait on an asynchronous copy gave up      */
+
+/* Shape and dtypes of one paged decode-attention call. */
+typedef struct {
+  int num_seqs;            /* S >= 0                                                   */
+  int num_q_heads;         /* Hq                                                       */
+  int num_kv_heads;        /* Hkv; Hq % Hkv == 0                                       */
+  int head_dim;            /* d                                                        */
+  int block_size;          /* tokens per block (16)                                    */
+  int max_blocks_per_seq;  /* row stride of block_tables                               */
+  int num_blocks;          /* physical blocks in the pool (bounds check)               */
+  int partition_size;      /* split-KV partition in tokens, a multiple of block_size;  */
+                           /* 0 = one pass over the whole context per (seq, kv head)   */
+  pa_dtype q_dtype, kv_dtype, out_dtype;
+} pa_decode_desc;
+
+/*
+ * Bytes of device workspace paged_attn_decode needs for this shape when no context is
+ * longer than max_context_len (0 when partition_size == 0). Returns 0 for an invalid
+ * descriptor as well; paged_attn_decode then reports the error.
+ */
+size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len);
+
+/*
+ * Decode attention over the paged cache ([KVPaged] "Core principle: what is the KV cache":
+ * attention(Q,K,V) = softmax(Q K^T / sqrt(d_k)) V, one new query per sequence; [Ch4PA]
+ * "PagedAttention algorithm": the kernel looks every logical block up in the block table
+ * and gathers the non-contiguous K and V blocks). For every sequence s and query head h,
+ * with g = h / (Hq/Hkv) and the cached tokens t < context_lens[s]:
+ *     z_t = scale * q[s][h] . K_t,   out[s][h] = sum_t softmax(z)_t V_t,
+ *     lse_out[s][h] = log sum_t exp(z_t)                    (natural log, float32)
+ * fp8 caches are dequantised as E4M3 value * scales[block][g]. Accumulation is float32.
+ * With partition_size > 0 the context is cut into partitions of that many logical tokens,
+ * each reduced to (max, sum, unnormalised output) in `workspace`, then combined by a
+ * log-sum-exp reduction; the result does not depend on where blocks sit physically.
+ *   q, out         [S][Hq][d] in desc->q_dtype / desc->out_dtype
+ *   k_cache/v_cache pool in desc->kv_dtype (layout above)
+ *   block_tables   int32 [S][max_blocks_per_seq];  context_lens int32 [S]
+ *   max_context_len  host int >= every context_lens entry (sizes the grid)
+ *   k_scales/v_scales float32 [num_blocks][Hkv], required for fp8, ignored otherwise
+ *   lse_out        float32 [S][Hq] or NULL
+ *   workspace      device bytes, >= paged_attn_workspace_size(desc, max_context_len),
+ *                  16-byte aligned; may be NULL when that size is 0
+ * A sequence with context length 0 gets out = 0 and lse = -inf.
+ */
+pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            float scale, void* out, const pa_decode_desc* desc,
+                            int max_context_len, const float* k_scales, const float* v_scales,
+                            float* lse_out, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * Slot-mapped write of new tokens' K and V into the pool ([KVPaged] "PagedAttention: OS
+ * virtual-memory style management": one block is allocated as tokens accumulate and the
+ * block table maps logical positions to physical blocks). For token t with
+ * slot = slot_mapping[t] >= 0, block = slot / block_size, offset = slot % block_size:
+ *     k_cache[block][h][offset][:] = convert(k[t][h][:])   for every kv head h (same for v)
+ * convert: f32->f32 and bf16->bf16 copy bits; f32->bf16 rounds to nearest even; f32 or
+ * bf16 -> fp8 stores E4M3(x / scale[block][h]) with an IEEE float32 division, round to
+ * nearest even, saturating to +-448. A negative slot is a padding token and is skipped.
+ *   k, v             device [num_tokens][Hkv][head_dim] rows, token stride k_stride /
+ *                    v_stride elements (>= Hkv*head_dim), in in_dtype
+ *   slot_mapping     int64 [num_tokens]
+ *   k_scales/v_scales float32 [num_blocks][Hkv], fp8 caches only (read, not written)
+ * Tokens must map to distinct slots (two writes to one slot race).
+ */
+pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                            const int64_t* slot_mapping, int num_tokens, int64_t k_stride,
+                            int64_t v_stride, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, pa_dtype in_dtype, pa_dtype cache_dtype,
+                            const float* k_scales, const float* v_scales, void* stream);
+
+/*
+ * Copy-on-write block copy ([KVPaged] "Prefix sharing and copy-on-write": a shared block is
+ * copied before one sharer modifies it; [Ch4PA] "Prefix Caching": copies happen only on
+ * write). For each pair i, (src, dst) = (pairs[2i], pairs[2i+1]) (device int32 [n][2]):
+ * the K and V tiles of every kv head of block src are copied to block dst, and for fp8
+ * caches the scales too (k_scales/v_scales may be NULL otherwise). No dst may appear twice
+ * or also be a src: such copies race. Enqueue it before the reshape_and_cache that writes
+ * into the destination blocks.
+ */
+pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_scales,
+                      const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, pa_dtype cache_dtype, void* stream);
+
+/*
+ * Reads and clears the device error word of the current device (a bitwise OR of
+ * PA_DEVERR_* recorded by kernels since the last call). Synchronises `stream` first.
+ * Returns PA_OK when the word was 0, PA_ERR_DEVICE otherwise (bits in *bits_out).
+ */
+pa_status pa_device_error(int* bits_out, void* stream);
+
+/* Library version string, e.g. "pagedattn 0.1 sm_100a". */
+const char* pa_version(void);
+
+/* ------------------------------------------------------------------------------------- */
+/* Host block allocator ([Ch4PA] "Borrowing the fix from OS paging": a free list of       */
+/* fixed-size units; [KVFail] Key Points: blocks come from a free queue and an allocation */
+/* fails when too few are free; [KVPaged] "Prefix sharing and copy-on-write" and [Ch4PA]  */
+/* "Prefix Caching": ref_count per block, copy only on write).                            */
+/*                                                                                       */
+/* Policy: FIFO free queue (initial order given or 0..N-1); allocation pops the front; a */
+/* block whose ref_count reaches 0 is pushed to the back. add_seq allocates              */
+/* ceil(n/block_size) blocks; fork copies the parent's table and length and increments  */
+/* every block's ref_count; append first copies the last block if it is partially filled */
+/* AND shared (one new block, the pair (old, new) reported, old loses one reference),    */
+/* then pops one block per new block boundary crossed. Every call either succeeds fully  */
+/* or returns an error and changes nothing. Host only; not thread-safe; the caller owns   */
+/* the object. Sequence ids are any non-negative int.                                    */
+/* ------------------------------------------------------------------------------------- */
+typedef struct pa_allocator pa_allocator;
+
+/* NULL on bad sizes / allocation failure. */
+pa_allocator* pa_alloc_create(int num_blocks, int block_size);
+/* `order`: host int32[num_blocks], a permutation of 0..num_blocks-1 giving the initial
+ * free-queue order. NULL when it is not a permutation. */
+pa_allocator* pa_alloc_create_ordered(int num_blocks, int block_size, const int32_t* order);
+void pa_alloc_destroy(pa_allocator* a);
+int pa_alloc_num_free(const pa_allocator* a);
+/* -1 for a block id out of range. */
+int pa_alloc_ref_count(const pa_allocator* a, int block);
+/* New sequence of num_tokens tokens; host int64 slots_out[num_tokens] (may be NULL)
+ * receives slot = block*block_size + offset of every token. */
+pa_status pa_alloc_add_seq(pa_allocator* a, int seq_id, int num_tokens, int64_t* slots_out);
+pa_status pa_alloc_fork(pa_allocator* a, int parent_id, int child_id);
+/* Appends num_tokens tokens; slots_out[num_tokens] receives their slots; cow_pairs_out
+ * (host int32[2], may be NULL only if no copy can occur) receives (src, dst) of the
+ * copy-on-write copy and *num_cow_out is 0 or 1. */
+pa_status pa_alloc_append(pa_allocator* a, int seq_id, int num_tokens, int64_t* slots_out,
+                          int32_t* cow_pairs_out, int* num_cow_out);
+pa_status pa_alloc_free_seq(pa_allocator* a, int seq_id);
+/* Copies at most `cap` entries of the sequence's block table into out (host int32) and
+ * returns the table's length, or -1 for an unknown sequence. */
+int pa_alloc_block_table(const pa_allocator* a, int seq_id, int32_t* out, int cap);
+/* Tokens held by the sequence, -1 if unknown. */
+int pa_alloc_seq_len(const pa_allocator* a, int seq_id);
+/* Writes the free queue front-to-back into out (at most cap entries); returns its size. */
+int pa_alloc_free_queue(const pa_allocator* a, int32_t* out, int cap);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDATTN_H_ */

@@ -1,0 +1,228 @@
+"""Paged KV-cache bookkeeping and cache writes of the oracle (test infrastructure only).
+
+Cache layout (a reading: the pages give no memory layout): ``cache[num_blocks][num_kv_heads]
+[block_size][head_dim]``, i.e. every (physical block, kv head) tile is contiguous. The oracle
+stores the cache in its storage codes: float32 values, uint16 bf16 bits or uint8 E4M3 codes.
+
+[KVPaged] "PagedAttention: OS virtual-memory style management": the cache is cut into small
+fixed-size blocks, one block is allocated as tokens accumulate, and a per-request block
+table maps logical token positions to physical blocks (16-token example: 40 tokens ->
+[blk0, blk3, blk5], 20 tokens -> [blk1, blk2]).
+[Ch4PA] "PagedAttention algorithm": logical block id -> physical block address, physical
+addresses need not be contiguous; "OS paging": a free list of fixed-size units always
+serves an allocation while enough units remain.
+[KVFail] Key Points: when free blocks are short the allocation fails (read: the call fails
+and changes nothing); blocks are handed out from a free queue.
+[KVPaged] "Prefix sharing and copy-on-write" and [Ch4PA] "Prefix Caching": sequences with a
+common prefix point at the same physical blocks, a ref_count tracks the sharers, and a
+shared block is copied only when a writer modifies it.
+"""
+from __future__ import annotations
+
+from collections import deque
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+from .codecs import bf16_encode, bf16_decode, e4m3_encode
+
+
+class NoBlocks(Exception):
+    """The free queue holds fewer blocks than the call needs; nothing was changed."""
+
+
+class InvalidCall(Exception):
+    """Unknown / duplicate sequence id or a bad argument; nothing was changed."""
+
+
+def slot_of(block_table_row: Sequence[int], pos: int, block_size: int) -> int:
+    """Slot of logical token ``pos``: physical block * block_size + offset in the block."""
+    return int(block_table_row[pos // block_size]) * block_size + pos % block_size
+
+
+class RefAllocator:
+    """Reference block allocator.
+
+    Policy (readings, stated once):
+    * the free queue is FIFO, initialised with ``order`` (default 0..N-1); allocation pops
+      from the front; a block whose ref_count drops to 0 is pushed to the back;
+    * ``add_seq(s, n)`` allocates ceil(n/B) blocks in logical order;
+    * ``fork(p, c)`` gives ``c`` a copy of ``p``'s block table and length and increments the
+      ref_count of every block in it;
+    * ``append(s, n)``: if the last block is partially filled AND shared (ref_count > 1) it is
+      copied first: one new block is popped, the pair (old, new) is reported, ``old`` loses a
+      reference and ``new`` takes its place in the table; then one block is popped for every
+      new 16-token boundary crossed. A full shared block is never written, so it is never
+      copied. At most one copy pair per call;
+    * every call checks first and changes nothing when it fails.
+    """
+
+    def __init__(self, num_blocks: int, block_size: int = 16,
+                 order: Optional[Sequence[int]] = None):
+        if num_blocks <= 0 or block_size <= 0:
+            raise InvalidCall("sizes")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        if order is None:
+            order = range(num_blocks)
+        order = [int(b) for b in order]
+        if sorted(order) != list(range(num_blocks)):
+            raise InvalidCall("order must be a permutation of the block ids")
+        self.free: deque = deque(order)
+        self.refs: List[int] = [0] * num_blocks
+        self.tables: Dict[int, List[int]] = {}
+        self.lens: Dict[int, int] = {}
+
+    # -- queries ------------------------------------------------------------------------
+    def num_free(self) -> int:
+        return len(self.free)
+
+    def ref_count(self, block: int) -> int:
+        return self.refs[block]
+
+    def block_table(self, seq: int) -> List[int]:
+        return list(self.tables[seq])
+
+    def seq_len(self, seq: int) -> int:
+        return self.lens[seq]
+
+    # -- mutations ----------------------------------------------------------------------
+    def _pop(self) -> int:
+        b = self.free.popleft()
+        self.refs[b] = 1
+        return b
+
+    def _slots(self, seq: int, start: int, n: int) -> np.ndarray:
+        row = self.tables[seq]
+        return np.array([slot_of(row, p, self.block_size) for p in range(start, start + n)],
+                        dtype=np.int64)
+
+    def add_seq(self, seq: int, num_tokens: int) -> np.ndarray:
+        if seq in self.tables or num_tokens < 0:
+            raise InvalidCall("add_seq")
+        need = -(-num_tokens // self.block_size)
+        if need > len(self.free):
+            raise NoBlocks()
+        self.tables[seq] = [self._pop() for _ in range(need)]
+        self.lens[seq] = num_tokens
+        return self._slots(seq, 0, num_tokens)
+
+    def fork(self, parent: int, child: int) -> None:
+        if parent not in self.tables or child in self.tables:
+            raise InvalidCall("fork")
+        self.tables[child] = list(self.tables[parent])
+        self.lens[child] = self.lens[parent]
+        for b in self.tables[child]:
+            self.refs[b] += 1
+
+    def append(self, seq: int, num_tokens: int) -> Tuple[np.ndarray, List[Tuple[int, int]]]:
+        if seq not in self.tables or num_tokens < 0:
+            raise InvalidCall("append")
+        B = self.block_size
+        L = self.lens[seq]
+        row = self.tables[seq]
+        cow = num_tokens > 0 and L % B != 0 and self.refs[row[-1]] > 1
+        grow = -(-(L + num_tokens) // B) - -(-L // B)
+        if int(cow) + grow > len(self.free):
+            raise NoBlocks()
+        pairs: List[Tuple[int, int]] = []
+        if cow:
+            old = row[-1]
+            new = self._pop()
+            self.refs[old] -= 1
+            row[-1] = new
+            pairs.append((old, new))
+        for _ in range(grow):
+            row.append(self._pop())
+        self.lens[seq] = L + num_tokens
+        return self._slots(seq, L, num_tokens), pairs
+
+    def free_seq(self, seq: int) -> None:
+        if seq not in self.tables:
+            raise InvalidCall("free_seq")
+        for b in self.tables.pop(seq):
+            self.refs[b] -= 1
+            if self.refs[b] == 0:
+                self.free.append(b)
+        del self.lens[seq]
+
+    def padded_tables(self, seqs: Sequence[int], max_blocks: int) -> np.ndarray:
+        """int32 [len(seqs), max_blocks] block tables, unused entries -1."""
+        out = np.full((len(seqs), max_blocks), -1, dtype=np.int32)
+        for i, s in enumerate(seqs):
+            row = self.tables[s]
+            out[i, :len(row)] = row
+        return out
+
+
+# ---------------------------------------------------------------------------------------
+# cache storage
+# ---------------------------------------------------------------------------------------
+_STORE = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}
+
+
+def new_cache(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
+              cache_dtype: str) -> np.ndarray:
+    """A zeroed cache of storage codes (zeros decode to +0.0 in every format)."""
+    return np.zeros((num_blocks, num_kv_heads, block_size, head_dim), dtype=_STORE[cache_dtype])
+
+
+def _to_f32(x: np.ndarray, in_dtype: str) -> np.ndarray:
+    if in_dtype == "f32":
+        return np.asarray(x, dtype=np.float32)
+    if in_dtype == "bf16":
+        return bf16_decode(x).astype(np.float32)  # exact
+    raise ValueError(in_dtype)
+
+
+def _convert(xf: np.ndarray, cache_dtype: str, scale: Optional[np.ndarray]) -> np.ndarray:
+    """float32 values -> storage codes of ``cache_dtype``.
+
+    fp8: code = E4M3(x / scale) with the division done in IEEE float32 (round to nearest),
+    ``scale`` broadcast over the head dimension."""
+    if cache_dtype == "f32":
+        return xf.astype(np.float32)
+    if cache_dtype == "bf16":
+        return bf16_encode(xf)
+    if cache_dtype == "fp8":
+        y = (xf / scale[..., None].astype(np.float32)).astype(np.float32)
+        return e4m3_encode(y)
+    raise ValueError(cache_dtype)
+
+
+def ref_reshape_and_cache(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,
+                          v_cache: np.ndarray, slot_mapping: np.ndarray, in_dtype: str,
+                          cache_dtype: str, k_scales: Optional[np.ndarray] = None,
+                          v_scales: Optional[np.ndarray] = None) -> None:
+    """Slot-mapped write of new tokens' K and V into the paged cache (in place).
+
+    For token t with slot = slot_mapping[t] >= 0: block = slot // B, offset = slot % B and
+    ``cache[block][h][offset][:] = convert(x[t][h][:])`` for every kv head h. A negative
+    slot marks a padding token and is skipped. fp8 caches use the per-(block, kv head)
+    scale of the destination block.
+    """
+    B = k_cache.shape[2]
+    slots = np.asarray(slot_mapping, dtype=np.int64)
+    for t, slot in enumerate(slots):
+        if slot < 0:
+            continue
+        blk, off = int(slot // B), int(slot % B)
+        for x, cache, sc in ((k, k_cache, k_scales), (v, v_cache, v_scales)):
+            xf = _to_f32(x[t], in_dtype)  # [Hkv, d]
+            s = None if sc is None else sc[blk]  # [Hkv]
+            cache[blk, :, off, :] = _convert(xf, cache_dtype, s)
+
+
+def ref_copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray,
+                    pairs: Sequence[Tuple[int, int]],
+                    k_scales: Optional[np.ndarray] = None,
+                    v_scales: Optional[np.ndarray] = None) -> None:
+    """Copy-on-write block copy: for each (src, dst) pair, in order, the K and V tiles of
+    every kv head (and the fp8 scales, when given) of ``src`` are copied to ``dst``."""
+    for src, dst in pairs:
+        k_cache[dst] = k_cache[src]
+        v_cache[dst] = v_cache[src]
+        if k_scales is not None:
+            k_scales[dst] = k_scales[src]
+        if v_scales is not None:
+            v_scales[dst] = v_scales[src]
