@@ -1,0 +1,444 @@
+#!/usr/bin/env python
+"""Paged decode attention on B200: KV-read GB/s (% of HBM peak) and decode tokens/s.
+
+One step = one decode step of the workload through the library: copy-on-write block copies
+(shared-prefix workload only), the slot-mapped write of this step's new K/V, and decode
+attention over the paged cache (split into partitions + log-sum-exp reduce where the
+workload says so). Inputs are resident in HBM when the timed region starts; L2 is flushed
+(a write of twice its size) between timed steps, outside the timed events.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload b256] [--impl ours|reference]
+
+N > 1 runs under torchrun: every rank runs an independent replica of the workload (decode
+has no exchange step; there is no collective on the data path), ``value`` counts the KV
+bytes of all ranks over the slowest rank's time ("weak" scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "paged decode attention KV GB/s (% of HBM peak) and decode tokens/s at 1 B200"
+UNIT = "GB/s"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DTYPE = {"f32": "f32", "bf16": "bf16-kv/f32-acc", "fp8": "fp8e4m3-kv/f32-acc"}
+DESCR = {
+    "tiny": "tiny paged decode: 4 seqs ctx {5,16,17,40}, 4q/2kv, d64, fp32",
+    "b32": "decode batch 32: ctx U[1,4096], 32q/8kv, d128, bf16 KV",
+    "shared": "shared prefix: 100 seqs x (200 shared + 50 private), 32q/8kv, d128, bf16, CoW",
+    "b256": "decode batch 256: ctx lognormal(1024,1) clip [16,8192], 32q/8kv, d128, fp8-e4m3 KV",
+    "long": "long context: 8 seqs x 131072, 64q/8kv, d128, bf16 KV, split-KV 512",
+}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------------------
+_REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+            0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+            0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+            0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    def __init__(self, index: int):
+        self.index = index
+        self.samples = []
+        self.proc = None
+
+    def __enter__(self):
+        q = "timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active"
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.index)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.samples:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 5:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), int(parts[4], 16)))
+            except ValueError:
+                continue
+        inside = [r for r in rows if t0 <= r[0] <= t1]
+        note = "inside timed region"
+        if not inside and rows:
+            inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:3]
+            note = "nearest samples (timed region shorter than the sampling period)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "nvidia-smi unavailable"}
+        mask = 0
+        for r in inside:
+            mask |= r[3]
+        reasons = [n for b, n in _REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": float(np.median([r[1] for r in inside])), "sm_max_mhz": inside[0][2],
+                "reasons": reasons, "samples": len(inside), "note": note}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+def _time_steps(torch, sc, steps: int, flush, per_step_events: bool = True):
+    """Device time of `steps` steps with an L2 flush between them (outside the events);
+    also the device time of the decode call alone inside each step."""
+    st = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        a, b, c = ev[i]
+        a.record(st)
+        if sc.pairs is not None:
+            sc.cache.copy(sc.pairs)
+        sc.cache.write(sc.step_k, sc.step_v, sc.step_slots)
+        b.record(st)
+        sc.cache.decode(sc.q, sc.block_tables, sc.context_lens, sc.scale, sc.out,
+                        max_context_len=sc.max_context_len, partition_size=sc.partition_size,
+                        lse_out=sc.lse, workspace=sc.workspace)
+        c.record(st)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(c) for a, b, c in ev) / 1e3
+    dec = [b.elapsed_time(c) / 1e3 for a, b, c in ev]
+    return total, float(np.mean(dec))
+
+
+def _e2e(torch, sc, steps: int, flush):
+    """Same step through the public API from pinned host buffers: H2D of the step's inputs,
+    the step, D2H of the output, all inside the timed events."""
+    st = torch.cuda.current_stream()
+    host = {}
+    for name in ("q", "step_k", "step_v", "step_slots", "block_tables", "context_lens"):
+        t = getattr(sc, name)
+        host[name] = t.cpu().pin_memory()
+    out_h = torch.empty(sc.out.shape, dtype=sc.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+    pairs_h = sc.pairs.cpu().pin_memory() if sc.pairs is not None else None
+    if pairs_h is not None:
+        h2d += pairs_h.numel() * 4
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    for i in range(steps):
+        flush()
+        a, c = ev[i]
+        a.record(st)
+        for name, t in host.items():
+            getattr(sc, name).copy_(t, non_blocking=True)
+        if pairs_h is not None:
+            sc.pairs.copy_(pairs_h, non_blocking=True)
+        sc.step()
+        out_h.copy_(sc.out, non_blocking=True)
+        c.record(st)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(c) for a, c in ev) / 1e3
+    return total, h2d, d2h
+
+
+def _cpu_baseline(draw, seconds: float = 12.0):
+    """The oracle, as it stands, on the host cores: this step's cache write plus decode for a
+    bounded sample of the workload's sequences (cycled until ~`seconds` elapse)."""
+    from oracle import flows, paged as opaged, attention
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+    wl = draw.wl
+    rng = np.random.default_rng(0)
+    sample = sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, 8), replace=False).tolist())
+    st = flows.build_state(draw, write_seqs=sample)
+    sc = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
+    es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+    done_bytes = 0
+    t0 = time.perf_counter()
+    i = 0
+    while True:
+        s = sample[i % len(sample)]
+        k, v = draw.kv(s)
+        opaged.ref_reshape_and_cache(k[-1:], v[-1:], st.k_cache, st.v_cache, st.step_slots[s],
+                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales)
+        attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                             sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype, st.k_scales,
+                             st.v_scales, seqs=[s])
+        done_bytes += int(draw.context_lens[s]) * 2 * wl.num_kv_heads * wl.head_dim * es
+        i += 1
+        el = time.perf_counter() - t0
+        if el >= seconds and i >= len(sample):
+            break
+    return {"value": done_bytes / el / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+            "sample": f"{i} (seq, all heads) decode steps cycling over {len(sample)} of "
+                      f"{wl.num_seqs} sequences of the same workload, float64 NumPy, "
+                      f"{el:.1f} s"}
+
+
+def run_ours(args):
+    import torch
+    from paged_kv_cache_465_b200.scenario import DeviceScenario
+    import paged_kv_cache_465_b200 as pa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    pa.set_decode_impl(args.decode_impl)
+    wl = workloads.WORKLOADS[args.workload]
+    draw = workloads.draw(wl)
+    sc = DeviceScenario(draw, draw_seqs=[], partition_size=args.partition)
+    l2 = torch.cuda.get_device_properties(local).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 64 << 20) // 4, dtype=torch.float32, device="cuda")
+
+    def flush():
+        flush_buf.fill_(1.0)
+
+    for _ in range(args.warmup):
+        flush()
+        sc.step()
+    torch.cuda.synchronize()
+    assert pa.device_error() == 0
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_wall0 = time.time()
+        total, dec_mean = _time_steps(torch, sc, args.steps, flush)
+        t_wall1 = time.time()
+    if dist is not None:
+        t = torch.tensor([total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+        dist.barrier()
+    torch.cuda.synchronize()
+    ms = total / args.steps * 1e3
+    b = sc.step_bytes()
+    peak, peak_kind = _peaks()
+    kv_gbs = world * b["kv"] * args.steps / total / 1e9
+    # e2e through the public API from host buffers
+    e2e_total, h2d, d2h = _e2e(torch, sc, max(args.steps // 4, 3), flush)
+    if dist is not None:
+        t = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_total = float(t.item())
+    e2e_steps = max(args.steps // 4, 3)
+    e2e_gbs = world * b["kv"] * e2e_steps / e2e_total / 1e9
+    # roofline of the dominant operation: paged_attn_decode (main kernel + LSE reduce)
+    dec_achieved = b["decode"] / dec_mean / 1e9
+    result = {
+        "metric": METRIC, "value": round(kv_gbs, 2), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": DTYPE[wl.kv_dtype], "data": "synthetic (seeded N(0,1) K/V/q, seeded lengths)",
+        "config": {"workload": DESCR[args.workload], "name": args.workload,
+                   "num_seqs": wl.num_seqs, "q_heads": wl.num_q_heads,
+                   "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
+                   "partition_size": sc.partition_size,
+                   "tokens_in_cache": int(draw.context_lens.sum()),
+                   "kv_bytes_per_step": b["kv"], "step_bytes": b,
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "flushed between timed steps (write of 2x L2), outside the events",
+                   "decode_impl": args.decode_impl},
+        "pct_hbm_peak": round(100 * kv_gbs / world / peak, 2),
+        "pct_hbm_nominal": round(100 * kv_gbs / world / NOMINAL_HBM_GBS, 2),
+        "tokens_per_s": round(world * wl.num_seqs / (total / args.steps), 1),
+        "tokens_per_s_note": "one attention layer per step; a 32-layer model would decode "
+                             "1/32 of this",
+        "roofline": {"kernel": "paged_attn_decode (main kernel + LSE reduce)", "bound": "hbm",
+                     "achieved": round(dec_achieved, 2), "peak": peak, "unit": "GB/s",
+                     "frac": round(dec_achieved / peak, 4), "traffic": None,
+                     "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": b["decode"],
+                     "launch_ms": round(dec_mean * 1e3, 5)},
+        "e2e": {"value": round(e2e_gbs, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": sc.launches_per_step() * args.steps,
+        "clocks": clk.summary(t_wall0, t_wall1),
+    }
+    traffic = _traffic_note(args.workload)
+    if traffic is not None:
+        result["roofline"]["traffic"] = traffic
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = _cpu_baseline(draw, args.cpu_seconds)
+    if rank == 0 and args.extra and world == 1:
+        result["workloads"] = _extra_workloads(torch, pa, args, flush)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+def _traffic_note(name):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary, if one
+    matches the current kernel build (profiles/traffic.json); else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        j = json.load(f)
+    e = j.get(name)
+    if not e:
+        return None
+    return e.get("bytes_per_launch")
+
+
+def _extra_workloads(torch, pa, args, flush):
+    from paged_kv_cache_465_b200.scenario import DeviceScenario
+    peak, _ = _peaks()
+    out = {}
+    for name in ("tiny", "b32", "shared", "b256", "long"):
+        if name == args.workload:
+            continue
+        draw = workloads.draw(name)
+        sc = DeviceScenario(draw, draw_seqs=[] if name in ("b256", "long", "b32") else None)
+        for _ in range(3):
+            flush()
+            sc.step()
+        steps = 50 if name == "long" else 200
+        total, dec = _time_steps(torch, sc, steps, flush)
+        b = sc.step_bytes()
+        gbs = b["kv"] * steps / total / 1e9
+        out[name] = {"value": round(gbs, 2), "unit": UNIT, "ms_per_step": round(total / steps * 1e3, 5),
+                     "pct_hbm_peak": round(100 * gbs / peak, 2),
+                     "pct_hbm_nominal": round(100 * gbs / NOMINAL_HBM_GBS, 2),
+                     "decode_ms": round(dec * 1e3, 5),
+                     "decode_gbs": round(b["decode"] / dec / 1e9, 2),
+                     "tokens_per_s": round(draw.wl.num_seqs / (total / steps), 1),
+                     "partition_size": sc.partition_size, "steps": steps}
+        del sc
+        torch.cuda.empty_cache()
+    return out
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the oracle on the host cores
+# ---------------------------------------------------------------------------------------
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from oracle import flows, paged as opaged, attention
+    wl = workloads.WORKLOADS[args.workload]
+    draw = workloads.draw(wl)
+    rng = np.random.default_rng(0)
+    sample = sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, 8), replace=False).tolist())
+    st = flows.build_state(draw, write_seqs=sample)
+    sc = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
+    es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:  # noqa: BLE001
+        cores = os.cpu_count()
+
+    def one(i):
+        s = sample[i % len(sample)]
+        k, v = draw.kv(s)
+        opaged.ref_reshape_and_cache(k[-1:], v[-1:], st.k_cache, st.v_cache, st.step_slots[s],
+                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales)
+        attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
+                             sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype, st.k_scales,
+                             st.v_scales, seqs=[s])
+        return int(draw.context_lens[s]) * 2 * wl.num_kv_heads * wl.head_dim * es
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    nbytes = 0
+    for i in range(args.steps):
+        nbytes += one(args.warmup + i)
+    el = time.perf_counter() - t0
+    val = nbytes / el / 1e9
+    res = {"metric": METRIC, "value": round(val, 4), "unit": UNIT, "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(el / args.steps * 1e3, 4),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64", "data": "synthetic (seeded N(0,1) K/V/q, seeded lengths)",
+           "config": {"workload": DESCR[args.workload], "name": args.workload},
+           "impl": "reference",
+           "cpu_baseline": {"kind": "oracle", "cores": int(cores), "value": round(val, 4),
+                            "unit": UNIT,
+                            "sample": f"each step = one sequence (all heads) of {len(sample)} "
+                                      f"sampled sequences of the workload, cache write + decode, "
+                                      f"float64 NumPy"},
+           "e2e": {"value": round(val, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="b256", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--decode-impl", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--partition", type=int, default=None,
+                    help="split-KV partition in tokens (default: the workload's)")
+    ap.add_argument("--no-extra", dest="extra", action="store_false",
+                    help="skip the other workloads' lines")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

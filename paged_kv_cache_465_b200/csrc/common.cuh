@@ -1,0 +1,80 @@
+// Shared device helpers of libpagedattn: dtype traits, conversions written as single PTX
+// instructions, the device error word, and launch-check macros.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "pagedattn.h"
+
+namespace pa {
+
+// ---------------------------------------------------------------------------------------
+// Device error word: kernels OR PA_DEVERR_* bits into it instead of faulting; the host
+// reads and clears it with pa_device_error(). One word per device (file-scope __device__).
+// ---------------------------------------------------------------------------------------
+__device__ unsigned int g_error_word;
+
+__device__ __forceinline__ void flag_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
+
+// ---------------------------------------------------------------------------------------
+// Conversions. Each is one documented PTX conversion instruction.
+// ---------------------------------------------------------------------------------------
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Two floats -> packed bf16x2 (a in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two floats -> packed f16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two floats -> two E4M3 bytes (lo in byte 0), round to nearest even, saturate to +-448.
+__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Two E4M3 bytes (byte 0 -> low half) -> f16x2. Exact: every E4M3 value is an f16 value.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t x) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(x));
+  return r;
+}
+
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t h) {
+  float lo, hi;
+  asm("{\n\t.reg .f16 l, h;\n\tmov.b32 {l, h}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, h;\n\t}"
+      : "=f"(lo), "=f"(hi) : "r"(h));
+  return make_float2(lo, hi);
+}
+
+// 2^x on the special-function unit (PTX ex2.approx; relative error ~2^-22).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+// Element size in bytes of a pa_dtype.
+inline int dtype_bytes(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_BF16 ? 2 : 1); }
+
+}  // namespace pa
+
+#define PA_CHECK_LAUNCH()                                  \
+  do {                                                     \
+    cudaError_t e_ = cudaGetLastError();                   \
+    if (e_ != cudaSuccess) return PA_ERR_CUDA;             \
+  } while (0)

@@ -1,0 +1,323 @@
+// Paged decode attention on the CUDA cores (fp32 FMA), the reference-precision path.
+//
+// [KVPaged] "Core principle: what is the KV cache": softmax(q K^T / sqrt(d)) V for one new
+// query per sequence; [Ch4PA] "PagedAttention algorithm": each logical block is looked up
+// in the block table and its K/V tile gathered; [KVPaged] "GQA and MQA": the G query heads
+// of a group share one kv head, so one CTA serves the whole group and reads each K/V tile
+// once for all G heads.
+//
+// Work item = (sequence, kv head, partition of `part_tokens` logical tokens). A CTA of 4
+// warps takes one item; warp w walks the item's blocks w, w+4, ... so the reduction order
+// depends only on logical positions (results are independent of physical placement).
+// Per block of 16 tokens a warp computes the 16 x G scores with lane = (token, half of d),
+// keeps a running max / sum per query head (online softmax in the log2 domain), and
+// accumulates P V with lane = 4-channel slice of d. Warps are merged through shared memory
+// at the end; the item either writes the normalised output (single pass) or its
+// (max, sum, unnormalised output) partial for the log-sum-exp reduction.
+//
+// This path issues roughly (G + 1) fp32 instructions per KV element and is therefore
+// ALU-bound on B200 for G >= 4 at full HBM bandwidth; the tensor-core path replaces it for
+// bf16 / fp8 caches and it stays the path for fp32 caches and unusual shapes.
+#pragma once
+
+#include "common.cuh"
+
+namespace pa {
+
+constexpr int kSimtWarps = 4;
+constexpr int kBS = 16;  // tokens per block (template constant of the whole library)
+
+template <pa_dtype KV>
+struct KvTraits;
+template <>
+struct KvTraits<PA_F32> { static constexpr int bytes = 4; };
+template <>
+struct KvTraits<PA_BF16> { static constexpr int bytes = 2; };
+template <>
+struct KvTraits<PA_FP8_E4M3> { static constexpr int bytes = 1; };
+
+// 16 bytes of KV -> 16/bytes floats (raw stored value, scale not applied).
+template <pa_dtype KV>
+__device__ __forceinline__ void unpack16(uint4 w, float* x) {
+  if constexpr (KV == PA_F32) {
+    x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
+    x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
+  } else if constexpr (KV == PA_BF16) {
+    x[0] = bf16_lo(w.x); x[1] = bf16_hi(w.x); x[2] = bf16_lo(w.y); x[3] = bf16_hi(w.y);
+    x[4] = bf16_lo(w.z); x[5] = bf16_hi(w.z); x[6] = bf16_lo(w.w); x[7] = bf16_hi(w.w);
+  } else {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 a = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(ws[j] & 0xffff)));
+      float2 b = f16x2_to_float2(e4m3x2_to_f16x2((uint16_t)(ws[j] >> 16)));
+      x[4 * j + 0] = a.x; x[4 * j + 1] = a.y; x[4 * j + 2] = b.x; x[4 * j + 3] = b.y;
+    }
+  }
+}
+
+// D/32 consecutive channels of one token row (the lane's P.V slice), as floats.
+template <pa_dtype KV, int D>
+__device__ __forceinline__ void load_vslice(const uint8_t* row, int lane, float* x) {
+  constexpr int N = D / 32;                     // channels per lane: 2, 4 or 8
+  constexpr int BYTES = N * KvTraits<KV>::bytes;  // 2..32
+  const uint8_t* p = row + lane * BYTES;
+  if constexpr (KV == PA_F32) {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) {
+      float2 a = __ldg(reinterpret_cast<const float2*>(p) + j / 2);
+      x[j] = a.x; x[j + 1] = a.y;
+    }
+  } else if constexpr (KV == PA_BF16) {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) {
+      uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p) + j / 2);
+      x[j] = bf16_lo(w); x[j + 1] = bf16_hi(w);
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) {
+      uint16_t w = __ldg(reinterpret_cast<const uint16_t*>(p) + j / 2);
+      float2 a = f16x2_to_float2(e4m3x2_to_f16x2(w));
+      x[j] = a.x; x[j + 1] = a.y;
+    }
+  }
+}
+
+struct DecodeArgs {
+  const void* q;
+  const void* k_cache;
+  const void* v_cache;
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  void* out;
+  float* lse_out;
+  const float* k_scales;
+  const float* v_scales;
+  float* part_m;    // [S][Hq][P]   log2-domain running max of each partition
+  float* part_l;    // [S][Hq][P]   sum of exp2(z - m)
+  float* part_acc;  // [S][Hq][P][D] unnormalised sum of exp2(z - m) V
+  float scale_log2;  // scale * log2(e)
+  int num_seqs, num_q_heads, num_kv_heads, group;
+  int max_blocks_per_seq, num_blocks;
+  int part_tokens;   // tokens per work item (a multiple of 16)
+  int max_parts;     // P: partitions per sequence in the workspace
+  int max_context_len;
+  int final_pass;    // 1: one item covers the whole context, write out directly
+  pa_dtype q_dtype, out_dtype;
+};
+
+__device__ __forceinline__ float load_q(const void* q, pa_dtype t, int64_t i) {
+  return t == PA_F32 ? static_cast<const float*>(q)[i]
+                     : __uint_as_float((uint32_t) static_cast<const uint16_t*>(q)[i] << 16);
+}
+
+__device__ __forceinline__ void store_out(void* out, pa_dtype t, int64_t i, float x) {
+  if (t == PA_F32) static_cast<float*>(out)[i] = x;
+  else static_cast<uint16_t*>(out)[i] = (uint16_t)(pack_bf16x2(x, 0.f) & 0xffff);
+}
+
+// Clamp a device-side context length into [0, max_context_len]; flag anything outside.
+__device__ __forceinline__ int checked_ctx(const DecodeArgs& a, int s) {
+  int c = a.context_lens[s];
+  if (c < 0 || c > a.max_context_len) {
+    if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
+    c = c < 0 ? 0 : a.max_context_len;
+  }
+  return c;
+}
+
+// Writes the merged state of a work item: either out/lse (final) or the partial.
+// m2 is the log2-domain max, l the sum, acc[d] the unnormalised output of head h.
+__device__ __forceinline__ void emit(const DecodeArgs& a, int s, int h, int part, int D, int d,
+                                     float m2, float l, float acc) {
+  const int64_t row = (int64_t)s * a.num_q_heads + h;
+  if (a.final_pass) {
+    const float o = l > 0.f ? acc / l : 0.f;
+    store_out(a.out, a.out_dtype, row * D + d, o);
+    if (d == 0 && a.lse_out != nullptr)
+      a.lse_out[row] = l > 0.f ? (m2 + __log2f(l)) * kLn2 : -INFINITY;
+  } else {
+    const int64_t pr = row * a.max_parts + part;
+    a.part_acc[pr * D + d] = acc;
+    if (d == 0) { a.part_m[pr] = m2; a.part_l[pr] = l; }
+  }
+}
+
+template <pa_dtype KV, int D, int GP>
+__global__ void __launch_bounds__(kSimtWarps * 32)
+decode_simt_kernel(const DecodeArgs a) {
+  constexpr int ES = KvTraits<KV>::bytes;
+  constexpr int HALF = D / 2;               // channels per lane in the score phase
+  constexpr int EPC = 16 / ES;              // elements per 16-byte chunk
+  constexpr int CH = HALF / EPC;            // chunks per lane per token row
+  constexpr int NV = D / 32;                // channels per lane in the P.V phase
+  constexpr int QROW = D + 4;               // padded q row (floats); halves in different banks
+  constexpr int TILE = kBS * D * ES;        // bytes of one (block, head) tile
+
+  __shared__ __align__(16) float sq[GP * QROW];
+  __shared__ __align__(16) float sp[kSimtWarps][kBS][GP];
+  __shared__ float sm[kSimtWarps][GP], sl[kSimtWarps][GP];
+  __shared__ __align__(16) float sacc[kSimtWarps][GP][D];
+
+  const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
+  const int ctx = checked_ctx(a, s);
+  const int t0 = part * a.part_tokens;
+  if (!a.final_pass && t0 >= ctx) return;  // empty partition: nothing to write
+  const int t1 = min(ctx, t0 + a.part_tokens);
+  const int G = a.group;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // q of the group, pre-multiplied by scale*log2(e); rows >= G are zero.
+  for (int i = threadIdx.x; i < GP * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    float x = 0.f;
+    if (g < G) x = load_q(a.q, a.q_dtype, ((int64_t)s * a.num_q_heads + kvh * G + g) * D + d) *
+                   a.scale_log2;
+    sq[g * QROW + d + (d >= HALF ? 4 : 0)] = x;
+  }
+  __syncthreads();
+
+  float m[GP], lsum[GP], acc[GP][NV];
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    m[g] = -INFINITY; lsum[g] = 0.f;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) acc[g][j] = 0.f;
+  }
+
+  const int tok = lane & 15, half = lane >> 4;
+  const int b_begin = t0 / kBS, b_end = (t1 + kBS - 1) / kBS;
+  const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+  const uint8_t* kbase = static_cast<const uint8_t*>(a.k_cache);
+  const uint8_t* vbase = static_cast<const uint8_t*>(a.v_cache);
+
+  for (int b = b_begin + warp; b < b_end; b += kSimtWarps) {
+    int phys = bt[b];
+    if (phys < 0 || phys >= a.num_blocks) {
+      if (lane == 0) flag_error(PA_DEVERR_BLOCK_ID);
+      continue;
+    }
+    const int64_t tile = ((int64_t)phys * a.num_kv_heads + kvh) * TILE;
+    float ks = 1.f, vs = 1.f;
+    if constexpr (KV == PA_FP8_E4M3) {
+      ks = a.k_scales[(int64_t)phys * a.num_kv_heads + kvh];
+      vs = a.v_scales[(int64_t)phys * a.num_kv_heads + kvh];
+    }
+    // ---- scores: lane (tok, half) -> partial dot over its half of d ----
+    float sc[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) sc[g] = 0.f;
+    const uint4* krow = reinterpret_cast<const uint4*>(kbase + tile + (int64_t)tok * D * ES + half * HALF * ES);
+#pragma unroll
+    for (int c = 0; c < CH; ++c) {
+      float kx[EPC];
+      unpack16<KV>(__ldg(krow + c), kx);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float* qr = sq + g * QROW + half * (HALF + 4) + c * EPC;
+#pragma unroll
+        for (int e = 0; e < EPC; e += 4) {
+          float4 qv = *reinterpret_cast<const float4*>(qr + e);
+          sc[g] = fmaf(qv.x, kx[e], sc[g]);
+          sc[g] = fmaf(qv.y, kx[e + 1], sc[g]);
+          sc[g] = fmaf(qv.z, kx[e + 2], sc[g]);
+          sc[g] = fmaf(qv.w, kx[e + 3], sc[g]);
+        }
+      }
+    }
+    const int t = b * kBS + tok;
+    const bool valid = t >= t0 && t < t1;
+    float p[GP];
+#pragma unroll
+    for (int g = 0; g < GP; ++g) {
+      float z = sc[g] + __shfl_xor_sync(0xffffffffu, sc[g], 16);
+      z = valid ? z * ks : -INFINITY;
+      float bm = z;
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+      const float mn = fmaxf(m[g], bm);   // finite: the block holds a valid token
+      const float alpha = fast_exp2(m[g] - mn);
+      m[g] = mn;
+      p[g] = valid ? fast_exp2(z - mn) : 0.f;
+      lsum[g] = lsum[g] * alpha + (half == 0 ? p[g] : 0.f);
+#pragma unroll
+      for (int j = 0; j < NV; ++j) acc[g][j] *= alpha;
+    }
+    if (half == 0) {
+#pragma unroll
+      for (int g = 0; g < GP; ++g) sp[warp][tok][g] = p[g] * vs;
+    }
+    __syncwarp();
+    // ---- P.V: lane -> channels [lane*NV, lane*NV + NV) ----
+#pragma unroll 4
+    for (int tt = 0; tt < kBS; ++tt) {
+      float vx[NV];
+      load_vslice<KV, D>(vbase + tile + (int64_t)tt * D * ES, lane, vx);
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        const float pg = sp[warp][tt][g];
+#pragma unroll
+        for (int j = 0; j < NV; ++j) acc[g][j] = fmaf(pg, vx[j], acc[g][j]);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ---- merge the warps ----
+#pragma unroll
+  for (int g = 0; g < GP; ++g) {
+    float l = lsum[g];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+    if (lane == 0) { sm[warp][g] = m[g]; sl[warp][g] = l; }
+#pragma unroll
+    for (int j = 0; j < NV; ++j) sacc[warp][g][lane * NV + j] = acc[g][j];
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kSimtWarps; ++w) M = fmaxf(M, sm[w][g]);
+    float L = 0.f, A = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kSimtWarps; ++w) {
+        const float f = fast_exp2(sm[w][g] - M);
+        L = fmaf(f, sl[w][g], L);
+        A = fmaf(f, sacc[w][g][d], A);
+      }
+    }
+    emit(a, s, kvh * G + g, part, D, d, M, L, A);
+  }
+}
+
+// Log-sum-exp merge of the partitions of one (sequence, query head): grid (Hq, S).
+template <int D>
+__global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
+  const int h = blockIdx.x, s = blockIdx.y;
+  const int ctx = checked_ctx(a, s);
+  const int np = (ctx + a.part_tokens - 1) / a.part_tokens;
+  const int64_t row = (int64_t)s * a.num_q_heads + h;
+  const float* pm = a.part_m + row * a.max_parts;
+  const float* pl = a.part_l + row * a.max_parts;
+  const float* pa_ = a.part_acc + row * a.max_parts * D;
+  float M = -INFINITY;
+  for (int p = 0; p < np; ++p) M = fmaxf(M, pm[p]);
+  for (int d = threadIdx.x; d < D; d += blockDim.x) {
+    float L = 0.f, A = 0.f;
+    for (int p = 0; p < np; ++p) {
+      const float f = fast_exp2(pm[p] - M);
+      L = fmaf(f, pl[p], L);
+      A = fmaf(f, pa_[(int64_t)p * D + d], A);
+    }
+    store_out(a.out, a.out_dtype, row * D + d, L > 0.f ? A / L : 0.f);
+    if (d == 0 && a.lse_out != nullptr)
+      a.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+  }
+}
+
+}  // namespace pa

@@ -1,0 +1,261 @@
+// C-ABI entry points of libpagedattn.so: argument validation and kernel dispatch.
+// Declarations and contracts: include/pagedattn.h.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+
+#include "common.cuh"
+#include "cache_ops.cuh"
+#include "decode_simt.cuh"
+#include "decode_tc.cuh"
+
+namespace pa {
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WorkspaceLayout {
+  size_t m_off, l_off, acc_off, total;
+  int parts;
+};
+
+bool desc_ok(const pa_decode_desc* d) {
+  if (d == nullptr) return false;
+  if (d->num_seqs < 0 || d->num_seqs > 65535) return false;
+  if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_kv_heads > 65535) return false;
+  if (d->num_q_heads % d->num_kv_heads != 0) return false;
+  if (d->head_dim <= 0 || d->block_size <= 0 || d->num_blocks <= 0) return false;
+  if (d->max_blocks_per_seq <= 0 || d->partition_size < 0) return false;
+  if (d->partition_size % d->block_size != 0) return false;
+  return true;
+}
+
+bool desc_supported(const pa_decode_desc* d) {
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (d->block_size != kBS) return false;
+  if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return false;
+  if (G > 16 || G * d->head_dim > 2048) return false;
+  if (d->kv_dtype == PA_F32) return d->q_dtype == PA_F32 && d->out_dtype == PA_F32;
+  if (d->kv_dtype == PA_BF16 || d->kv_dtype == PA_FP8_E4M3)
+    return d->q_dtype == PA_BF16 && d->out_dtype == PA_BF16;
+  return false;
+}
+
+WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
+  WorkspaceLayout w{0, 0, 0, 0, 0};
+  if (d->partition_size == 0 || max_context_len <= 0) return w;
+  w.parts = (max_context_len + d->partition_size - 1) / d->partition_size;
+  const size_t rows = (size_t)d->num_seqs * d->num_q_heads * w.parts;
+  w.m_off = 0;
+  w.l_off = round_up(rows * sizeof(float), 256);
+  w.acc_off = w.l_off + round_up(rows * sizeof(float), 256);
+  w.total = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
+  return w;
+}
+
+int pad_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
+
+template <pa_dtype KV, int D, int GP>
+cudaError_t launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
+  if constexpr (GP * D <= 2048) {
+    decode_simt_kernel<KV, D, GP><<<grid, kSimtWarps * 32, 0, st>>>(a);
+    return cudaGetLastError();
+  } else {
+    return cudaErrorInvalidValue;
+  }
+}
+
+template <pa_dtype KV, int D>
+cudaError_t launch_simt_g(const DecodeArgs& a, int gp, dim3 grid, cudaStream_t st) {
+  switch (gp) {
+    case 1: return launch_simt<KV, D, 1>(a, grid, st);
+    case 2: return launch_simt<KV, D, 2>(a, grid, st);
+    case 4: return launch_simt<KV, D, 4>(a, grid, st);
+    case 8: return launch_simt<KV, D, 8>(a, grid, st);
+    default: return launch_simt<KV, D, 16>(a, grid, st);
+  }
+}
+
+template <pa_dtype KV>
+cudaError_t launch_simt_d(const DecodeArgs& a, int D, int gp, dim3 grid, cudaStream_t st) {
+  switch (D) {
+    case 64: return launch_simt_g<KV, 64>(a, gp, grid, st);
+    case 128: return launch_simt_g<KV, 128>(a, gp, grid, st);
+    default: return launch_simt_g<KV, 256>(a, gp, grid, st);
+  }
+}
+
+cudaError_t launch_reduce(const DecodeArgs& a, int D, cudaStream_t st) {
+  dim3 grid(a.num_q_heads, a.num_seqs);
+  switch (D) {
+    case 64: lse_reduce_kernel<64><<<grid, 128, 0, st>>>(a); break;
+    case 128: lse_reduce_kernel<128><<<grid, 128, 0, st>>>(a); break;
+    default: lse_reduce_kernel<256><<<grid, 128, 0, st>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char* pa_version(void) { return "pagedattn 0.1 sm_100a"; }
+
+pa_status pa_set_decode_impl(int impl) {
+  if (impl < 0 || impl > 2) return PA_ERR_INVALID;
+  g_decode_impl = impl;
+  return PA_OK;
+}
+
+size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len) {
+  if (!desc_ok(desc) || max_context_len < 0) return 0;
+  return layout_for(desc, max_context_len).total;
+}
+
+pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_tables, const int32_t* context_lens,
+                            float scale, void* out, const pa_decode_desc* desc,
+                            int max_context_len, const float* k_scales, const float* v_scales,
+                            float* lse_out, void* workspace, size_t workspace_bytes,
+                            void* stream) {
+  if (!desc_ok(desc) || max_context_len < 0 || !std::isfinite(scale)) return PA_ERR_INVALID;
+  if (!desc_supported(desc)) return PA_ERR_UNSUPPORTED;
+  if (desc->num_seqs == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out))
+    return PA_ERR_INVALID;
+  if ((int64_t)desc->max_blocks_per_seq * desc->block_size < (int64_t)max_context_len)
+    return PA_ERR_INVALID;
+  const bool fp8 = desc->kv_dtype == PA_FP8_E4M3;
+  if (fp8 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  const WorkspaceLayout wl = layout_for(desc, max_context_len);
+  if (wl.total > 0 && (workspace == nullptr || workspace_bytes < wl.total || !aligned16(workspace)))
+    return PA_ERR_WORKSPACE;
+
+  DecodeArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+  a.block_tables = block_tables; a.context_lens = context_lens;
+  a.out = out; a.lse_out = lse_out; a.k_scales = k_scales; a.v_scales = v_scales;
+  a.scale_log2 = scale * kLog2e;
+  a.num_seqs = desc->num_seqs; a.num_q_heads = desc->num_q_heads;
+  a.num_kv_heads = desc->num_kv_heads; a.group = desc->num_q_heads / desc->num_kv_heads;
+  a.max_blocks_per_seq = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
+  a.max_context_len = max_context_len;
+  a.q_dtype = desc->q_dtype; a.out_dtype = desc->out_dtype;
+  const bool split = wl.total > 0;
+  if (split) {
+    char* ws = static_cast<char*>(workspace);
+    a.part_m = reinterpret_cast<float*>(ws + wl.m_off);
+    a.part_l = reinterpret_cast<float*>(ws + wl.l_off);
+    a.part_acc = reinterpret_cast<float*>(ws + wl.acc_off);
+    a.part_tokens = desc->partition_size;
+    a.max_parts = wl.parts;
+    a.final_pass = 0;
+  } else {
+    a.part_tokens = (int)round_up((size_t)(max_context_len > 0 ? max_context_len : 1), kBS);
+    a.max_parts = 1;
+    a.final_pass = 1;
+  }
+  const cudaStream_t st = as_stream(stream);
+  const dim3 grid(split ? wl.parts : 1, desc->num_kv_heads, desc->num_seqs);
+  const int D = desc->head_dim;
+  const int gp = pad_group(a.group);
+  cudaError_t e;
+  if (g_decode_impl != 1 && tc_supported(desc)) {
+    e = launch_tc(a, desc, grid, st);
+  } else {
+    switch (desc->kv_dtype) {
+      case PA_F32: e = launch_simt_d<PA_F32>(a, D, gp, grid, st); break;
+      case PA_BF16: e = launch_simt_d<PA_BF16>(a, D, gp, grid, st); break;
+      default: e = launch_simt_d<PA_FP8_E4M3>(a, D, gp, grid, st); break;
+    }
+  }
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  if (split && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
+  return PA_OK;
+}
+
+pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
+                            const int64_t* slot_mapping, int num_tokens, int64_t k_stride,
+                            int64_t v_stride, int num_kv_heads, int head_dim, int block_size,
+                            int num_blocks, pa_dtype in_dtype, pa_dtype cache_dtype,
+                            const float* k_scales, const float* v_scales, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
+      block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (in_dtype != PA_F32 && in_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+  if (cache_dtype == PA_F32 && in_dtype != PA_F32) return PA_ERR_UNSUPPORTED;
+  if (num_tokens == 0) return PA_OK;
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return PA_ERR_INVALID;
+  const int64_t row = (int64_t)num_kv_heads * head_dim;
+  if (k_stride < row || v_stride < row) return PA_ERR_INVALID;
+  // 16-byte vector loads of 8 input elements
+  const int64_t align_elems = in_dtype == PA_F32 ? 4 : 8;
+  if (k_stride % align_elems || v_stride % align_elems || !aligned16(k) || !aligned16(v) ||
+      !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  if (cache_dtype == PA_FP8_E4M3 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  const cudaStream_t st = as_stream(stream);
+  const dim3 grid(num_tokens);
+  const int threads = 128;
+#define PA_RC(IN, C)                                                                         \
+  reshape_and_cache_kernel<IN, C><<<grid, threads, 0, st>>>(k, v, k_cache, v_cache,           \
+                                                            slot_mapping, k_stride, v_stride, \
+                                                            num_kv_heads, head_dim,           \
+                                                            block_size, num_blocks, k_scales, \
+                                                            v_scales)
+  if (in_dtype == PA_F32) {
+    if (cache_dtype == PA_F32) PA_RC(PA_F32, PA_F32);
+    else if (cache_dtype == PA_BF16) PA_RC(PA_F32, PA_BF16);
+    else if (cache_dtype == PA_FP8_E4M3) PA_RC(PA_F32, PA_FP8_E4M3);
+    else return PA_ERR_UNSUPPORTED;
+  } else {
+    if (cache_dtype == PA_BF16) PA_RC(PA_BF16, PA_BF16);
+    else if (cache_dtype == PA_FP8_E4M3) PA_RC(PA_BF16, PA_FP8_E4M3);
+    else return PA_ERR_UNSUPPORTED;
+  }
+#undef PA_RC
+  PA_CHECK_LAUNCH();
+  return PA_OK;
+}
+
+pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_scales,
+                      const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
+                      int block_size, int num_blocks, pa_dtype cache_dtype, void* stream) {
+  if (num_pairs < 0 || num_pairs > 65535 * 1024 || num_kv_heads <= 0 || head_dim <= 0 ||
+      block_size <= 0 || num_blocks <= 0)
+    return PA_ERR_INVALID;
+  if (cache_dtype != PA_F32 && cache_dtype != PA_BF16 && cache_dtype != PA_FP8_E4M3)
+    return PA_ERR_UNSUPPORTED;
+  if (num_pairs == 0) return PA_OK;
+  if (!k_cache || !v_cache || !pairs || !aligned16(k_cache) || !aligned16(v_cache))
+    return PA_ERR_INVALID;
+  const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * dtype_bytes(cache_dtype);
+  if (block_bytes % 16 != 0) return PA_ERR_INVALID;
+  if (cache_dtype == PA_FP8_E4M3 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  copy_blocks_kernel<<<dim3(num_pairs, 2), 256, 0, as_stream(stream)>>>(
+      static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
+      cache_dtype == PA_FP8_E4M3 ? k_scales : nullptr,
+      cache_dtype == PA_FP8_E4M3 ? v_scales : nullptr, pairs, block_bytes, num_kv_heads,
+      num_blocks);
+  PA_CHECK_LAUNCH();
+  return PA_OK;
+}
+
+pa_status pa_device_error(int* bits_out, void* stream) {
+  if (bits_out == nullptr) return PA_ERR_INVALID;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return PA_ERR_CUDA;
+  unsigned int w = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&w, g_error_word, sizeof(w)) != cudaSuccess) return PA_ERR_CUDA;
+  if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero)) != cudaSuccess) return PA_ERR_CUDA;
+  *bits_out = (int)w;
+  return w == 0 ? PA_OK : PA_ERR_DEVICE;
+}
+
+}  // extern "C"

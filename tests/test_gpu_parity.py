@@ -1,0 +1,294 @@
+"""GPU parity of the CUDA path against the oracle, through the C ABI (the Python binding).
+
+Bit-exact: slot-mapped cache writes, block copies, cache contents after a whole workload.
+Within the per-dtype tolerances of tests/gpu_common.py: decode outputs and lse, on the five
+workloads (full size; the two largest on sampled sequences, in the launch configuration the
+bench times), on both kernel families, on edge cases and needle variants. Bit-identical:
+outputs under a different physical placement of the same logical KV, and shared-prefix
+sequences against private unshared copies.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import workloads
+from oracle import flows, paged as opaged, codecs
+from tests.gpu_common import TOL, compare_decode, cache_codes, to_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import paged_kv_cache_465_b200 as pa
+    pa.set_decode_impl("auto")
+    yield pa
+    pa.set_decode_impl("auto")
+
+
+@pytest.fixture(scope="module")
+def scen():
+    from paged_kv_cache_465_b200.scenario import DeviceScenario
+    return DeviceScenario
+
+
+def _bf16_dev(x):
+    return torch.from_numpy(np.ascontiguousarray(x)).view(torch.int16).view(torch.bfloat16).cuda()
+
+
+# ---------------------------------------------------------------------------------------
+# cache write and block copy: bit-exact
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("in_dt,cache_dt,d", [("f32", "f32", 64), ("f32", "bf16", 128),
+                                              ("bf16", "bf16", 128), ("bf16", "fp8", 128),
+                                              ("f32", "fp8", 64), ("bf16", "bf16", 256)])
+def test_reshape_and_cache_bitexact(pa, in_dt, cache_dt, d):
+    rng = np.random.default_rng(hash((in_dt, cache_dt, d)) % 2 ** 32)
+    NB, H, B, T = 40, 4, 16, 300
+    xf = (rng.standard_normal((T, H, d)) * rng.choice([1e-3, 1, 30, 700], (T, H, 1))).astype(np.float32)
+    xin = xf if in_dt == "f32" else codecs.bf16_encode(xf)
+    slots = rng.permutation(NB * B)[:T].astype(np.int64)
+    slots[::17] = -1
+    ks = rng.uniform(0.01, 2.0, (NB, H)).astype(np.float32)
+    vs = rng.uniform(0.01, 2.0, (NB, H)).astype(np.float32)
+    kref = opaged.new_cache(NB, H, B, d, cache_dt)
+    vref = opaged.new_cache(NB, H, B, d, cache_dt)
+    opaged.ref_reshape_and_cache(xin, xin[::-1].copy(), kref, vref, slots, in_dt, cache_dt, ks, vs)
+    # device inputs: rows strided along T (a wider row buffer) to exercise k_stride
+    tdt = torch.float32 if in_dt == "f32" else torch.bfloat16
+    pad = 8
+    wide = torch.zeros((T, H * d + pad), dtype=tdt)
+    src = torch.from_numpy(xin) if in_dt == "f32" else torch.from_numpy(xin).view(torch.int16).view(torch.bfloat16)
+    wide[:, :H * d] = src.reshape(T, H * d)
+    k = wide.cuda()[:, :H * d].view(T, H, d)
+    v = src.flip(0).contiguous().cuda()
+    cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}[cache_dt]
+    kc = torch.zeros((NB, H, B, d), dtype=cdt, device="cuda")
+    vc = torch.zeros_like(kc)
+    sc = dict(k_scales=torch.from_numpy(ks).cuda(), v_scales=torch.from_numpy(vs).cuda()) \
+        if cache_dt == "fp8" else {}
+    pa.reshape_and_cache(k, v, kc, vc, torch.from_numpy(slots).cuda(), **sc)
+    assert pa.device_error() == 0
+    assert np.array_equal(cache_codes(kc), kref)
+    assert np.array_equal(cache_codes(vc), vref)
+
+
+@pytest.mark.parametrize("cache_dt", ["f32", "bf16", "fp8"])
+def test_copy_blocks_bitexact(pa, cache_dt):
+    rng = np.random.default_rng(5)
+    NB, H, B, d = 64, 8, 16, 128
+    store = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}[cache_dt]
+    if cache_dt == "f32":
+        k0 = rng.standard_normal((NB, H, B, d)).astype(np.float32)
+        v0 = rng.standard_normal((NB, H, B, d)).astype(np.float32)
+    else:
+        hi = 2 ** 16 if cache_dt == "bf16" else 256
+        k0 = rng.integers(0, hi, (NB, H, B, d)).astype(store)
+        v0 = rng.integers(0, hi, (NB, H, B, d)).astype(store)
+    ks0 = rng.uniform(size=(NB, H)).astype(np.float32)
+    vs0 = rng.uniform(size=(NB, H)).astype(np.float32)
+    srcs = rng.choice(NB, 20, replace=False)
+    dsts = rng.choice(np.setdiff1d(np.arange(NB), srcs), 20, replace=False)
+    pairs = [(int(s), int(t)) for s, t in zip(srcs, dsts)]
+    kr, vr, ksr, vsr = k0.copy(), v0.copy(), ks0.copy(), vs0.copy()
+    opaged.ref_copy_blocks(kr, vr, pairs, ksr if cache_dt == "fp8" else None,
+                           vsr if cache_dt == "fp8" else None)
+
+    def dev(x):
+        t = torch.from_numpy(x)
+        if cache_dt == "bf16":
+            t = t.view(torch.int16).view(torch.bfloat16)
+        return t.cuda()
+    kc, vc = dev(k0), dev(v0)
+    ksd, vsd = torch.from_numpy(ks0).cuda(), torch.from_numpy(vs0).cuda()
+    pa.copy_blocks(kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
+                   k_scales=ksd if cache_dt == "fp8" else None,
+                   v_scales=vsd if cache_dt == "fp8" else None)
+    assert pa.device_error() == 0
+    assert np.array_equal(cache_codes(kc), kr) and np.array_equal(cache_codes(vc), vr)
+    assert np.array_equal(ksd.cpu().numpy(), ksr) and np.array_equal(vsd.cpu().numpy(), vsr)
+
+
+# ---------------------------------------------------------------------------------------
+# whole workloads
+# ---------------------------------------------------------------------------------------
+def _run_and_compare(pa, scen, draw, impl="auto", draw_seqs=None, partition_size=None,
+                     check_cache=True, shared=True):
+    pa.set_decode_impl(impl)
+    try:
+        sc = scen(draw, draw_seqs=draw_seqs, partition_size=partition_size, shared=shared)
+        sc.step()
+        torch.cuda.synchronize()
+        assert pa.device_error() == 0
+        st = flows.build_state(draw, write_seqs=draw_seqs, shared=shared)
+        seqs = sorted(sc.draw_seqs)
+        out_ref, lse_ref = flows.ref_outputs(draw, st, seqs=seqs)
+        stats = compare_decode(sc.out, sc.lse, out_ref, lse_ref, draw.wl.kv_dtype, seqs=seqs)
+        if check_cache:
+            assert np.array_equal(sc.block_tables.cpu().numpy(), st.block_tables)
+            assert np.array_equal(cache_codes(sc.cache.k_cache), st.k_cache)
+            assert np.array_equal(cache_codes(sc.cache.v_cache), st.v_cache)
+        return sc, stats
+    finally:
+        pa.set_decode_impl("auto")
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+def test_tiny_workload(pa, scen, impl):
+    d = workloads.draw("tiny")
+    _run_and_compare(pa, scen, d, impl)
+    # the four decode tokens land at offsets 4, 15, 0 (a new block) and 7
+    sc = scen(d)
+    offs = (sc.step_slots.cpu().numpy() % 16).tolist()
+    assert offs == [4, 15, 0, 7]
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("part", [0, 512])
+def test_batch32_workload(pa, scen, impl, part):
+    _run_and_compare(pa, scen, workloads.draw("b32"), impl, partition_size=part)
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+def test_shared_prefix_workload(pa, scen, impl):
+    d = workloads.draw("shared")
+    sc, _ = _run_and_compare(pa, scen, d, impl)
+    assert len(sc.cow_pairs) == 99
+    assert sc.cache.num_blocks - sc.cache.alloc.num_free() == 412
+    # shared-prefix sequences == private unshared copies, bit for bit
+    pa.set_decode_impl(impl)
+    try:
+        un = scen(d, shared=False)
+        un.step()
+        torch.cuda.synchronize()
+        assert torch.equal(un.out, sc.out) and torch.equal(un.lse, sc.lse)
+    finally:
+        pa.set_decode_impl("auto")
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("part", [512, 0])
+def test_batch256_fp8_full_size_sampled(pa, scen, impl, part):
+    d = workloads.draw("b256")
+    lens = d.context_lens
+    sample = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 7, 100, 200, 255})
+    _run_and_compare(pa, scen, d, impl, draw_seqs=sample, partition_size=part, check_cache=False)
+
+
+def test_long_context_full_size_sampled(pa, scen):
+    d = workloads.draw("long")
+    _run_and_compare(pa, scen, d, "auto", draw_seqs=[5], check_cache=False)
+
+
+# ---------------------------------------------------------------------------------------
+# invariances, needles, closed forms, edge cases
+# ---------------------------------------------------------------------------------------
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512)])
+def test_physical_placement_bit_identical(pa, scen, impl, name, part):
+    wl = workloads.WORKLOADS[name].scaled(num_seqs=6)
+    pa.set_decode_impl(impl)
+    try:
+        d1 = workloads.draw(wl)
+        s1 = scen(d1, partition_size=part)
+        s1.step()
+        d2 = workloads.draw(wl)
+        d2.pool_order = np.roll(d2.pool_order[::-1], 7).copy()
+        s2 = scen(d2, partition_size=part)
+        s2.step()
+        torch.cuda.synchronize()
+        assert not torch.equal(s1.block_tables, s2.block_tables)
+        assert torch.equal(s1.out, s2.out) and torch.equal(s1.lse, s2.lse)
+    finally:
+        pa.set_decode_impl("auto")
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("name,part,lens", [
+    ("b32", 0, [1, 2, 15, 16, 17, 31, 33, 4096]),
+    ("b32", 512, [511, 512, 513, 1024, 1025, 3000]),
+    ("b256", 512, [16, 17, 500, 512, 2049, 8192]),
+    ("b256", 0, [1, 16, 100, 8192]),
+    ("long", 512, [20000, 513]),
+])
+def test_ragged_lengths_and_needles(pa, scen, impl, name, part, lens):
+    wl = workloads.WORKLOADS[name].scaled(num_seqs=len(lens))
+    for needle in (False, True):
+        d = workloads.draw(wl, lens_override=lens, needle=needle)
+        _run_and_compare(pa, scen, d, impl, partition_size=part)
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+def test_zero_query_is_mean_of_values(pa, scen, impl):
+    wl = workloads.WORKLOADS["b32"].scaled(num_seqs=3)
+    d = workloads.draw(wl, q_zero=True, lens_override=[5, 300, 1000])
+    sc, _ = _run_and_compare(pa, scen, d, impl)
+    out = to_f64(sc.out)
+    for s in range(3):
+        k, v = d.kv(s)
+        vm = codecs.bf16_decode(v).mean(axis=0)      # [Hkv, d]
+        G = wl.group
+        for h in range(wl.num_q_heads):
+            assert np.abs(out[s, h] - vm[h // G]).max() < TOL["bf16"]["max_abs"]
+        assert np.allclose(to_f64(sc.lse)[s], math.log(d.context_lens[s]), atol=1e-3)
+
+
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("hq,hkv,dim,kv", [(8, 8, 128, "bf16"), (16, 8, 128, "bf16"),
+                                            (64, 4, 128, "bf16"), (16, 2, 64, "bf16"),
+                                            (8, 1, 256, "bf16"), (32, 8, 128, "fp8"),
+                                            (64, 8, 128, "fp8"), (8, 2, 128, "f32"),
+                                            (6, 2, 128, "bf16")])
+def test_head_shapes(pa, scen, impl, hq, hkv, dim, kv):
+    in_dt = "f32" if kv == "f32" else "bf16"
+    wl = workloads.Workload("shape", 9, 5, hq, hkv, dim, 16, 512, kv, in_dt,
+                            ("fixed", [1, 17, 100, 700, 1500]))
+    for part in (0, 256):
+        _run_and_compare(pa, scen, workloads.draw(wl), impl, partition_size=part)
+
+
+def test_empty_context_and_error_flags(pa):
+    S, Hq, Hkv, d, NB = 3, 8, 2, 128, 16
+    q = torch.randn(S, Hq, d, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(NB, Hkv, 16, d, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(NB, Hkv, 16, d, device="cuda").to(torch.bfloat16)
+    bt = torch.tensor([[0, 1], [2, -1], [3, 4]], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    lse = torch.empty(S, Hq, device="cuda")
+    assert pa.device_error() == 0
+    for part in (0, 16):
+        ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+        pa.paged_attn_decode(q, kc, vc, bt, torch.tensor([0, 5, 0], dtype=torch.int32,
+                                                         device="cuda"),
+                             0.1, out, max_context_len=32, partition_size=part, lse_out=lse,
+                             workspace=ws)
+        torch.cuda.synchronize()
+        assert pa.device_error() == 0
+        assert torch.all(out[0] == 0) and torch.all(out[2] == 0)
+        assert torch.all(torch.isneginf(lse[0])) and torch.all(torch.isfinite(lse[1]))
+    # an out-of-range block id is skipped and flagged, never dereferenced
+    bad = torch.tensor([[0, 1_000_000], [2, -1], [3, 4]], dtype=torch.int32, device="cuda")
+    pa.paged_attn_decode(q, kc, vc, bad, torch.tensor([20, 5, 30], dtype=torch.int32,
+                                                      device="cuda"),
+                         0.1, out, max_context_len=32)
+    assert pa.device_error() & pa.PA_DEVERR_BLOCK_ID
+    assert pa.device_error() == 0
+    # a context longer than max_context_len is clamped and flagged
+    pa.paged_attn_decode(q, kc, vc, bt, torch.tensor([20, 5, 40], dtype=torch.int32,
+                                                     device="cuda"),
+                         0.1, out, max_context_len=32)
+    assert pa.device_error() & pa.PA_DEVERR_CONTEXT
+    # a slot past the pool and a copy pair past the pool are skipped and flagged
+    k1 = torch.randn(2, Hkv, d, device="cuda").to(torch.bfloat16)
+    before = kc.clone()
+    pa.reshape_and_cache(k1, k1, kc, vc, torch.tensor([5, NB * 16 + 3], dtype=torch.int64,
+                                                      device="cuda"))
+    assert pa.device_error() & pa.PA_DEVERR_SLOT
+    assert torch.equal(kc[1:], before[1:]) and torch.equal(kc[0, :, 6:], before[0, :, 6:])
+    pa.copy_blocks(kc, vc, torch.tensor([[0, NB]], dtype=torch.int32, device="cuda"))
+    assert pa.device_error() & pa.PA_DEVERR_PAIR

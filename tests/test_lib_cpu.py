@@ -1,0 +1,182 @@
+"""CPU checks of the native library: it builds, loads and exports every symbol the header
+declares; its host allocator matches the oracle's allocator state bit for bit on random
+traces and on the shared-prefix example; host-side validation rejects bad calls before any
+device work (none of these calls touches a GPU)."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def pa():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_pa_build", os.path.join(ROOT, "paged_kv_cache_465_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import paged_kv_cache_465_b200 as pa
+    return pa
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w\s\*]*?\b(\w+)\s*\([^;]*\)\s*;", src, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "while", "return")))
+
+
+def test_exports_every_declared_symbol(pa):
+    names = _declared_functions()
+    assert "paged_attn_decode" in names and "pa_alloc_append" in names
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+    assert pa.version().startswith("pagedattn")
+
+
+def _state(a):
+    return a.free_queue(), [a.ref_count(b) for b in range(a.num_blocks)]
+
+
+def test_allocator_matches_oracle_random_traces(pa):
+    from oracle.paged import RefAllocator, NoBlocks as RefNoBlocks, InvalidCall
+    rng = np.random.default_rng(123)
+    for trial in range(25):
+        nb = int(rng.integers(4, 300))
+        order = rng.permutation(nb) if trial % 2 else None
+        ref = RefAllocator(nb, 16, order=order)
+        nat = pa.BlockAllocator(nb, 16, order=order)
+        live, nxt = [], 0
+        for step in range(400):
+            op = int(rng.integers(0, 5))
+            args = None
+            if op == 0 or not live:
+                args = ("add_seq", nxt, int(rng.integers(0, 120)))
+            elif op == 1:
+                args = ("fork", live[int(rng.integers(len(live)))], nxt)
+            elif op in (2, 3):
+                args = ("append", live[int(rng.integers(len(live)))], int(rng.integers(0, 50)))
+            else:
+                args = ("free_seq", live[int(rng.integers(len(live)))])
+            r_exc = n_exc = None
+            try:
+                r_res = getattr(ref, args[0])(*args[1:])
+            except (RefNoBlocks, InvalidCall) as e:
+                r_exc = type(e).__name__
+            try:
+                n_res = getattr(nat, args[0])(*args[1:])
+            except pa.NoBlocks:
+                n_exc = "NoBlocks"
+            except pa.PagedAttnError:
+                n_exc = "InvalidCall"
+            assert r_exc == n_exc, (args, r_exc, n_exc)
+            if r_exc is None:
+                if args[0] in ("add_seq", "fork"):
+                    live.append(args[1] if args[0] == "add_seq" else args[2])
+                    nxt += 1
+                if args[0] == "free_seq":
+                    live.remove(args[1])
+                if args[0] == "add_seq":
+                    assert np.array_equal(r_res, n_res)
+                if args[0] == "append":
+                    assert np.array_equal(r_res[0], n_res[0]) and list(r_res[1]) == n_res[1]
+            assert _state(nat) == (list(ref.free), ref.refs)
+            for s in live:
+                assert nat.block_table(s) == ref.block_table(s)
+                assert nat.seq_len(s) == ref.seq_len(s)
+
+
+def test_allocator_shared_prefix_example(pa):
+    a = pa.BlockAllocator(512, 16)
+    a.add_seq(0, 200)
+    for c in range(1, 100):
+        a.fork(0, c)
+    prefix = a.block_table(0)
+    pairs = []
+    for s in range(100):
+        pairs += a.append(s, 50)[1]
+    assert len(pairs) == 99 and all(p[0] == prefix[-1] for p in pairs)
+    assert [a.ref_count(b) for b in prefix[:12]] == [100] * 12
+    assert a.ref_count(prefix[-1]) == 1
+    assert 512 - a.num_free() == 412
+
+
+def test_allocator_rejects_and_stays_unchanged(pa):
+    a = pa.BlockAllocator(4, 16)
+    a.add_seq(0, 40)
+    before = _state(a)
+    with pytest.raises(pa.NoBlocks):
+        a.add_seq(1, 17)
+    with pytest.raises(pa.NoBlocks):
+        a.append(0, 30)
+    with pytest.raises(pa.PagedAttnError):
+        a.add_seq(0, 1)
+    with pytest.raises(pa.PagedAttnError):
+        a.fork(7, 8)
+    assert _state(a) == before
+    with pytest.raises(ValueError):
+        pa.BlockAllocator(3, 16, order=[0, 0, 1])
+
+
+def test_host_validation_without_device(pa):
+    lib = pa._lib
+    d = pa.make_desc(4, 4, 2, 64, 3, 32, 0, pa.PA_F32, pa.PA_F32, pa.PA_F32)
+    assert pa.workspace_size(d, 40) == 0
+    d2 = pa.make_desc(4, 4, 2, 64, 3, 32, 16, pa.PA_F32, pa.PA_F32, pa.PA_F32)
+    assert pa.workspace_size(d2, 40) > 0
+    nul = ctypes.c_void_p(0)
+    bad = [
+        pa.make_desc(4, 5, 2, 64, 3, 32, 0, pa.PA_F32, pa.PA_F32, pa.PA_F32),   # Hq % Hkv
+        pa.make_desc(4, 4, 2, 64, 3, 32, 8, pa.PA_F32, pa.PA_F32, pa.PA_F32),   # partition % 16
+        pa.make_desc(-1, 4, 2, 64, 3, 32, 0, pa.PA_F32, pa.PA_F32, pa.PA_F32),
+    ]
+    for b in bad:
+        st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
+                                   ctypes.byref(b), 40, nul, nul, nul, nul, 0, nul)
+        assert st == pa.PA_ERR_INVALID
+    uns = pa.make_desc(4, 4, 2, 96, 3, 32, 0, pa.PA_F32, pa.PA_F32, pa.PA_F32)    # head_dim 96
+    st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
+                               ctypes.byref(uns), 40, nul, nul, nul, nul, 0, nul)
+    assert st == pa.PA_ERR_UNSUPPORTED
+    mixed = pa.make_desc(4, 4, 2, 64, 3, 32, 0, pa.PA_F32, pa.PA_BF16, pa.PA_F32)
+    st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
+                               ctypes.byref(mixed), 40, nul, nul, nul, nul, 0, nul)
+    assert st == pa.PA_ERR_UNSUPPORTED
+    # null pointers with a valid descriptor are rejected before any launch
+    st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
+                               ctypes.byref(d), 40, nul, nul, nul, nul, 0, nul)
+    assert st == pa.PA_ERR_INVALID
+    # split path without workspace
+    st = lib.paged_attn_decode(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256),
+                               ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_float(0.1),
+                               ctypes.c_void_p(256), ctypes.byref(d2), 40, nul, nul, nul, nul,
+                               0, nul)
+    assert st == pa.PA_ERR_WORKSPACE
+    # zero-sized work is a successful no-op
+    assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 0, 128, 128, 2, 64, 16, 32,
+                                 pa.PA_F32, pa.PA_F32, nul, nul, nul) == pa.PA_OK
+    assert lib.copy_blocks(nul, nul, nul, nul, nul, 0, 2, 64, 16, 32, pa.PA_BF16, nul) == pa.PA_OK
+    assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 3, 128, 128, 2, 60, 16, 32,
+                                 pa.PA_F32, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_INVALID
+    assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 3, 128, 128, 2, 64, 16, 32,
+                                 pa.PA_BF16, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_UNSUPPORTED
+    assert lib.pa_set_decode_impl(3) == pa.PA_ERR_INVALID
+
+
+def test_binding_refuses_host_tensors(pa):
+    import torch
+    q = torch.zeros(4, 4, 64)
+    kc = torch.zeros(32, 2, 16, 64)
+    with pytest.raises(ValueError):
+        pa.paged_attn_decode(q, kc, kc, torch.zeros(4, 3, dtype=torch.int32),
+                             torch.zeros(4, dtype=torch.int32), 0.125, q.clone(), max_context_len=40)
