@@ -252,8 +252,10 @@ decode_simt_kernel(const DecodeArgs a) {
     }
     __syncwarp();
     // ---- P.V: lane -> channels [lane*NV, lane*NV + NV) ----
+    // tokens past the context are skipped: their slots may hold anything (even NaN)
+    const int nv = min(kBS, t1 - b * kBS);
 #pragma unroll 4
-    for (int tt = 0; tt < kBS; ++tt) {
+    for (int tt = 0; tt < nv; ++tt) {
       float vx[NV];
       load_vslice<KV, D>(vbase + tile + (int64_t)tt * D * ES, lane, vx);
 #pragma unroll
