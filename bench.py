@@ -218,6 +218,22 @@ def _cpu_baseline(draw, seconds: float = 12.0):
                       f"{el:.1f} s"}
 
 
+def slowest_rank_seconds(seconds: float, dist=None, device="cpu") -> float:
+    """Device time of the slowest rank (max over ranks); identity without a process group.
+    Every rank must call it the same number of times."""
+    if dist is None:
+        return float(seconds)
+    import torch
+    t = torch.tensor([float(seconds)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(bytes_per_rank_step: int, steps: int, world: int, slowest_s: float) -> float:
+    """Whole-job GB/s: every rank's bytes over the slowest rank's time (weak scaling)."""
+    return world * bytes_per_rank_step * steps / slowest_s / 1e9
+
+
 def run_ours(args):
     import torch
     from paged_kv_cache_465_b200.scenario import DeviceScenario
@@ -255,24 +271,19 @@ def run_ours(args):
         t_wall0 = time.time()
         total, dec_mean = _time_steps(torch, sc, args.steps, flush)
         t_wall1 = time.time()
+    total = slowest_rank_seconds(total, dist, "cuda")
     if dist is not None:
-        t = torch.tensor([total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
         dist.barrier()
     torch.cuda.synchronize()
     ms = total / args.steps * 1e3
     b = sc.step_bytes()
     peak, peak_kind = _peaks()
-    kv_gbs = world * b["kv"] * args.steps / total / 1e9
+    kv_gbs = job_throughput(b["kv"], args.steps, world, total)
     # e2e through the public API from host buffers
     e2e_total, h2d, d2h = _e2e(torch, sc, max(args.steps // 4, 3), flush)
-    if dist is not None:
-        t = torch.tensor([e2e_total], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_total = float(t.item())
+    e2e_total = slowest_rank_seconds(e2e_total, dist, "cuda")
     e2e_steps = max(args.steps // 4, 3)
-    e2e_gbs = world * b["kv"] * e2e_steps / e2e_total / 1e9
+    e2e_gbs = job_throughput(b["kv"], e2e_steps, world, e2e_total)
     # roofline of the dominant operation: paged_attn_decode (main kernel + LSE reduce)
     dec_achieved = b["decode"] / dec_mean / 1e9
     result = {

@@ -165,11 +165,14 @@ pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_sc
 pa_status pa_device_error(int* bits_out, void* stream);
 
 /*
- * Selects the decode kernel family used by later paged_attn_decode calls in this process:
+ * Selects the decode kernels used by later paged_attn_decode calls in this process:
  * 0 = automatic (tensor cores for bf16 / fp8 caches where the shape is supported, else the
- * CUDA-core fp32 path), 1 = CUDA-core path only, 2 = same as 0 (tensor cores where
- * supported). Both families compute the same function; they differ in how q.K and P.V are
- * multiplied. Returns PA_ERR_INVALID for any other value. Not thread-safe.
+ * CUDA-core fp32 path), 1 = CUDA-core path only, 2 = same as 0, 3 / 4 / 5 = tensor cores
+ * with a fixed kernel where the call allows it: 3 one CTA per work item, 4 persistent CTAs
+ * that share each work item (split path, partitions <= 2048 tokens), 5 persistent warp
+ * workers, one work item per warp (split path, partitions <= 512 tokens). All compute the
+ * same function; they differ in how work is scheduled and how q.K and P.V are multiplied.
+ * Returns PA_ERR_INVALID for any other value. Not thread-safe.
  */
 pa_status pa_set_decode_impl(int impl);
 

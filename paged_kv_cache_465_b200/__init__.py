@@ -135,10 +135,15 @@ def _stream(stream) -> ctypes.c_void_p:
     return ctypes.c_void_p(s.cuda_stream)
 
 
+DECODE_IMPLS = {"auto": 0, "simt": 1, "tc": 2, "tc-grid": 3, "tc-cta": 4, "tc-warps": 5}
+
+
 def set_decode_impl(impl: str = "auto") -> None:
-    """Chooses the decode kernel family: "auto" (tensor cores where supported), "simt"
-    (CUDA-core fp32 path everywhere) or "tc" (tensor cores where supported)."""
-    code = {"auto": 0, "simt": 1, "tc": 2}[impl]
+    """Chooses the decode kernels: "auto" (tensor cores where supported), "simt" (CUDA-core
+    fp32 path everywhere), "tc" (tensor cores, automatic kernel), or a fixed tensor-core
+    kernel: "tc-grid" (one CTA per work item), "tc-cta" (persistent CTAs), "tc-warps"
+    (persistent warp workers) where the call allows it."""
+    code = DECODE_IMPLS[impl]
     _check(_lib.pa_set_decode_impl(code), "pa_set_decode_impl")
 
 

@@ -104,6 +104,7 @@ struct DecodeArgs {
   int max_parts;     // P: partitions per sequence in the workspace
   int max_context_len;
   int final_pass;    // 1: one item covers the whole context, write out directly
+  int skip_single;   // split path: single-partition sequences were written directly
   pa_dtype q_dtype, out_dtype;
 };
 
@@ -297,27 +298,75 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, query head): grid (Hq, S).
+// Log-sum-exp merge of the partitions of one (sequence, query head): grid (Hq, S), 128
+// threads. Pass 1: M = max_p m_p (block reduction); pass 2: w_p = 2^(m_p - M) into shared
+// memory and L = sum_p w_p l_p; pass 3: out = sum_p w_p acc_p / L with every thread owning
+// 4 channels and one of 512/D interleaved partition groups (independent loads in flight),
+// the groups then added in a fixed order. The order depends only on partition indices, so
+// the result is deterministic and independent of physical block placement.
 template <int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
+  constexpr int QUADS = D / 4;           // float4 columns of one partial row
+  constexpr int NG = 128 / QUADS;        // partition groups (4 at D=128)
+  constexpr int CHUNK = 2048;            // weights held in shared memory at a time
+  __shared__ float sw[CHUNK];
+  __shared__ float red[32];
+  __shared__ float part[NG][D];
   const int h = blockIdx.x, s = blockIdx.y;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int ctx = checked_ctx(a, s);
   const int np = (ctx + a.part_tokens - 1) / a.part_tokens;
+  if (a.skip_single && np <= 1) return;
   const int64_t row = (int64_t)s * a.num_q_heads + h;
   const float* pm = a.part_m + row * a.max_parts;
   const float* pl = a.part_l + row * a.max_parts;
-  const float* pa_ = a.part_acc + row * a.max_parts * D;
-  float M = -INFINITY;
-  for (int p = 0; p < np; ++p) M = fmaxf(M, pm[p]);
-  for (int d = threadIdx.x; d < D; d += blockDim.x) {
-    float L = 0.f, A = 0.f;
-    for (int p = 0; p < np; ++p) {
-      const float f = fast_exp2(pm[p] - M);
-      L = fmaf(f, pl[p], L);
-      A = fmaf(f, pa_[(int64_t)p * D + d], A);
+  const float* pacc = a.part_acc + row * a.max_parts * D;
+
+  float mx = -INFINITY;
+  for (int p = tid; p < np; p += 128) mx = fmaxf(mx, pm[p]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (lane == 0) red[warp] = mx;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
+
+  const int q = tid % QUADS, grp = tid / QUADS;
+  float lsum = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int c0 = 0; c0 < np; c0 += CHUNK) {
+    const int n = min(CHUNK, np - c0);
+    for (int p = tid; p < n; p += 128) {
+      const float w = M == -INFINITY ? 0.f : fast_exp2(pm[c0 + p] - M);
+      sw[p] = w;
+      lsum = fmaf(w, pl[c0 + p], lsum);
     }
-    store_out(a.out, a.out_dtype, row * D + d, L > 0.f ? A / L : 0.f);
-    if (d == 0 && a.lse_out != nullptr)
+    __syncthreads();
+    const float4* src = reinterpret_cast<const float4*>(pacc + (int64_t)c0 * D) + q;
+#pragma unroll 4
+    for (int p = grp; p < n; p += NG) {
+      const float w = sw[p];
+      const float4 v = __ldg(src + (int64_t)p * QUADS);
+      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  if (lane == 0) red[8 + warp] = lsum;
+  part[grp][4 * q] = acc.x;
+  part[grp][4 * q + 1] = acc.y;
+  part[grp][4 * q + 2] = acc.z;
+  part[grp][4 * q + 3] = acc.w;
+  __syncthreads();
+  const float L = (red[8] + red[9]) + (red[10] + red[11]);
+  if (tid < D) {
+    float A = 0.f;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) A += part[g][tid];
+    store_out(a.out, a.out_dtype, row * D + tid, L > 0.f ? A / L : 0.f);
+    if (tid == 0 && a.lse_out != nullptr)
       a.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
   }
 }

@@ -41,8 +41,18 @@
 
 namespace pa {
 
-// 0 = automatic, 1 = CUDA-core path only, 2 = tensor cores where supported.
+// 0 = automatic, 1 = CUDA-core path only, 2 = tensor cores where supported (automatic
+// kernel choice), 3 / 4 / 5 = tensor cores with the grid / persistent-CTA / warp-worker
+// kernel where the shape allows it (see tc_kind).
 static int g_decode_impl = 0;
+
+// Stage depth of the persistent kernel's per-warp rings (blocks in flight per warp).
+#ifndef PA_TC_PSTAGE_BF16
+#define PA_TC_PSTAGE_BF16 2
+#endif
+#ifndef PA_TC_PSTAGE_FP8
+#define PA_TC_PSTAGE_FP8 3
+#endif
 
 namespace tc {
 
@@ -140,15 +150,294 @@ __device__ __forceinline__ uint32_t swz(uint32_t tile, int r, int c) {
   return tile + r * 128 + ((c ^ (r & 7)) << 4);
 }
 
+__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint32_t bytes,
+                                             uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 template <pa_dtype KV>
 struct TcCfg {
   static constexpr bool kFp8 = KV == PA_FP8_E4M3;
   static constexpr int kTile = kFp8 ? 2048 : 4096;      // one (block, head) tile of K or V
   static constexpr int kStage = 2 * kTile;              // K + V
-  static constexpr int kNStage = kFp8 ? 4 : 3;          // blocks in flight per warp
+  static constexpr int kRows = kTile / 128;             // tensor-map rows per tile
+  // CTA-per-item kernel (single pass): stages only
+  static constexpr int kNStage = kFp8 ? 4 : 3;
   static constexpr int kSmem = kNW * kNStage * kStage + kNW * kNStage * 8 + 1024;
+  // persistent kernel (split path): blocks in flight per warp
+  static constexpr int kPStage = kFp8 ? PA_TC_PSTAGE_FP8 : PA_TC_PSTAGE_BF16;
+  static constexpr int kPStageBytes = kNW * kPStage * kStage;
+  static constexpr int kQBytes = 8 * kD * 2;            // one group's q (<= 8 heads, bf16)
+  static constexpr int kMergeBytes = kNW * 8 * kD * 4 + 2 * kNW * 8 * 4;
+  static constexpr int kPSmem = kPStageBytes + 2 * kQBytes + kMergeBytes + 256 + 1024;
 };
 
+// Per-warp running state of one work item: O^T fragments (8 tiles of 16 channels x 8
+// heads), running max / sum of the two heads this thread holds, fp8 V-scale reference.
+struct WarpAcc {
+  float acc[8][4];
+  float m0, m1, l0, l1, vref;
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+    vref = 0.f;
+  }
+};
+
+// q of one group in the registers of the mma B fragments (rows g >= G zero), raw bf16
+// words: bf16 path word (j, 0/1) = channels 16j + 2tq + {0,1} / 16j + 8 + 2tq + {0,1};
+// fp8 path words (c, 0/1) = channels 16c + 4tq + {0,1} / {2,3}. `qp` points at the group's
+// first row (global or shared memory, rows of kD).
+template <bool FP8>
+__device__ __forceinline__ void load_q_raw(const uint16_t* qp, int G, int lane,
+                                           uint32_t (&raw)[8][2]) {
+  const int gq = lane >> 2, tq = lane & 3;
+  const bool live = gq < G;
+  const uint16_t* r = qp + gq * kD;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    if constexpr (!FP8) {
+      raw[j][0] = live ? *reinterpret_cast<const uint32_t*>(r + 16 * j + 2 * tq) : 0u;
+      raw[j][1] = live ? *reinterpret_cast<const uint32_t*>(r + 16 * j + 8 + 2 * tq) : 0u;
+    } else {
+      const uint2 w = live ? *reinterpret_cast<const uint2*>(r + 16 * j + 4 * tq) : make_uint2(0, 0);
+      raw[j][0] = w.x;
+      raw[j][1] = w.y;
+    }
+  }
+}
+
+// B fragments from the raw words; returns the log2-domain score scale. fp8: q is scaled by
+// the power of two putting max|q| of the group in [2^14, 2^15) and converted to f16 (exact
+// for bf16 inputs in that range); the scale is undone in the returned factor.
+template <bool FP8>
+__device__ __forceinline__ float q_frags(const uint32_t (&raw)[8][2], float scale_log2,
+                                         uint32_t (&qf)[8][2]) {
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { qf[j][0] = raw[j][0]; qf[j][1] = raw[j][1]; }
+    return scale_log2;
+  } else {
+    float amax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(raw[j][h])), fabsf(bf16_hi(raw[j][h]))));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int e = 0;
+    const uint32_t ebits = (__float_as_uint(amax) >> 23) & 0xff;
+    if (ebits != 0 && ebits != 0xff) e = 15 - ((int)ebits - 126);
+    e = max(-100, min(100, e));
+    const float up = __uint_as_float((uint32_t)(127 + e) << 23);
+    const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        qf[j][h] = pack_f16x2(bf16_lo(raw[j][h]) * up, bf16_hi(raw[j][h]) * up);
+    return scale_log2 * down;
+  }
+}
+
+template <bool FP8>
+__device__ __forceinline__ float load_q_frags(const uint16_t* qp, int G, int lane,
+                                              float scale_log2, uint32_t (&qf)[8][2]) {
+  uint32_t raw[8][2];
+  load_q_raw<FP8>(qp, G, lane, raw);
+  return q_frags<FP8>(raw, scale_log2, qf);
+}
+
+// One 16-token block: S^T = K Q^T on the tensor cores, online softmax, O^T += V^T P^T.
+// kt / vt: shared addresses of the block's swizzled K and V tiles; nvalid: tokens of the
+// block inside the work item; zs: log2-domain score scale (x fp8 K scale); vs: fp8 V scale.
+// The K products run as two independent accumulation chains and the V fragments are read
+// before the softmax, so a warp has independent work in flight at every step.
+template <bool FP8>
+__device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, float zs,
+                                         float vs, const uint32_t (&qf)[8][2], WarpAcc& w,
+                                         int lane) {
+  constexpr int TILE = FP8 ? 2048 : 4096;
+  const int gq = lane >> 2;
+  float pv = 1.f, beta = 1.f;
+  if constexpr (FP8) {
+    const float vnew = fmaxf(w.vref, vs);
+    beta = w.vref > 0.f ? w.vref / vnew : 1.f;
+    pv = vnew > 0.f ? vs / vnew : 0.f;
+    w.vref = vnew;
+  }
+  // rows of tokens past the item may hold anything (even NaN): zero them before P.V reads
+  if (nvalid < kBS) {
+    const int bytes_per_tok = TILE / kBS;
+    for (int o = nvalid * bytes_per_tok + lane * 16; o < TILE; o += 32 * 16)
+      asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(vt + o), "r"(0) : "memory");
+    __syncwarp();
+  }
+  const int mi = lane >> 3;
+  // ---- S^T = K Q^T : 16 tokens x 8 heads, two independent chains ----
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const int tok = (lane & 7) + 8 * (mi & 1);
+    if constexpr (!FP8) {
+      // rows of the tile: 2*token + (channel >= 64); chunk = (channel % 64) / 8
+      uint32_t r[8][4];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int d0 = 16 * j + 8 * (mi >> 1);
+        ldsm_x4(swz(kt, 2 * tok + (d0 >> 6), (d0 & 63) >> 3), r[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; j += 2) {
+        mma16816<false>(sa, r[j], qf[j][0], qf[j][1]);
+        mma16816<false>(sb, r[j + 1], qf[j + 1][0], qf[j + 1][1]);
+      }
+    } else {
+      uint32_t r[4][4];
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) ldsm_x4(swz(kt, tok, 2 * cp + (mi >> 1)), r[cp]);
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) {
+        uint32_t x0[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[cp][0])), e4m3x2_to_f16x2((uint16_t)lo16(r[cp][1])),
+                          e4m3x2_to_f16x2((uint16_t)hi16(r[cp][0])), e4m3x2_to_f16x2((uint16_t)hi16(r[cp][1]))};
+        mma16816<true>(sa, x0, qf[2 * cp][0], qf[2 * cp][1]);
+        uint32_t x1[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[cp][2])), e4m3x2_to_f16x2((uint16_t)lo16(r[cp][3])),
+                          e4m3x2_to_f16x2((uint16_t)hi16(r[cp][2])), e4m3x2_to_f16x2((uint16_t)hi16(r[cp][3]))};
+        mma16816<true>(sb, x1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+      }
+    }
+  }
+  // ---- V fragments (independent of the softmax) ----
+  uint32_t vr[8][4];
+  {
+    const int tok = (lane & 7) + 8 * (mi >> 1);
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        const int d0 = 16 * t + 8 * (mi & 1);
+        ldsm_x4_t(swz(vt, 2 * tok + (d0 >> 6), (d0 & 63) >> 3), vr[t]);
+      }
+    } else {
+#pragma unroll
+      for (int cp = 0; cp < 4; ++cp) ldsm_x4_t(swz(vt, tok, 2 * cp + (mi & 1)), vr[cp]);
+    }
+  }
+  // ---- online softmax (log2 domain); thread holds tokens gq, gq+8 x heads 2tq, 2tq+1 ----
+  const bool va = gq < nvalid, vb = gq + 8 < nvalid;
+  const float z0 = va ? (sa[0] + sb[0]) * zs : -INFINITY, z1 = va ? (sa[1] + sb[1]) * zs : -INFINITY;
+  const float z2 = vb ? (sa[2] + sb[2]) * zs : -INFINITY, z3 = vb ? (sa[3] + sb[3]) * zs : -INFINITY;
+  float bm0 = fmaxf(z0, z2), bm1 = fmaxf(z1, z3);
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
+    bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
+  }
+  const float mn0 = fmaxf(w.m0, bm0), mn1 = fmaxf(w.m1, bm1);
+  const float al0 = fast_exp2(w.m0 - mn0), al1 = fast_exp2(w.m1 - mn1);
+  w.m0 = mn0;
+  w.m1 = mn1;
+  const float p0 = fast_exp2(z0 - mn0), p1 = fast_exp2(z1 - mn1);
+  const float p2 = fast_exp2(z2 - mn0), p3 = fast_exp2(z3 - mn1);
+  w.l0 = w.l0 * al0 + (p0 + p2);
+  w.l1 = w.l1 * al1 + (p1 + p3);
+  if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f || beta != 1.f)) {
+    const float f0 = al0 * beta, f1 = al1 * beta;
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      w.acc[t][0] *= f0; w.acc[t][1] *= f1; w.acc[t][2] *= f0; w.acc[t][3] *= f1;
+    }
+  }
+  // P^T as B fragments: pack [token][head] pairs, transpose 8x8 in registers
+  uint32_t pb0, pb1;
+  if constexpr (FP8) {
+    pb0 = movm_t(pack_f16x2(p0 * pv, p1 * pv));
+    pb1 = movm_t(pack_f16x2(p2 * pv, p3 * pv));
+  } else {
+    pb0 = movm_t(pack_bf16x2(p0, p1));
+    pb1 = movm_t(pack_bf16x2(p2, p3));
+  }
+  // ---- O^T += V^T P^T ----
+  if constexpr (!FP8) {
+#pragma unroll
+    for (int t = 0; t < 8; ++t) mma16816<false>(w.acc[t], vr[t], pb0, pb1);
+  } else {
+#pragma unroll
+    for (int cp = 0; cp < 4; ++cp) {
+      uint32_t y[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) y[u] = __byte_perm(vr[cp][u], 0, 0x3120);
+      uint32_t ev[4] = {e4m3x2_to_f16x2((uint16_t)lo16(y[0])), e4m3x2_to_f16x2((uint16_t)lo16(y[1])),
+                        e4m3x2_to_f16x2((uint16_t)lo16(y[2])), e4m3x2_to_f16x2((uint16_t)lo16(y[3]))};
+      mma16816<true>(w.acc[2 * cp], ev, pb0, pb1);
+      uint32_t od[4] = {e4m3x2_to_f16x2((uint16_t)hi16(y[0])), e4m3x2_to_f16x2((uint16_t)hi16(y[1])),
+                        e4m3x2_to_f16x2((uint16_t)hi16(y[2])), e4m3x2_to_f16x2((uint16_t)hi16(y[3]))};
+      mma16816<true>(w.acc[2 * cp + 1], od, pb0, pb1);
+    }
+  }
+}
+
+// Writes a warp's finished state into the merge area: m/l per head and the unnormalised
+// output [8][kD] (true units: fp8 accumulators are scaled back by vref).
+template <bool FP8>
+__device__ __forceinline__ void stash_warp(WarpAcc& w, float* sacc, float* smx, float* slx,
+                                           int warp, int lane) {
+  const int gq = lane >> 2, tq = lane & 3;
+#pragma unroll
+  for (int o = 4; o < 32; o <<= 1) {
+    w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, o);
+    w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, o);
+  }
+  if (gq == 0) {
+    smx[warp * 8 + 2 * tq] = w.m0; smx[warp * 8 + 2 * tq + 1] = w.m1;
+    slx[warp * 8 + 2 * tq] = w.l0; slx[warp * 8 + 2 * tq + 1] = w.l1;
+  }
+  const float unit = FP8 ? w.vref : 1.f;
+  float* wacc = sacc + warp * 8 * kD;
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    int dA, dB;
+    if constexpr (FP8) {
+      const int cp = t >> 1, par = t & 1;
+      dA = 32 * cp + 2 * gq + par;
+      dB = 32 * cp + 16 + 2 * gq + par;
+    } else {
+      dA = 16 * t + gq;
+      dB = 16 * t + 8 + gq;
+    }
+    wacc[(2 * tq) * kD + dA] = w.acc[t][0] * unit;
+    wacc[(2 * tq + 1) * kD + dA] = w.acc[t][1] * unit;
+    wacc[(2 * tq) * kD + dB] = w.acc[t][2] * unit;
+    wacc[(2 * tq + 1) * kD + dB] = w.acc[t][3] * unit;
+  }
+}
+
+// Combines the kNW warps' states of head g, channel d (after stash_warp + __syncthreads).
+__device__ __forceinline__ void combine_warps(const float* sacc, const float* smx,
+                                              const float* slx, int g, int d, float& M, float& L,
+                                              float& A) {
+  M = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < kNW; ++w) M = fmaxf(M, smx[w * 8 + g]);
+  L = 0.f;
+  A = 0.f;
+  if (M != -INFINITY) {
+#pragma unroll
+    for (int w = 0; w < kNW; ++w) {
+      const float f = fast_exp2(smx[w * 8 + g] - M);
+      L = fmaf(f, slx[w * 8 + g], L);
+      A = fmaf(f, sacc[(w * 8 + g) * kD + d], A);
+    }
+  }
+}
+
+// =======================================================================================
+// Single pass: one CTA per (sequence, kv head) work item, grid (1, Hkv, S).
+// =======================================================================================
 template <pa_dtype KV>
 __global__ void __launch_bounds__(kNW * 32)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
@@ -156,7 +445,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   using C = TcCfg<KV>;
   constexpr bool FP8 = C::kFp8;
   constexpr int TILE = C::kTile, STAGE = C::kStage, NST = C::kNStage;
-  constexpr int ROWS = TILE / 128;  // tensor-map rows per tile (32 bf16 / 16 fp8)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -168,7 +456,6 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   const int t1 = min(ctx, t0 + a.part_tokens);
   const int G = a.group;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gq = lane >> 2, tq = lane & 3;
 
   const uint32_t wtiles = smem_u32(smem + warp * NST * STAGE);
   const uint32_t bars = smem_u32(smem + kNW * NST * STAGE) + warp * NST * 8;
@@ -180,48 +467,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   }
   __syncwarp();
 
-  // ---- q of the group as mma B fragments (rows g >= G are zero) ----
   uint32_t qf[8][2];
-  float zscale = a.scale_log2;
-  {
-    const uint16_t* qp = static_cast<const uint16_t*>(a.q) +
-                         ((int64_t)s * a.num_q_heads + kvh * G + gq) * kD;
-    const bool live = gq < G;
-    if constexpr (!FP8) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        qf[j][0] = live ? *reinterpret_cast<const uint32_t*>(qp + 16 * j + 2 * tq) : 0u;
-        qf[j][1] = live ? *reinterpret_cast<const uint32_t*>(qp + 16 * j + 8 + 2 * tq) : 0u;
-      }
-    } else {
-      // k-step c uses channels 16c + 4tq + {0,1} (low pair) and + {2,3} (high pair)
-      float qv[8][4];
-      float amax = 0.f;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint2 w = live ? *reinterpret_cast<const uint2*>(qp + 16 * c + 4 * tq) : make_uint2(0, 0);
-        qv[c][0] = bf16_lo(w.x); qv[c][1] = bf16_hi(w.x);
-        qv[c][2] = bf16_lo(w.y); qv[c][3] = bf16_hi(w.y);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) amax = fmaxf(amax, fabsf(qv[c][e]));
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      // power of two putting max|q| in [2^14, 2^15): exact scaling into f16 range
-      int e = 0;
-      const uint32_t ebits = (__float_as_uint(amax) >> 23) & 0xff;
-      if (ebits != 0 && ebits != 0xff) e = 15 - ((int)ebits - 126);
-      e = max(-100, min(100, e));
-      const float up = __uint_as_float((uint32_t)(127 + e) << 23);
-      const float down = __uint_as_float((uint32_t)(127 - e) << 23);
-      zscale *= down;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        qf[c][0] = pack_f16x2(qv[c][0] * up, qv[c][1] * up);
-        qf[c][1] = pack_f16x2(qv[c][2] * up, qv[c][3] * up);
-      }
-    }
-  }
+  const float zscale = load_q_frags<FP8>(
+      static_cast<const uint16_t*>(a.q) + ((int64_t)s * a.num_q_heads + kvh * G) * kD, G, lane,
+      a.scale_log2, qf);
 
   // ---- this warp's blocks and its block-table windows (32 entries per register) ----
   const int b_begin = t0 / kBS, b_end = (t1 + kBS - 1) / kBS;
@@ -249,15 +498,16 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   load_window(0, cur_p, cur_ks, cur_vs);
   load_window(32, nxt_p, nxt_ks, nxt_vs);
   const uint64_t policy = evict_first_policy();
-  const int kvrow_stride = ROWS;  // tensor-map rows per (block, head) tile
   auto issue = [&](int k, int wbase, int stage) {
     const int rel = k - wbase;
     const int p = rel < 32 ? __shfl_sync(0xffffffffu, cur_p, rel)
                            : __shfl_sync(0xffffffffu, nxt_p, rel - 32);
     if (lane == 0) {
       const uint32_t bar = bars + 8 * stage;
+      // the stage was last read (and maybe written) through the generic proxy
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       if (p >= 0) {
-        const int row = (p * a.num_kv_heads + kvh) * kvrow_stride;
+        const int row = (p * a.num_kv_heads + kvh) * C::kRows;
         const uint32_t dst = wtiles + stage * STAGE;
         mbar_arrive_tx(bar, STAGE);
         tma_load_2d(dst, &kmap, 0, row, bar, policy);
@@ -269,14 +519,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   };
   for (int k = 0; k < NST && k < nmine; ++k) issue(k, 0, k);
 
-  float acc[8][4];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  float vref = 0.f;  // fp8: running max of the V scales seen (acc is in units of vref)
+  WarpAcc w;
+  w.reset();
   bool timed_out = false;
   int consumed = 0;
-
   for (int i = 0; i < nmine; ++i) {
     const int wbase = i & ~31;
     if ((i & 31) == 0 && i > 0) {
@@ -284,9 +530,10 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
       load_window(i + 32, nxt_p, nxt_ks, nxt_vs);
     }
     const int stage = i % NST;
-    const uint32_t par = (uint32_t)((i / NST) & 1);
     const int p = __shfl_sync(0xffffffffu, cur_p, i & 31);
-    if (!mbar_wait(bars + 8 * stage, par)) {
+    const float ks = __shfl_sync(0xffffffffu, cur_ks, i & 31);
+    const float vs = __shfl_sync(0xffffffffu, cur_vs, i & 31);
+    if (!mbar_wait(bars + 8 * stage, (uint32_t)((i / NST) & 1))) {
       if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
       timed_out = true;
       break;
@@ -294,117 +541,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
     consumed = i + 1;
     if (p >= 0) {
       const int b = b_begin + warp + i * kNW;
-      const int nvalid = min(kBS, t1 - b * kBS);
-      const uint32_t kt = wtiles + stage * STAGE, vt = kt + TILE;
-      float zs = zscale;
-      float pv = 1.f, beta = 1.f;
-      if constexpr (FP8) {
-        const float ks = __shfl_sync(0xffffffffu, cur_ks, i & 31);
-        const float vs = __shfl_sync(0xffffffffu, cur_vs, i & 31);
-        zs *= ks;
-        const float vnew = fmaxf(vref, vs);
-        beta = vref > 0.f ? vref / vnew : 1.f;
-        pv = vnew > 0.f ? vs / vnew : 0.f;
-        vref = vnew;
-      }
-      // ---- S^T = K Q^T : 16 tokens x 8 heads ----
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (!FP8) {
-        // rows of the tile: 2*token + (channel >= 64); chunk = (channel % 64) / 8
-        const int mi = lane >> 3;
-        const int tok = (lane & 7) + 8 * (mi & 1);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int d0 = 16 * j + 8 * (mi >> 1);
-          uint32_t r[4];
-          ldsm_x4(swz(kt, 2 * tok + (d0 >> 6), (d0 & 63) >> 3), r);
-          mma16816<false>(sc, r, qf[j][0], qf[j][1]);
-        }
-      } else {
-        const int mi = lane >> 3;
-        const int tok = (lane & 7) + 8 * (mi & 1);
-#pragma unroll
-        for (int cp = 0; cp < 4; ++cp) {
-          uint32_t r[4];
-          ldsm_x4(swz(kt, tok, 2 * cp + (mi >> 1)), r);
-          uint32_t x0[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[0])), e4m3x2_to_f16x2((uint16_t)lo16(r[1])),
-                            e4m3x2_to_f16x2((uint16_t)hi16(r[0])), e4m3x2_to_f16x2((uint16_t)hi16(r[1]))};
-          mma16816<true>(sc, x0, qf[2 * cp][0], qf[2 * cp][1]);
-          uint32_t x1[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[2])), e4m3x2_to_f16x2((uint16_t)lo16(r[3])),
-                            e4m3x2_to_f16x2((uint16_t)hi16(r[2])), e4m3x2_to_f16x2((uint16_t)hi16(r[3]))};
-          mma16816<true>(sc, x1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
-        }
-      }
-      // ---- online softmax (log2 domain); thread holds tokens gq, gq+8 x heads 2tq, 2tq+1 ----
-      const bool va = gq < nvalid, vb = gq + 8 < nvalid;
-      const float z0 = va ? sc[0] * zs : -INFINITY, z1 = va ? sc[1] * zs : -INFINITY;
-      const float z2 = vb ? sc[2] * zs : -INFINITY, z3 = vb ? sc[3] * zs : -INFINITY;
-      float bm0 = fmaxf(z0, z2), bm1 = fmaxf(z1, z3);
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
-        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
-      }
-      const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-      const float al0 = fast_exp2(m0 - mn0), al1 = fast_exp2(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      const float p0 = fast_exp2(z0 - mn0), p1 = fast_exp2(z1 - mn1);
-      const float p2 = fast_exp2(z2 - mn0), p3 = fast_exp2(z3 - mn1);
-      l0 = l0 * al0 + (p0 + p2);
-      l1 = l1 * al1 + (p1 + p3);
-      if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f || beta != 1.f)) {
-        const float f0 = al0 * beta, f1 = al1 * beta;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          acc[t][0] *= f0; acc[t][1] *= f1; acc[t][2] *= f0; acc[t][3] *= f1;
-        }
-      }
-      // P^T as B fragments: pack [token][head] pairs, transpose 8x8 in registers
-      uint32_t pb0, pb1;
-      if constexpr (FP8) {
-        pb0 = movm_t(pack_f16x2(p0 * pv, p1 * pv));
-        pb1 = movm_t(pack_f16x2(p2 * pv, p3 * pv));
-      } else {
-        pb0 = movm_t(pack_bf16x2(p0, p1));
-        pb1 = movm_t(pack_bf16x2(p2, p3));
-      }
-      // rows of tokens past the context may hold anything: zero them before P.V
-      if (nvalid < kBS) {
-        const int bytes_per_tok = TILE / kBS;
-        for (int o = nvalid * bytes_per_tok + lane * 16; o < TILE; o += 32 * 16)
-          asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(vt + o), "r"(0) : "memory");
-        __syncwarp();
-      }
-      // ---- O^T += V^T P^T ----
-      if constexpr (!FP8) {
-        const int mi = lane >> 3;
-        const int tok = (lane & 7) + 8 * (mi >> 1);
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-          const int d0 = 16 * t + 8 * (mi & 1);
-          uint32_t r[4];
-          ldsm_x4_t(swz(vt, 2 * tok + (d0 >> 6), (d0 & 63) >> 3), r);
-          mma16816<false>(acc[t], r, pb0, pb1);
-        }
-      } else {
-        const int mi = lane >> 3;
-        const int tok = (lane & 7) + 8 * (mi >> 1);
-#pragma unroll
-        for (int cp = 0; cp < 4; ++cp) {
-          uint32_t r[4];
-          ldsm_x4_t(swz(vt, tok, 2 * cp + (mi & 1)), r);
-          uint32_t y[4];
-#pragma unroll
-          for (int u = 0; u < 4; ++u) y[u] = __byte_perm(r[u], 0, 0x3120);
-          uint32_t ev[4] = {e4m3x2_to_f16x2((uint16_t)lo16(y[0])), e4m3x2_to_f16x2((uint16_t)lo16(y[1])),
-                            e4m3x2_to_f16x2((uint16_t)lo16(y[2])), e4m3x2_to_f16x2((uint16_t)lo16(y[3]))};
-          mma16816<true>(acc[2 * cp], ev, pb0, pb1);
-          uint32_t od[4] = {e4m3x2_to_f16x2((uint16_t)hi16(y[0])), e4m3x2_to_f16x2((uint16_t)hi16(y[1])),
-                            e4m3x2_to_f16x2((uint16_t)hi16(y[2])), e4m3x2_to_f16x2((uint16_t)hi16(y[3]))};
-          mma16816<true>(acc[2 * cp + 1], od, pb0, pb1);
-        }
-      }
+      const uint32_t kt = wtiles + stage * STAGE;
+      tc_block<FP8>(kt, kt + TILE, min(kBS, t1 - b * kBS), zscale * ks, vs, qf, w, lane);
     }
     __syncwarp();
     if (i + NST < nmine) issue(i + NST, wbase, stage);
@@ -412,59 +550,528 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   if (timed_out) {
     // wait (bounded) for every copy this warp issued and did not consume
     const int issued = min(nmine, consumed + NST);
-    for (int k = consumed; k < issued; ++k) {
+    for (int k = consumed; k < issued; ++k)
       if (!mbar_wait(bars + 8 * (k % NST), (uint32_t)((k / NST) & 1))) break;
-    }
   }
 
   // ---- merge the warps through shared memory (stage buffers are free now) ----
-#pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-  }
   __syncthreads();
-  float* sacc = reinterpret_cast<float*>(smem);             // [kNW][8][kD]
-  float* smx = sacc + kNW * 8 * kD;                          // [kNW][8]
-  float* slx = smx + kNW * 8;                                // [kNW][8]
-  if (gq == 0) {
-    smx[warp * 8 + 2 * tq] = m0; smx[warp * 8 + 2 * tq + 1] = m1;
-    slx[warp * 8 + 2 * tq] = l0; slx[warp * 8 + 2 * tq + 1] = l1;
-  }
-  const float unit = FP8 ? vref : 1.f;
-  float* wacc = sacc + warp * 8 * kD;
-#pragma unroll
-  for (int t = 0; t < 8; ++t) {
-    int dA, dB;
-    if constexpr (FP8) {
-      const int cp = t >> 1, par = t & 1;
-      dA = 32 * cp + 2 * gq + par;
-      dB = 32 * cp + 16 + 2 * gq + par;
-    } else {
-      dA = 16 * t + gq;
-      dB = 16 * t + 8 + gq;
-    }
-    wacc[(2 * tq) * kD + dA] = acc[t][0] * unit;
-    wacc[(2 * tq + 1) * kD + dA] = acc[t][1] * unit;
-    wacc[(2 * tq) * kD + dB] = acc[t][2] * unit;
-    wacc[(2 * tq + 1) * kD + dB] = acc[t][3] * unit;
-  }
+  float* sacc = reinterpret_cast<float*>(smem);  // [kNW][8][kD]
+  float* smx = sacc + kNW * 8 * kD;               // [kNW][8]
+  float* slx = smx + kNW * 8;                     // [kNW][8]
+  stash_warp<FP8>(w, sacc, smx, slx, warp, lane);
   __syncthreads();
   for (int idx = threadIdx.x; idx < G * kD; idx += blockDim.x) {
     const int g = idx / kD, d = idx % kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kNW; ++w) M = fmaxf(M, smx[w * 8 + g]);
-    float L = 0.f, A = 0.f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) {
-        const float f = fast_exp2(smx[w * 8 + g] - M);
-        L = fmaf(f, slx[w * 8 + g], L);
-        A = fmaf(f, sacc[(w * 8 + g) * kD + d], A);
+    float M, L, A;
+    combine_warps(sacc, smx, slx, g, d, M, L, A);
+    emit(a, s, kvh * G + g, part, kD, d, M, L, A);
+  }
+}
+
+// =======================================================================================
+// Split path: plan kernel + persistent kernel with the log-sum-exp merge fused in.
+// =======================================================================================
+// Workspace of the split path (offsets in bytes, each region 256-aligned):
+//   [0]     uint32 fetch counter, uint32 total items
+//   list    int2 (seq, partition) per partition item, largest items first
+//   m, l    float [S][Hq][P];  acc float [S][Hq][P][kD]   (partials, as the CUDA-core path)
+// Sequences with a single partition are written to `out` directly; the others are merged
+// by lse_reduce_kernel afterwards (spread over every (seq, q head)).
+struct PlanView {
+  uint32_t* counters;  // [0] fetch, [1] total
+  int2* list;
+};
+
+// One CTA of 1024 threads: counts partitions per size (blocks per item), orders them
+// largest first (full partitions, then partial ones by size), writes the list, zeroes the
+// fetch counter, and writes out = 0 / lse = -inf for empty sequences.
+__global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
+  __shared__ int cnt[130], off[130];
+  const int P = a.part_tokens;
+  const int nbk = P / kBS;  // blocks of a full partition (<= 128)
+  for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+    const int ctx = checked_ctx(a, s);
+    if (ctx == 0) {
+      for (int h = 0; h < a.num_q_heads; ++h) {
+        const int64_t row = (int64_t)s * a.num_q_heads + h;
+        for (int d = 0; d < kD; ++d) store_out(a.out, a.out_dtype, row * kD + d, 0.f);
+        if (a.lse_out != nullptr) a.lse_out[row] = -INFINITY;
+      }
+      continue;
+    }
+    const int full = ctx / P, rem = ctx % P;
+    if (full) atomicAdd(&cnt[nbk], full);
+    if (rem) atomicAdd(&cnt[(rem + kBS - 1) / kBS], 1);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int acc = 0;
+    for (int b = nbk; b >= 1; --b) {
+      off[b] = acc;
+      acc += cnt[b];
+    }
+    pl.counters[0] = 0;
+    pl.counters[1] = (uint32_t)acc * (uint32_t)a.num_kv_heads;
+  }
+  __syncthreads();
+  for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
+    const int ctx = checked_ctx(a, s);
+    const int full = ctx / P, rem = ctx % P;
+    if (full) {
+      const int base = atomicAdd(&off[nbk], full);
+      for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
+    }
+    if (rem) pl.list[atomicAdd(&off[(rem + kBS - 1) / kBS], 1)] = make_int2(s, full);
+  }
+}
+
+// Work item slot shared by the CTA (written by thread 0 between barriers).
+struct ItemSlot {
+  int valid, s, part, kvh;
+};
+
+template <pa_dtype KV>
+__global__ void __launch_bounds__(kNW * 32)
+decode_tc_persistent(const DecodeArgs a, const PlanView pl,
+                     const __grid_constant__ CUtensorMap kmap,
+                     const __grid_constant__ CUtensorMap vmap) {
+  using C = TcCfg<KV>;
+  constexpr bool FP8 = C::kFp8;
+  constexpr int TILE = C::kTile, STAGE = C::kStage, NST = C::kPStage;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  uint8_t* qbuf = smem + C::kPStageBytes;                        // [2][8][kD] bf16
+  float* sacc = reinterpret_cast<float*>(qbuf + 2 * C::kQBytes);  // [kNW][8][kD]
+  float* smx = sacc + kNW * 8 * kD;
+  float* slx = smx + kNW * 8;
+  uint64_t* barmem = reinterpret_cast<uint64_t*>(slx + kNW * 8);  // [kNW*NST] + [2] q
+  ItemSlot* slots = reinterpret_cast<ItemSlot*>(barmem + kNW * NST + 2);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = a.group, Hkv = a.num_kv_heads, P = a.part_tokens;
+  const uint32_t wtiles = smem_u32(smem + warp * NST * STAGE);
+  const uint32_t bars = smem_u32(barmem) + warp * NST * 8;
+  const uint32_t qbars = smem_u32(barmem + kNW * NST);
+  const uint32_t total = pl.counters[1];
+  const uint64_t policy = evict_first_policy();
+
+  // thread 0: take the next item from the shared counter into slot `sl`, start its q copy
+  auto fetch = [&](int sl) {
+    const uint32_t it = atomicAdd(&pl.counters[0], 1u);
+    ItemSlot x{0, 0, 0, 0};
+    if (it < total) {
+      const int2 sp = pl.list[it / Hkv];
+      x = ItemSlot{1, sp.x, sp.y, (int)(it % Hkv)};
+      const uint32_t qb = qbars + 8 * sl;
+      mbar_arrive_tx(qb, (uint32_t)(G * kD * 2));
+      bulk_load_1d(smem_u32(qbuf + sl * C::kQBytes),
+                   static_cast<const uint16_t*>(a.q) + ((int64_t)x.s * a.num_q_heads + x.kvh * G) * kD,
+                   (uint32_t)(G * kD * 2), qb);
+    }
+    slots[sl] = x;
+  };
+
+  if (tid == 0) {
+    for (int i = 0; i < kNW * NST + 2; ++i) mbar_init(smem_u32(barmem + i), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    fetch(0);
+    fetch(1);
+  }
+  __syncthreads();
+
+  // Per-warp view of an item: its blocks are b_begin + warp + k*kNW, k < nmine (<= 32).
+  struct WarpItem {
+    int valid, s, kvh, part, t1, b_begin, nmine, np;
+  };
+  auto item_view = [&](int sl) {
+    const ItemSlot x = slots[sl];
+    WarpItem v{x.valid, x.s, x.kvh, x.part, 0, 0, 0, 0};
+    if (x.valid) {
+      const int ctx = checked_ctx(a, x.s);
+      const int t0 = x.part * P;
+      v.t1 = min(ctx, t0 + P);
+      v.b_begin = t0 / kBS;
+      const int nblk = (v.t1 + kBS - 1) / kBS - v.b_begin;
+      v.nmine = nblk > warp ? (nblk - warp + kNW - 1) / kNW : 0;
+      v.np = (ctx + P - 1) / P;
+    }
+    return v;
+  };
+  // block-table window of an item for this warp: lane k holds block k's (phys, ks, vs)
+  auto load_window = [&](const WarpItem& v, int& p, float& ks, float& vs) {
+    p = -2;
+    ks = 1.f;
+    vs = 1.f;
+    if (v.valid && lane < v.nmine) {
+      p = a.block_tables[(int64_t)v.s * a.max_blocks_per_seq + v.b_begin + warp + lane * kNW];
+      if (p < 0 || p >= a.num_blocks) {
+        flag_error(PA_DEVERR_BLOCK_ID);
+        p = -1;
+      } else if constexpr (FP8) {
+        ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
+        vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
       }
     }
-    emit(a, s, kvh * G + g, part, kD, d, M, L, A);
+  };
+
+  int k = 0;  // CTA-local item counter: item k lives in slot k & 1
+  WarpItem cur = item_view(0), nxt = item_view(1);
+  int cur_p, nxt_p;
+  float cur_ks, cur_vs, nxt_ks, nxt_vs;
+  load_window(cur, cur_p, cur_ks, cur_vs);
+  load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+
+  // producer position in this warp's block stream: (pslot 0 = cur / 1 = nxt, pk)
+  int pslot = 0, pk = 0;
+  uint32_t g_iss = 0, g_cons = 0;
+  bool dead = false;
+  auto produce = [&]() {
+    while (!dead && g_iss - g_cons < (uint32_t)NST) {
+      if (pslot == 0 && pk >= cur.nmine) { pslot = 1; pk = 0; }
+      if (pslot == 1 && (!nxt.valid || pk >= nxt.nmine)) break;
+      const WarpItem& v = pslot == 0 ? cur : nxt;
+      const int p = __shfl_sync(0xffffffffu, pslot == 0 ? cur_p : nxt_p, pk);
+      const int stage = g_iss % NST;
+      if (lane == 0) {
+        const uint32_t bar = bars + 8 * stage;
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (p >= 0) {
+          const int row = (p * Hkv + v.kvh) * C::kRows;
+          const uint32_t dst = wtiles + stage * STAGE;
+          mbar_arrive_tx(bar, STAGE);
+          tma_load_2d(dst, &kmap, 0, row, bar, policy);
+          tma_load_2d(dst + TILE, &vmap, 0, row, bar, policy);
+        } else {
+          mbar_arrive(bar);
+        }
+      }
+      ++g_iss;
+      ++pk;
+    }
+  };
+  produce();
+
+  uint32_t qf[8][2];
+  WarpAcc w;
+  while (cur.valid) {
+    // q of the item (bulk copy completes on its slot's barrier)
+    const int sl = k & 1;
+    if (!dead && !mbar_wait(qbars + 8 * sl, (uint32_t)((k >> 1) & 1))) {
+      if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+      dead = true;
+    }
+    const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf + sl * C::kQBytes),
+                                           G, lane, a.scale_log2, qf);
+    w.reset();
+    for (int i = 0; i < cur.nmine; ++i) {
+      const int p = __shfl_sync(0xffffffffu, cur_p, i);
+      const float ks = __shfl_sync(0xffffffffu, cur_ks, i);
+      const float vs = __shfl_sync(0xffffffffu, cur_vs, i);
+      const int stage = g_cons % NST;
+      if (!dead && !mbar_wait(bars + 8 * stage, (g_cons / NST) & 1)) {
+        if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+        dead = true;
+      }
+      if (!dead && p >= 0) {
+        const int b = cur.b_begin + warp + i * kNW;
+        const uint32_t kt = wtiles + stage * STAGE;
+        tc_block<FP8>(kt, kt + TILE, min(kBS, cur.t1 - b * kBS), zscale * ks, vs, qf, w, lane);
+      }
+      __syncwarp();
+      ++g_cons;
+      produce();
+    }
+    // ---- item finished by this warp: merge the warps ----
+    stash_warp<FP8>(w, sacc, smx, slx, warp, lane);
+    __syncthreads();  // [A] merge area complete; slot k&1 and its q buffer are free
+    if (tid == 0) fetch(sl);  // item k+2 into the slot item k used
+    const int s = cur.s, kvh = cur.kvh, part = cur.part, np = cur.np;
+    for (int idx = tid; idx < G * kD; idx += blockDim.x) {
+      const int g = idx / kD, d = idx % kD;
+      float M, L, A;
+      combine_warps(sacc, smx, slx, g, d, M, L, A);
+      const int64_t row = (int64_t)s * a.num_q_heads + kvh * G + g;
+      if (np == 1) {
+        store_out(a.out, a.out_dtype, row * kD + d, L > 0.f ? A / L : 0.f);
+        if (d == 0 && a.lse_out != nullptr)
+          a.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+      } else {
+        const int64_t pr = row * a.max_parts + part;
+        a.part_acc[pr * kD + d] = A;
+        if (d == 0) { a.part_m[pr] = M; a.part_l[pr] = L; }
+      }
+    }
+    __syncthreads();  // [A2] merge area read by every thread; slot k&1 holds item k+2
+    // ---- advance: item k+1 becomes current, item k+2 (just fetched) the next ----
+    ++k;
+    cur = nxt;
+    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs;
+    nxt = item_view((k + 1) & 1);
+    load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+    pslot = 0;  // the producer finished item k, so it was positioned in item k+1
+    produce();
+  }
+  if (dead) {
+    // wait (bounded) for the copies this warp issued and did not consume
+    for (uint32_t j = g_cons; j < g_iss; ++j)
+      if (!mbar_wait(bars + 8 * (j % NST), (j / NST) & 1)) break;
+  }
+}
+
+// =======================================================================================
+// Split path, warp workers: every warp of the grid is an independent worker that takes
+// (sequence, partition, kv head) items from the shared counter and streams all blocks of
+// the item through its own TMA ring; no shared merge area and no CTA barrier after set-up.
+// q of the next item and its block-table window are fetched while the current one runs.
+// Partitions of at most 512 tokens (32 blocks: one register window per item).
+// =======================================================================================
+#ifndef PA_TCW_WARPS
+#define PA_TCW_WARPS 2
+#endif
+#ifndef PA_TCW_STAGE_BF16
+#define PA_TCW_STAGE_BF16 3
+#endif
+#ifndef PA_TCW_STAGE_FP8
+#define PA_TCW_STAGE_FP8 3
+#endif
+constexpr int kWW = PA_TCW_WARPS;
+
+#ifndef PA_TCW_MIN_WARPS
+#define PA_TCW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
+#endif
+
+template <pa_dtype KV>
+struct TcwCfg {
+  static constexpr int kNStage = KV == PA_FP8_E4M3 ? PA_TCW_STAGE_FP8 : PA_TCW_STAGE_BF16;
+  static constexpr int kQBytes = 8 * kD * 2;  // one group's q, <= 8 heads
+  static constexpr int kSmem =
+      kWW * kNStage * TcCfg<KV>::kStage + kWW * kQBytes + kWW * (kNStage + 1) * 8 + 1024;
+};
+
+template <pa_dtype KV>
+__global__ void __launch_bounds__(kWW * 32, PA_TCW_MIN_WARPS / kWW)
+decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ CUtensorMap kmap,
+                const __grid_constant__ CUtensorMap vmap) {
+  using C = TcCfg<KV>;
+  constexpr bool FP8 = C::kFp8;
+  constexpr int TILE = C::kTile, STAGE = C::kStage, NST = TcwCfg<KV>::kNStage;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int G = a.group, Hkv = a.num_kv_heads, P = a.part_tokens;
+  const uint32_t wtiles = smem_u32(smem + warp * NST * STAGE);
+  uint8_t* qbuf = smem + kWW * NST * STAGE + warp * TcwCfg<KV>::kQBytes;
+  const uint32_t bars = smem_u32(smem + kWW * NST * STAGE + kWW * TcwCfg<KV>::kQBytes) +
+                        warp * (NST + 1) * 8;
+  const uint32_t qbar = bars + NST * 8;
+  if (lane == 0) {
+#pragma unroll
+    for (int i = 0; i <= NST; ++i) mbar_init(bars + 8 * i, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  __syncwarp();
+  const uint32_t total = pl.counters[1];
+  const uint64_t policy = evict_first_policy();
+
+  struct Item {
+    int valid, s, kvh, part, t1, b_begin, nblk, np;
+  };
+  auto fetch = [&]() {
+    uint32_t it = 0;
+    if (lane == 0) it = atomicAdd(&pl.counters[0], 1u);
+    it = __shfl_sync(0xffffffffu, it, 0);
+    Item v{0, 0, 0, 0, 0, 0, 0, 0};
+    if (it < total) {
+      const int2 sp = pl.list[it / Hkv];
+      const int ctx = checked_ctx(a, sp.x);
+      const int t0 = sp.y * P;
+      v.valid = 1;
+      v.s = sp.x;
+      v.kvh = (int)(it % Hkv);
+      v.part = sp.y;
+      v.t1 = min(ctx, t0 + P);
+      v.b_begin = t0 / kBS;
+      v.nblk = (v.t1 + kBS - 1) / kBS - v.b_begin;
+      v.np = (ctx + P - 1) / P;
+    }
+    return v;
+  };
+  // lane k holds block k's (phys, ks, vs) of an item
+  auto load_window = [&](const Item& v, int& p, float& ks, float& vs) {
+    p = -2;
+    ks = 1.f;
+    vs = 1.f;
+    if (v.valid && lane < v.nblk) {
+      p = a.block_tables[(int64_t)v.s * a.max_blocks_per_seq + v.b_begin + lane];
+      if (p < 0 || p >= a.num_blocks) {
+        flag_error(PA_DEVERR_BLOCK_ID);
+        p = -1;
+      } else if constexpr (FP8) {
+        ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
+        vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
+      }
+    }
+  };
+  // lane 0: copy an item's q group (G rows, contiguous) into this warp's q buffer
+  uint32_t qwaits = 0;  // q copies waited for (barrier phase)
+  bool qpend = false;   // a q copy is in flight
+  auto copy_q = [&](const Item& v) {
+    qpend = v.valid;
+    if (lane == 0 && v.valid) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      mbar_arrive_tx(qbar, (uint32_t)(G * kD * 2));
+      bulk_load_1d(smem_u32(qbuf),
+                   static_cast<const uint16_t*>(a.q) + ((int64_t)v.s * a.num_q_heads + v.kvh * G) * kD,
+                   (uint32_t)(G * kD * 2), qbar);
+    }
+  };
+
+  Item cur = fetch();
+  Item nxt = fetch();
+  int cur_p, nxt_p;
+  float cur_ks, cur_vs, nxt_ks, nxt_vs;
+  load_window(cur, cur_p, cur_ks, cur_vs);
+  load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+  copy_q(cur);
+
+  int pslot = 0, pk = 0;
+  uint32_t g_iss = 0, g_cons = 0;
+  bool dead = false;
+  auto produce = [&]() {
+    while (!dead && g_iss - g_cons < (uint32_t)NST) {
+      if (pslot == 0 && pk >= cur.nblk) { pslot = 1; pk = 0; }
+      if (pslot == 1 && (!nxt.valid || pk >= nxt.nblk)) break;
+      const int kvh = pslot == 0 ? cur.kvh : nxt.kvh;
+      const int p = __shfl_sync(0xffffffffu, pslot == 0 ? cur_p : nxt_p, pk);
+      const int stage = g_iss % NST;
+      if (lane == 0) {
+        const uint32_t bar = bars + 8 * stage;
+        // the stage was last read (and maybe written) through the generic proxy
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        if (p >= 0) {
+          const int row = (p * Hkv + kvh) * C::kRows;
+          const uint32_t dst = wtiles + stage * STAGE;
+          mbar_arrive_tx(bar, STAGE);
+          tma_load_2d(dst, &kmap, 0, row, bar, policy);
+          tma_load_2d(dst + TILE, &vmap, 0, row, bar, policy);
+        } else {
+          mbar_arrive(bar);  // completes the phase; the consumer skips the block
+        }
+      }
+      ++g_iss;
+      ++pk;
+    }
+  };
+  produce();
+
+  uint32_t qf[8][2];
+  WarpAcc w;
+  while (cur.valid) {
+    if (!dead) {
+      if (mbar_wait(qbar, qwaits & 1)) {
+        ++qwaits;
+        qpend = false;
+      } else {
+        if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+        dead = true;
+      }
+    }
+    const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf), G, lane,
+                                           a.scale_log2, qf);
+    __syncwarp();
+    if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
+    w.reset();
+    for (int i = 0; i < cur.nblk; ++i) {
+      const int p = __shfl_sync(0xffffffffu, cur_p, i);
+      const float ks = __shfl_sync(0xffffffffu, cur_ks, i);
+      const float vs = __shfl_sync(0xffffffffu, cur_vs, i);
+      const int stage = g_cons % NST;
+      if (!dead && !mbar_wait(bars + 8 * stage, (g_cons / NST) & 1)) {
+        if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+        dead = true;
+      }
+      if (!dead && p >= 0) {
+        const uint32_t kt = wtiles + stage * STAGE;
+        tc_block<FP8>(kt, kt + TILE, min(kBS, cur.t1 - (cur.b_begin + i) * kBS), zscale * ks, vs,
+                      qf, w, lane);
+      }
+      __syncwarp();
+      ++g_cons;
+      produce();
+    }
+    // ---- item done: its output (single partition) or its partial ----
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      w.l0 += __shfl_xor_sync(0xffffffffu, w.l0, o);
+      w.l1 += __shfl_xor_sync(0xffffffffu, w.l1, o);
+    }
+    const float unit = FP8 ? w.vref : 1.f;
+    const int64_t row0 = (int64_t)cur.s * a.num_q_heads + cur.kvh * G;
+    const int g0 = 2 * tq, g1 = 2 * tq + 1;
+    const bool live0 = g0 < G, live1 = g1 < G;
+    const float ms[2] = {w.m0, w.m1}, ls[2] = {w.l0, w.l1};
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      int dA, dB;
+      if constexpr (FP8) {
+        dA = 32 * (t >> 1) + 2 * gq + (t & 1);
+        dB = dA + 16;
+      } else {
+        dA = 16 * t + gq;
+        dB = dA + 8;
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!(h == 0 ? live0 : live1)) continue;
+        const int64_t row = row0 + 2 * tq + h;
+        const float x0 = w.acc[t][h] * unit, x1 = w.acc[t][2 + h] * unit;
+        if (cur.np == 1) {
+          const float inv = ls[h] > 0.f ? 1.f / ls[h] : 0.f;
+          store_out(a.out, a.out_dtype, row * kD + dA, x0 * inv);
+          store_out(a.out, a.out_dtype, row * kD + dB, x1 * inv);
+        } else {
+          const int64_t pr = (row * a.max_parts + cur.part) * kD;
+          a.part_acc[pr + dA] = x0;
+          a.part_acc[pr + dB] = x1;
+        }
+      }
+    }
+    if (gq == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (!(h == 0 ? live0 : live1)) continue;
+        const int64_t row = row0 + 2 * tq + h;
+        if (cur.np == 1) {
+          if (a.lse_out != nullptr)
+            a.lse_out[row] = ls[h] > 0.f ? (ms[h] + __log2f(ls[h])) * kLn2 : -INFINITY;
+        } else {
+          const int64_t pr = row * a.max_parts + cur.part;
+          a.part_m[pr] = ms[h];
+          a.part_l[pr] = ls[h];
+        }
+      }
+    }
+    // ---- advance ----
+    cur = nxt;
+    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs;
+    nxt = fetch();
+    load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+    pslot = 0;
+    produce();
+  }
+  if (dead) {
+    // wait (bounded) for the copies this warp issued and did not consume
+    for (uint32_t j = g_cons; j < g_iss; ++j)
+      if (!mbar_wait(bars + 8 * (j % NST), (j / NST) & 1)) break;
+    if (qpend) mbar_wait(qbar, qwaits & 1);
   }
 }
 
@@ -486,7 +1093,7 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// The pool seen as rows of 128 bytes: a (block, head) tile is `rows` consecutive rows.
+// The pool seen as rows of 128 bytes: a (block, head) tile is kRows consecutive rows.
 inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dtype kv) {
   auto enc = encoder();
   if (enc == nullptr) return false;
@@ -502,22 +1109,67 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dt
   return r == CUDA_SUCCESS;
 }
 
+inline int sm_count() {
+  static int dev_cached = -1, sms = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev != dev_cached) {
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 0;
+    dev_cached = dev;
+  }
+  return sms;
+}
+
+// Tensor-core kernel families: grid of one CTA per item, persistent CTAs sharing an item,
+// persistent warp workers.
+enum TcKind { kTcGrid = 0, kTcCta = 1, kTcWarps = 2 };
+
+template <typename K>
+inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kernel, threads, smem);
+  if (e == cudaSuccess && *per_sm <= 0) e = cudaErrorInvalidConfiguration;
+  return e;
+}
+
 template <pa_dtype KV>
 inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
-                                cudaStream_t st) {
+                                const PlanView* pl, TcKind kind, cudaStream_t st) {
   using C = TcCfg<KV>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<KV>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * (C::kTile / 128);
+  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * C::kRows;
   CUtensorMap km, vm;
   if (!make_map(&km, a.k_cache, rows, KV) || !make_map(&vm, a.v_cache, rows, KV))
     return cudaErrorInvalidValue;
-  decode_tc_kernel<KV><<<grid, kNW * 32, C::kSmem, st>>>(a, km, vm);
+  if (kind == kTcGrid) {
+    static int per_sm = 0;
+    if (per_sm == 0) {
+      cudaError_t e = occupancy(decode_tc_kernel<KV>, kNW * 32, C::kSmem, &per_sm);
+      if (e != cudaSuccess) { per_sm = 0; return e; }
+    }
+    decode_tc_kernel<KV><<<grid, kNW * 32, C::kSmem, st>>>(a, km, vm);
+    return cudaGetLastError();
+  }
+  const int sms = sm_count();
+  if (sms <= 0 || pl == nullptr) return cudaErrorInvalidValue;
+  plan_kernel<<<1, 1024, 0, st>>>(a, *pl);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  if (kind == kTcCta) {
+    static int per_sm = 0;
+    if (per_sm == 0) {
+      e = occupancy(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, &per_sm);
+      if (e != cudaSuccess) { per_sm = 0; return e; }
+    }
+    decode_tc_persistent<KV><<<sms * per_sm, kNW * 32, C::kPSmem, st>>>(a, *pl, km, vm);
+  } else {
+    static int per_sm = 0;
+    if (per_sm == 0) {
+      e = occupancy(decode_tc_warps<KV>, kWW * 32, TcwCfg<KV>::kSmem, &per_sm);
+      if (e != cudaSuccess) { per_sm = 0; return e; }
+    }
+    decode_tc_warps<KV><<<sms * per_sm, kWW * 32, TcwCfg<KV>::kSmem, st>>>(a, *pl, km, vm);
+  }
   return cudaGetLastError();
 }
 
@@ -532,10 +1184,25 @@ inline bool tc_supported(const pa_decode_desc* d) {
   return rows < (int64_t)1 << 31;
 }
 
+// Which tensor-core kernel runs a call. impl: 2 = automatic, 3 = grid, 4 = persistent
+// CTAs, 5 = persistent warps. The persistent kernels need the split path (a workspace for
+// the plan) and keep one partition's blocks per warp in 32-entry register windows:
+// persistent CTAs up to 32 * 4 blocks (2048 tokens), warp workers up to 32 blocks (512).
+inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
+  const int P = d->partition_size;
+  const bool cta_ok = split && P <= 32 * tc::kNW * kBS;
+  const bool warps_ok = split && P <= 32 * kBS;
+  if (impl == 3) return tc::kTcGrid;
+  if (impl == 4) return cta_ok ? tc::kTcCta : tc::kTcGrid;
+  if (impl == 5) return warps_ok ? tc::kTcWarps : (cta_ok ? tc::kTcCta : tc::kTcGrid);
+  if (warps_ok) return tc::kTcWarps;
+  return cta_ok ? tc::kTcCta : tc::kTcGrid;
+}
+
 inline cudaError_t launch_tc(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
-                             cudaStream_t st) {
-  if (d->kv_dtype == PA_BF16) return tc::launch_tc_kv<PA_BF16>(a, d, grid, st);
-  return tc::launch_tc_kv<PA_FP8_E4M3>(a, d, grid, st);
+                             const tc::PlanView* pl, tc::TcKind kind, cudaStream_t st) {
+  if (d->kv_dtype == PA_BF16) return tc::launch_tc_kv<PA_BF16>(a, d, grid, pl, kind, st);
+  return tc::launch_tc_kv<PA_FP8_E4M3>(a, d, grid, pl, kind, st);
 }
 
 }  // namespace pa

@@ -16,8 +16,10 @@ inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Split-path workspace: plan area (counters, item list) followed by the partials
+// (m, l, acc) of every (seq, q head, partition).
 struct WorkspaceLayout {
-  size_t m_off, l_off, acc_off, total;
+  size_t cnt_off, list_off, m_off, l_off, acc_off, total;
   int parts;
 };
 
@@ -44,12 +46,14 @@ bool desc_supported(const pa_decode_desc* d) {
 }
 
 WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
-  WorkspaceLayout w{0, 0, 0, 0, 0};
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0};
   if (d->partition_size == 0 || max_context_len <= 0) return w;
   w.parts = (max_context_len + d->partition_size - 1) / d->partition_size;
   const size_t rows = (size_t)d->num_seqs * d->num_q_heads * w.parts;
-  w.m_off = 0;
-  w.l_off = round_up(rows * sizeof(float), 256);
+  w.cnt_off = 0;
+  w.list_off = 256;
+  w.m_off = w.list_off + round_up((size_t)d->num_seqs * w.parts * 8, 256);
+  w.l_off = w.m_off + round_up(rows * sizeof(float), 256);
   w.acc_off = w.l_off + round_up(rows * sizeof(float), 256);
   w.total = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
   return w;
@@ -107,7 +111,7 @@ extern "C" {
 const char* pa_version(void) { return "pagedattn 0.1 sm_100a"; }
 
 pa_status pa_set_decode_impl(int impl) {
-  if (impl < 0 || impl > 2) return PA_ERR_INVALID;
+  if (impl < 0 || impl > 5) return PA_ERR_INVALID;
   g_decode_impl = impl;
   return PA_OK;
 }
@@ -168,7 +172,15 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   const int gp = pad_group(a.group);
   cudaError_t e;
   if (g_decode_impl != 1 && tc_supported(desc)) {
-    e = launch_tc(a, desc, grid, st);
+    const tc::TcKind kind = tc_kind(desc, split, g_decode_impl);
+    tc::PlanView pl;
+    if (kind != tc::kTcGrid) {
+      char* ws = static_cast<char*>(workspace);
+      pl.counters = reinterpret_cast<uint32_t*>(ws + wl.cnt_off);
+      pl.list = reinterpret_cast<int2*>(ws + wl.list_off);
+      a.skip_single = 1;  // single-partition sequences are written by the kernel itself
+    }
+    e = launch_tc(a, desc, grid, kind == tc::kTcGrid ? nullptr : &pl, kind, st);
   } else {
     switch (desc->kv_dtype) {
       case PA_F32: e = launch_simt_d<PA_F32>(a, D, gp, grid, st); break;

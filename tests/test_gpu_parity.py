@@ -148,7 +148,10 @@ def test_tiny_workload(pa, scen, impl):
     assert offs == [4, 15, 0, 7]
 
 
-@pytest.mark.parametrize("impl", ["simt", "auto"])
+SPLIT_IMPLS = ["simt", "tc-grid", "tc-cta", "tc-warps"]
+
+
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("part", [0, 512])
 def test_batch32_workload(pa, scen, impl, part):
     _run_and_compare(pa, scen, workloads.draw("b32"), impl, partition_size=part)
@@ -171,7 +174,7 @@ def test_shared_prefix_workload(pa, scen, impl):
         pa.set_decode_impl("auto")
 
 
-@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("part", [512, 0])
 def test_batch256_fp8_full_size_sampled(pa, scen, impl, part):
     d = workloads.draw("b256")
@@ -180,15 +183,16 @@ def test_batch256_fp8_full_size_sampled(pa, scen, impl, part):
     _run_and_compare(pa, scen, d, impl, draw_seqs=sample, partition_size=part, check_cache=False)
 
 
-def test_long_context_full_size_sampled(pa, scen):
+@pytest.mark.parametrize("impl", ["auto", "tc-cta"])
+def test_long_context_full_size_sampled(pa, scen, impl):
     d = workloads.draw("long")
-    _run_and_compare(pa, scen, d, "auto", draw_seqs=[5], check_cache=False)
+    _run_and_compare(pa, scen, d, impl, draw_seqs=[5], check_cache=False)
 
 
 # ---------------------------------------------------------------------------------------
 # invariances, needles, closed forms, edge cases
 # ---------------------------------------------------------------------------------------
-@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512)])
 def test_physical_placement_bit_identical(pa, scen, impl, name, part):
     wl = workloads.WORKLOADS[name].scaled(num_seqs=6)
@@ -208,7 +212,7 @@ def test_physical_placement_bit_identical(pa, scen, impl, name, part):
         pa.set_decode_impl("auto")
 
 
-@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("name,part,lens", [
     ("b32", 0, [1, 2, 15, 16, 17, 31, 33, 4096]),
     ("b32", 512, [511, 512, 513, 1024, 1025, 3000]),
@@ -238,7 +242,7 @@ def test_zero_query_is_mean_of_values(pa, scen, impl):
         assert np.allclose(to_f64(sc.lse)[s], math.log(d.context_lens[s]), atol=1e-3)
 
 
-@pytest.mark.parametrize("impl", ["simt", "auto"])
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("hq,hkv,dim,kv", [(8, 8, 128, "bf16"), (16, 8, 128, "bf16"),
                                             (64, 4, 128, "bf16"), (16, 2, 64, "bf16"),
                                             (8, 1, 256, "bf16"), (32, 8, 128, "fp8"),
@@ -248,7 +252,7 @@ def test_head_shapes(pa, scen, impl, hq, hkv, dim, kv):
     in_dt = "f32" if kv == "f32" else "bf16"
     wl = workloads.Workload("shape", 9, 5, hq, hkv, dim, 16, 512, kv, in_dt,
                             ("fixed", [1, 17, 100, 700, 1500]))
-    for part in (0, 256):
+    for part in (0, 256, 1024):
         _run_and_compare(pa, scen, workloads.draw(wl), impl, partition_size=part)
 
 
@@ -273,11 +277,14 @@ def test_empty_context_and_error_flags(pa):
         assert torch.all(torch.isneginf(lse[0])) and torch.all(torch.isfinite(lse[1]))
     # an out-of-range block id is skipped and flagged, never dereferenced
     bad = torch.tensor([[0, 1_000_000], [2, -1], [3, 4]], dtype=torch.int32, device="cuda")
-    pa.paged_attn_decode(q, kc, vc, bad, torch.tensor([20, 5, 30], dtype=torch.int32,
-                                                      device="cuda"),
-                         0.1, out, max_context_len=32)
-    assert pa.device_error() & pa.PA_DEVERR_BLOCK_ID
-    assert pa.device_error() == 0
+    for part in (0, 16):
+        ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+        pa.paged_attn_decode(q, kc, vc, bad, torch.tensor([20, 5, 30], dtype=torch.int32,
+                                                          device="cuda"),
+                             0.1, out, max_context_len=32, partition_size=part, workspace=ws)
+        assert pa.device_error() & pa.PA_DEVERR_BLOCK_ID
+        assert pa.device_error() == 0
+        assert torch.isfinite(out[2].float()).all()
     # a context longer than max_context_len is clamped and flagged
     pa.paged_attn_decode(q, kc, vc, bt, torch.tensor([20, 5, 40], dtype=torch.int32,
                                                      device="cuda"),
