@@ -435,7 +435,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="b256", choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--decode-impl", default="auto", choices=["auto", "simt", "tc"])
+    ap.add_argument("--decode-impl", default="auto",
+                    choices=["auto", "simt", "tc", "tc-grid", "tc-cta", "tc-warps"])
     ap.add_argument("--partition", type=int, default=None,
                     help="split-KV partition in tokens (default: the workload's)")
     ap.add_argument("--no-extra", dest="extra", action="store_false",
