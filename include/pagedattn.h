@@ -124,6 +124,38 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
                             void* stream);
 
 /*
+ * Largest workspace (bytes) that paged_attn_decode_noalloc can serve from its fixed device
+ * array: 32 MiB.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/*
+ * paged_attn_decode for callers that cannot allocate device memory. Some callers may not
+ * call cudaMalloc at all: code running while a stream is being captured, a plugin inside a
+ * host runtime that owns every device allocation through its own allocator, a caller with
+ * no workspace argument to forward. This entry point takes the same arguments as
+ * paged_attn_decode minus the workspace and computes the same result; the split-KV scratch
+ * comes from one fixed array compiled into this library (PA_NOALLOC_SCRATCH_BYTES per GPU,
+ * held by every GPU that loads the library until the process exits). The pages have no
+ * counterpart of this call; it exists only for such callers.
+ * - Calls that need more scratch than PA_NOALLOC_SCRATCH_BYTES
+ *   (paged_attn_workspace_size(desc, max_context_len) larger than it) return
+ *   PA_ERR_WORKSPACE and enqueue nothing.
+ * - The first call on a device looks the array's device address up (once per device, with
+ *   that device current); make that first call before any stream capture.
+ * - It calls no cudaMalloc, cudaFree or other allocating routine.
+ * - Every call on a device shares the one array, which keeps the last call's contents. The
+ *   kernels re-initialise what they read (work counter, partials) on every call, so stale
+ *   contents never matter; but calls that overlap on the GPU (different streams, or
+ *   different host threads) race on the array: serialise them.
+ */
+pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, const int32_t* context_lens,
+                                    float scale, void* out, const pa_decode_desc* desc,
+                                    int max_context_len, const float* k_scales,
+                                    const float* v_scales, float* lse_out, void* stream);
+
+/*
  * Slot-mapped write of new tokens' K and V into the pool ([KVPaged] "PagedAttention: OS
  * virtual-memory style management": one block is allocated as tokens accumulate and the
  * block table maps logical positions to physical blocks). For token t with

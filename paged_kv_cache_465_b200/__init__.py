@@ -63,6 +63,8 @@ _SIGS = {
     "paged_attn_workspace_size": (_sz, [_P(pa_decode_desc), _i]),
     "paged_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i, _vp,
                                _vp, _vp, _vp, _sz, _vp]),
+    "paged_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i,
+                                       _vp, _vp, _vp, _vp]),
     "reshape_and_cache": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _i, _i, _i, _i,
                                _vp, _vp, _vp]),
     "copy_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
@@ -203,6 +205,29 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: fl
     if st == PA_ERR_WORKSPACE:
         raise PagedAttnError(st, f"paged_attn_decode needs {ws_need} workspace bytes")
     _check(st, "paged_attn_decode")
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 32 << 20
+
+
+def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float,
+                              out, *, max_context_len: int, partition_size: int = 0,
+                              k_scales=None, v_scales=None, lse_out=None, stream=None):
+    """paged_attn_decode without a caller workspace: the split-KV scratch comes from a fixed
+    array inside the library (at most NOALLOC_SCRATCH_BYTES per GPU), for callers that
+    cannot allocate device memory. Overlapping calls on one GPU race on that array."""
+    torch = _torch()
+    desc = decode_desc_for(q, k_cache, block_tables, partition_size)
+    if tuple(out.shape) != tuple(q.shape) or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    st = _lib.paged_attn_decode_noalloc(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32), _dev(context_lens, "context_lens", torch.int32),
+        ctypes.c_float(scale), _dev(out, "out"), ctypes.byref(desc), int(max_context_len),
+        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(lse_out, "lse_out", torch.float32), _stream(stream))
+    _check(st, "paged_attn_decode_noalloc")
     return out
 
 

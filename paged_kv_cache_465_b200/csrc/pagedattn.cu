@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <mutex>
 
 #include "common.cuh"
 #include "cache_ops.cuh"
@@ -258,6 +259,47 @@ pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_sc
       num_blocks);
   PA_CHECK_LAUNCH();
   return PA_OK;
+}
+
+// ---------------------------------------------------------------------------------------
+// Allocation-free decode: the split-KV scratch lives in one fixed array of this library's
+// device image. In host code `g_noalloc_scratch` names a host-side stand-in, not device
+// memory, so it is never passed to a kernel: the device address is looked up with
+// cudaGetSymbolAddress, once per device, with that device current.
+// ---------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+constexpr int kMaxDevices = 128;
+void* g_noalloc_ptr[kMaxDevices];
+std::mutex g_noalloc_mu;
+}  // namespace
+
+pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
+                                    const int32_t* block_tables, const int32_t* context_lens,
+                                    float scale, void* out, const pa_decode_desc* desc,
+                                    int max_context_len, const float* k_scales,
+                                    const float* v_scales, float* lse_out, void* stream) {
+  if (!desc_ok(desc) || max_context_len < 0) return PA_ERR_INVALID;
+  const size_t need = paged_attn_workspace_size(desc, max_context_len);
+  if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return PA_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    ws = g_noalloc_ptr[dev];
+  }
+  return paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, desc,
+                           max_context_len, k_scales, v_scales, lse_out, ws,
+                           ws ? (size_t)PA_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
 
 pa_status pa_device_error(int* bits_out, void* stream) {
