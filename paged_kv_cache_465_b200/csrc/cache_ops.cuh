@@ -37,6 +37,8 @@ __global__ void reshape_and_cache_kernel(const void* __restrict__ k, const void*
                                          int head_dim, int block_size, int num_blocks,
                                          const float* __restrict__ k_scales,
                                          const float* __restrict__ v_scales) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int64_t slot = slot_mapping[t];
   if (slot < 0) return;  // padding token
@@ -85,6 +87,8 @@ __global__ void copy_blocks_kernel(uint8_t* __restrict__ k_cache, uint8_t* __res
                                    float* __restrict__ k_scales, float* __restrict__ v_scales,
                                    const int32_t* __restrict__ pairs, int64_t block_bytes,
                                    int num_kv_heads, int num_blocks) {
+  pdl_wait();
+  pdl_trigger();
   const int i = blockIdx.x;
   const bool is_v = blockIdx.y == 1;
   const int src = pairs[2 * i], dst = pairs[2 * i + 1];

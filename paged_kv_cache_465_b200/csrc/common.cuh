@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "pagedattn.h"
 
 namespace pa {
@@ -65,6 +67,16 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start before its predecessor in the stream finishes; it must wait here before it
+// reads anything the predecessor (or earlier work) wrote. No-op for ordinary launches.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Lets the next kernel in the stream (launched with programmatic serialization) be
+// scheduled; it still waits for this grid's completion in its own pdl_wait().
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -72,6 +84,23 @@ constexpr float kLn2 = 0.6931471805599453f;
 inline int dtype_bytes(pa_dtype t) { return t == PA_F32 ? 4 : (t == PA_BF16 ? 2 : 1); }
 
 }  // namespace pa
+
+// Launch with programmatic stream serialization (the kernel must call pdl_wait() first).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 #define PA_CHECK_LAUNCH()                                  \
   do {                                                     \

@@ -298,77 +298,145 @@ decode_simt_kernel(const DecodeArgs a) {
   }
 }
 
-// Log-sum-exp merge of the partitions of one (sequence, query head): grid (Hq, S), 128
-// threads. Pass 1: M = max_p m_p (block reduction); pass 2: w_p = 2^(m_p - M) into shared
-// memory and L = sum_p w_p l_p; pass 3: out = sum_p w_p acc_p / L with every thread owning
-// 4 channels and one of 512/D interleaved partition groups (independent loads in flight),
-// the groups then added in a fixed order. The order depends only on partition indices, so
-// the result is deterministic and independent of physical block placement.
+// Log-sum-exp merge of the partitions of each (sequence, query head), one warp per row:
+// 4 rows per CTA of 128 threads, grid ceil(S * Hq / 4). Lane p holds partition p's max and
+// sum (32 partitions at a time): M = max_p m_p and L = sum_p 2^(m_p - M) l_p by shuffles;
+// every lane owns float4 channel quads and accumulates sum_p 2^(m_p - M) acc_p in partition
+// order. The order depends only on partition indices, so the result is deterministic and
+// independent of physical block placement.
 template <int D>
 __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
-  constexpr int QUADS = D / 4;           // float4 columns of one partial row
-  constexpr int NG = 128 / QUADS;        // partition groups (4 at D=128)
-  constexpr int CHUNK = 2048;            // weights held in shared memory at a time
-  __shared__ float sw[CHUNK];
-  __shared__ float red[32];
-  __shared__ float part[NG][D];
+  constexpr int QUADS = D / 4;
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int64_t rowid = (int64_t)blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (rowid >= (int64_t)a.num_seqs * a.num_q_heads) return;
+  const int s = (int)(rowid / a.num_q_heads);
+  const int ctx = checked_ctx(a, s);
+  const int np = (ctx + a.part_tokens - 1) / a.part_tokens;
+  if (a.skip_single && np <= 1) return;
+  const int64_t row = rowid;
+  const float* pm = a.part_m + row * a.max_parts;
+  const float* pl = a.part_l + row * a.max_parts;
+  const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * D);
+
+  float M = -INFINITY;
+  for (int p = lane; p < np; p += 32) M = fmaxf(M, pm[p]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+
+  constexpr int NQ = (QUADS + 31) / 32;  // quads per lane
+  float4 acc[NQ];
+#pragma unroll
+  for (int j = 0; j < NQ; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lsum = 0.f;
+  for (int c0 = 0; c0 < np; c0 += 32) {
+    const int p = c0 + lane;
+    const float w = (p < np && M != -INFINITY) ? fast_exp2(pm[p] - M) : 0.f;
+    if (p < np) lsum = fmaf(w, pl[p], lsum);
+    const int n = min(32, np - c0);
+#pragma unroll 4
+    for (int k = 0; k < n; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float4* src = pacc + (int64_t)(c0 + k) * QUADS;
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const int q = lane + 32 * j;
+        if (q < QUADS) {
+          const float4 v = __ldg(src + q);
+          acc[j].x = fmaf(wk, v.x, acc[j].x); acc[j].y = fmaf(wk, v.y, acc[j].y);
+          acc[j].z = fmaf(wk, v.z, acc[j].z); acc[j].w = fmaf(wk, v.w, acc[j].w);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll
+  for (int j = 0; j < NQ; ++j) {
+    const int q = lane + 32 * j;
+    if (q < QUADS) {
+      const int64_t o = row * D + 4 * q;
+      store_out(a.out, a.out_dtype, o, acc[j].x * inv);
+      store_out(a.out, a.out_dtype, o + 1, acc[j].y * inv);
+      store_out(a.out, a.out_dtype, o + 2, acc[j].z * inv);
+      store_out(a.out, a.out_dtype, o + 3, acc[j].w * inv);
+    }
+  }
+  if (lane == 0 && a.lse_out != nullptr)
+    a.lse_out[row] = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
+}
+
+// Same merge for rows with many partitions: one CTA of 4 warps per (sequence, query head),
+// grid (Hq, S). Warp w takes the 32-partition chunks c with c % 4 == w (in order); the
+// four warps' sums are added in warp order, so the order again depends only on partition
+// indices.
+template <int D>
+__global__ void __launch_bounds__(128) lse_reduce_block_kernel(const DecodeArgs a) {
+  constexpr int QUADS = D / 4;
+  constexpr int NQ = (QUADS + 31) / 32;
+  __shared__ float sm_max[4], sm_l[4];
+  __shared__ __align__(16) float sm_acc[4][D];
+  pdl_wait();
   const int h = blockIdx.x, s = blockIdx.y;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ctx = checked_ctx(a, s);
   const int np = (ctx + a.part_tokens - 1) / a.part_tokens;
   if (a.skip_single && np <= 1) return;
   const int64_t row = (int64_t)s * a.num_q_heads + h;
   const float* pm = a.part_m + row * a.max_parts;
   const float* pl = a.part_l + row * a.max_parts;
-  const float* pacc = a.part_acc + row * a.max_parts * D;
+  const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * D);
 
-  float mx = -INFINITY;
-  for (int p = tid; p < np; p += 128) mx = fmaxf(mx, pm[p]);
+  float M = -INFINITY;
+  for (int p = threadIdx.x; p < np; p += 128) M = fmaxf(M, pm[p]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  if (lane == 0) red[warp] = mx;
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) sm_max[warp] = M;
   __syncthreads();
-  const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-  __syncthreads();
+  M = fmaxf(fmaxf(sm_max[0], sm_max[1]), fmaxf(sm_max[2], sm_max[3]));
 
-  const int q = tid % QUADS, grp = tid / QUADS;
+  float4 acc[NQ];
+#pragma unroll
+  for (int j = 0; j < NQ; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
   float lsum = 0.f;
-  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int c0 = 0; c0 < np; c0 += CHUNK) {
-    const int n = min(CHUNK, np - c0);
-    for (int p = tid; p < n; p += 128) {
-      const float w = M == -INFINITY ? 0.f : fast_exp2(pm[c0 + p] - M);
-      sw[p] = w;
-      lsum = fmaf(w, pl[c0 + p], lsum);
-    }
-    __syncthreads();
-    const float4* src = reinterpret_cast<const float4*>(pacc + (int64_t)c0 * D) + q;
+  for (int c0 = 32 * warp; c0 < np; c0 += 128) {
+    const int p = c0 + lane;
+    const float w = (p < np && M != -INFINITY) ? fast_exp2(pm[p] - M) : 0.f;
+    if (p < np) lsum = fmaf(w, pl[p], lsum);
+    const int n = min(32, np - c0);
 #pragma unroll 4
-    for (int p = grp; p < n; p += NG) {
-      const float w = sw[p];
-      const float4 v = __ldg(src + (int64_t)p * QUADS);
-      acc.x = fmaf(w, v.x, acc.x); acc.y = fmaf(w, v.y, acc.y);
-      acc.z = fmaf(w, v.z, acc.z); acc.w = fmaf(w, v.w, acc.w);
+    for (int k = 0; k < n; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float4* src = pacc + (int64_t)(c0 + k) * QUADS;
+#pragma unroll
+      for (int j = 0; j < NQ; ++j) {
+        const int q = lane + 32 * j;
+        if (q < QUADS) {
+          const float4 v = __ldg(src + q);
+          acc[j].x = fmaf(wk, v.x, acc[j].x); acc[j].y = fmaf(wk, v.y, acc[j].y);
+          acc[j].z = fmaf(wk, v.z, acc[j].z); acc[j].w = fmaf(wk, v.w, acc[j].w);
+        }
+      }
     }
-    __syncthreads();
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  if (lane == 0) red[8 + warp] = lsum;
-  part[grp][4 * q] = acc.x;
-  part[grp][4 * q + 1] = acc.y;
-  part[grp][4 * q + 2] = acc.z;
-  part[grp][4 * q + 3] = acc.w;
-  __syncthreads();
-  const float L = (red[8] + red[9]) + (red[10] + red[11]);
-  if (tid < D) {
-    float A = 0.f;
+  if (lane == 0) sm_l[warp] = lsum;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) A += part[g][tid];
-    store_out(a.out, a.out_dtype, row * D + tid, L > 0.f ? A / L : 0.f);
-    if (tid == 0 && a.lse_out != nullptr)
-      a.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+  for (int j = 0; j < NQ; ++j) {
+    const int q = lane + 32 * j;
+    if (q < QUADS) reinterpret_cast<float4*>(sm_acc[warp])[q] = acc[j];
   }
+  __syncthreads();
+  const float L = ((sm_l[0] + sm_l[1]) + sm_l[2]) + sm_l[3];
+  for (int d = threadIdx.x; d < D; d += 128) {
+    const float A = ((sm_acc[0][d] + sm_acc[1][d]) + sm_acc[2][d]) + sm_acc[3][d];
+    store_out(a.out, a.out_dtype, row * D + d, L > 0.f ? A / L : 0.f);
+  }
+  if (threadIdx.x == 0 && a.lse_out != nullptr)
+    a.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace pa

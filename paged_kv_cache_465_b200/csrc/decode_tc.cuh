@@ -570,7 +570,7 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
 }
 
 // =======================================================================================
-// Split path: plan kernel + persistent kernel with the log-sum-exp merge fused in.
+// Split path: plan kernel + persistent kernels; lse_reduce_kernel merges the partitions.
 // =======================================================================================
 // Workspace of the split path (offsets in bytes, each region 256-aligned):
 //   [0]     uint32 fetch counter, uint32 total items
@@ -588,6 +588,8 @@ struct PlanView {
 // fetch counter, and writes out = 0 / lse = -inf for empty sequences.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
   __shared__ int cnt[130], off[130];
+  pdl_wait();
+  pdl_trigger();
   const int P = a.part_tokens;
   const int nbk = P / kBS;  // blocks of a full partition (<= 128)
   for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
@@ -656,6 +658,7 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
   const uint32_t wtiles = smem_u32(smem + warp * NST * STAGE);
   const uint32_t bars = smem_u32(barmem) + warp * NST * 8;
   const uint32_t qbars = smem_u32(barmem + kNW * NST);
+  pdl_wait();  // the plan kernel's list and counters
   const uint32_t total = pl.counters[1];
   const uint64_t policy = evict_first_policy();
 
@@ -831,7 +834,7 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
 // Partitions of at most 512 tokens (32 blocks: one register window per item).
 // =======================================================================================
 #ifndef PA_TCW_WARPS
-#define PA_TCW_WARPS 2
+#define PA_TCW_WARPS 1
 #endif
 #ifndef PA_TCW_STAGE_BF16
 #define PA_TCW_STAGE_BF16 3
@@ -878,6 +881,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncwarp();
+  pdl_wait();  // the plan kernel's list and counters
   const uint32_t total = pl.counters[1];
   const uint64_t policy = evict_first_policy();
 
@@ -1067,6 +1071,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     pslot = 0;
     produce();
   }
+  pdl_trigger();  // no more items: the reduce may be scheduled (it waits for this grid)
   if (dead) {
     // wait (bounded) for the copies this warp issued and did not consume
     for (uint32_t j = g_cons; j < g_iss; ++j)
@@ -1152,8 +1157,7 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   }
   const int sms = sm_count();
   if (sms <= 0 || pl == nullptr) return cudaErrorInvalidValue;
-  plan_kernel<<<1, 1024, 0, st>>>(a, *pl);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, a, *pl);
   if (e != cudaSuccess) return e;
   if (kind == kTcCta) {
     static int per_sm = 0;
@@ -1161,14 +1165,18 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
       e = occupancy(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, &per_sm);
       if (e != cudaSuccess) { per_sm = 0; return e; }
     }
-    decode_tc_persistent<KV><<<sms * per_sm, kNW * 32, C::kPSmem, st>>>(a, *pl, km, vm);
+    e = launch_pdl(decode_tc_persistent<KV>, dim3(sms * per_sm), dim3(kNW * 32), C::kPSmem, st,
+                   a, *pl, km, vm);
+    if (e != cudaSuccess) return e;
   } else {
     static int per_sm = 0;
     if (per_sm == 0) {
       e = occupancy(decode_tc_warps<KV>, kWW * 32, TcwCfg<KV>::kSmem, &per_sm);
       if (e != cudaSuccess) { per_sm = 0; return e; }
     }
-    decode_tc_warps<KV><<<sms * per_sm, kWW * 32, TcwCfg<KV>::kSmem, st>>>(a, *pl, km, vm);
+    e = launch_pdl(decode_tc_warps<KV>, dim3(sms * per_sm), dim3(kWW * 32), TcwCfg<KV>::kSmem,
+                   st, a, *pl, km, vm);
+    if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
 }

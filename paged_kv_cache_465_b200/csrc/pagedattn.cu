@@ -92,14 +92,24 @@ cudaError_t launch_simt_d(const DecodeArgs& a, int D, int gp, dim3 grid, cudaStr
   }
 }
 
+// Rows with up to 32 partitions: one warp per row; more: one CTA of 4 warps per row.
 cudaError_t launch_reduce(const DecodeArgs& a, int D, cudaStream_t st) {
-  dim3 grid(a.num_q_heads, a.num_seqs);
-  switch (D) {
-    case 64: lse_reduce_kernel<64><<<grid, 128, 0, st>>>(a); break;
-    case 128: lse_reduce_kernel<128><<<grid, 128, 0, st>>>(a); break;
-    default: lse_reduce_kernel<256><<<grid, 128, 0, st>>>(a); break;
+  const dim3 block(128);
+  if (a.max_parts > 32) {
+    const dim3 grid(a.num_q_heads, a.num_seqs);
+    switch (D) {
+      case 64: return launch_pdl(lse_reduce_block_kernel<64>, grid, block, 0, st, a);
+      case 128: return launch_pdl(lse_reduce_block_kernel<128>, grid, block, 0, st, a);
+      default: return launch_pdl(lse_reduce_block_kernel<256>, grid, block, 0, st, a);
+    }
   }
-  return cudaGetLastError();
+  const int64_t rows = (int64_t)a.num_seqs * a.num_q_heads;
+  const dim3 grid((unsigned)((rows + 3) / 4));
+  switch (D) {
+    case 64: return launch_pdl(lse_reduce_kernel<64>, grid, block, 0, st, a);
+    case 128: return launch_pdl(lse_reduce_kernel<128>, grid, block, 0, st, a);
+    default: return launch_pdl(lse_reduce_kernel<256>, grid, block, 0, st, a);
+  }
 }
 
 }  // namespace
@@ -217,12 +227,11 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
   const cudaStream_t st = as_stream(stream);
   const dim3 grid(num_tokens);
   const int threads = 128;
-#define PA_RC(IN, C)                                                                         \
-  reshape_and_cache_kernel<IN, C><<<grid, threads, 0, st>>>(k, v, k_cache, v_cache,           \
-                                                            slot_mapping, k_stride, v_stride, \
-                                                            num_kv_heads, head_dim,           \
-                                                            block_size, num_blocks, k_scales, \
-                                                            v_scales)
+  cudaError_t e = cudaSuccess;
+#define PA_RC(IN, C)                                                                          \
+  e = launch_pdl(reshape_and_cache_kernel<IN, C>, grid, dim3(threads), 0, st, k, v, k_cache,  \
+                 v_cache, slot_mapping, k_stride, v_stride, num_kv_heads, head_dim,          \
+                 block_size, num_blocks, k_scales, v_scales)
   if (in_dtype == PA_F32) {
     if (cache_dtype == PA_F32) PA_RC(PA_F32, PA_F32);
     else if (cache_dtype == PA_BF16) PA_RC(PA_F32, PA_BF16);
@@ -234,8 +243,7 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
     else return PA_ERR_UNSUPPORTED;
   }
 #undef PA_RC
-  PA_CHECK_LAUNCH();
-  return PA_OK;
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_scales,
@@ -252,13 +260,13 @@ pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_sc
   const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * dtype_bytes(cache_dtype);
   if (block_bytes % 16 != 0) return PA_ERR_INVALID;
   if (cache_dtype == PA_FP8_E4M3 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
-  copy_blocks_kernel<<<dim3(num_pairs, 2), 256, 0, as_stream(stream)>>>(
+  const cudaError_t e = launch_pdl(
+      copy_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, as_stream(stream),
       static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
       cache_dtype == PA_FP8_E4M3 ? k_scales : nullptr,
       cache_dtype == PA_FP8_E4M3 ? v_scales : nullptr, pairs, block_bytes, num_kv_heads,
       num_blocks);
-  PA_CHECK_LAUNCH();
-  return PA_OK;
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------------------

@@ -170,7 +170,9 @@ def test_host_validation_without_device(pa):
                                  pa.PA_F32, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_INVALID
     assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 3, 128, 128, 2, 64, 16, 32,
                                  pa.PA_BF16, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_UNSUPPORTED
-    assert lib.pa_set_decode_impl(3) == pa.PA_ERR_INVALID
+    assert lib.pa_set_decode_impl(6) == pa.PA_ERR_INVALID
+    assert lib.pa_set_decode_impl(-1) == pa.PA_ERR_INVALID
+    assert lib.pa_set_decode_impl(0) == pa.PA_OK
 
 
 def test_binding_refuses_host_tensors(pa):
