@@ -316,7 +316,7 @@ def run_ours(args):
         "gpu_launches": sc.launches_per_step() * args.steps,
         "clocks": clk.summary(t_wall0, t_wall1),
     }
-    traffic = _traffic_note(args.workload)
+    traffic = _traffic_note(args.workload, pa.version())
     if traffic is not None:
         result["roofline"]["traffic"] = traffic
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -330,16 +330,16 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def _traffic_note(name):
-    """Per-launch DRAM bytes of the dominant kernel from the committed ncu summary, if one
-    matches the current kernel build (profiles/traffic.json); else None."""
+def _traffic_note(name, version):
+    """DRAM bytes of one decode call from the committed ncu summary (profiles/traffic.json)
+    when it was taken on this exact library build; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     e = j.get(name)
-    if not e:
+    if not e or j.get("version") != version:
         return None
     return e.get("bytes_per_launch")
 
