@@ -35,13 +35,15 @@ METRIC = "paged decode attention KV GB/s (% of HBM peak) and decode tokens/s at 
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
-DTYPE = {"f32": "f32", "bf16": "bf16-kv/f32-acc", "fp8": "fp8e4m3-kv/f32-acc"}
+DTYPE = {"f32": "f32", "bf16": "bf16-kv/f32-acc", "fp8": "fp8e4m3-kv/f32-acc",
+         "int8": "int8-kv/f32-acc"}
 DESCR = {
     "tiny": "tiny paged decode: 4 seqs ctx {5,16,17,40}, 4q/2kv, d64, fp32",
     "b32": "decode batch 32: ctx U[1,4096], 32q/8kv, d128, bf16 KV",
     "shared": "shared prefix: 100 seqs x (200 shared + 50 private), 32q/8kv, d128, bf16, CoW",
     "b256": "decode batch 256: ctx lognormal(1024,1) clip [16,8192], 32q/8kv, d128, fp8-e4m3 KV",
     "long": "long context: 8 seqs x 131072, 64q/8kv, d128, bf16 KV, split-KV 512",
+    "b256_int8": "decode batch 256 with an int8 KV cache (scale + zero point per block, kv head)",
 }
 
 
@@ -195,7 +197,7 @@ def _cpu_baseline(draw, seconds: float = 12.0):
     sample = sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, 8), replace=False).tolist())
     st = flows.build_state(draw, write_seqs=sample)
     sc = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
-    es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+    es = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[wl.kv_dtype]
     done_bytes = 0
     t0 = time.perf_counter()
     i = 0
@@ -203,10 +205,11 @@ def _cpu_baseline(draw, seconds: float = 12.0):
         s = sample[i % len(sample)]
         k, v = draw.kv(s)
         opaged.ref_reshape_and_cache(k[-1:], v[-1:], st.k_cache, st.v_cache, st.step_slots[s],
-                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales)
+                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales,
+                                     st.k_zeros, st.v_zeros)
         attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                              sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype, st.k_scales,
-                             st.v_scales, seqs=[s])
+                             st.v_scales, seqs=[s], k_zeros=st.k_zeros, v_zeros=st.v_zeros)
         done_bytes += int(draw.context_lens[s]) * 2 * wl.num_kv_heads * wl.head_dim * es
         i += 1
         el = time.perf_counter() - t0
@@ -348,11 +351,12 @@ def _extra_workloads(torch, pa, args, flush):
     from paged_kv_cache_465_b200.scenario import DeviceScenario
     peak, _ = _peaks()
     out = {}
-    for name in ("tiny", "b32", "shared", "b256", "long"):
+    for name in ("tiny", "b32", "shared", "b256", "long", "b256_int8"):
         if name == args.workload:
             continue
         draw = workloads.draw(name)
-        sc = DeviceScenario(draw, draw_seqs=[] if name in ("b256", "long", "b32") else None)
+        sc = DeviceScenario(draw, draw_seqs=[] if name in ("b256", "long", "b32", "b256_int8")
+                            else None)
         for _ in range(3):
             flush()
             sc.step()
@@ -387,7 +391,7 @@ def run_reference(args):
     sample = sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, 8), replace=False).tolist())
     st = flows.build_state(draw, write_seqs=sample)
     sc = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
-    es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+    es = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[wl.kv_dtype]
     try:
         from threadpoolctl import threadpool_info
         cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
@@ -398,10 +402,11 @@ def run_reference(args):
         s = sample[i % len(sample)]
         k, v = draw.kv(s)
         opaged.ref_reshape_and_cache(k[-1:], v[-1:], st.k_cache, st.v_cache, st.step_slots[s],
-                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales)
+                                     wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales,
+                                     st.k_zeros, st.v_zeros)
         attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
                              sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype, st.k_scales,
-                             st.v_scales, seqs=[s])
+                             st.v_scales, seqs=[s], k_zeros=st.k_zeros, v_zeros=st.v_zeros)
         return int(draw.context_lens[s]) * 2 * wl.num_kv_heads * wl.head_dim * es
 
     for i in range(args.warmup):

@@ -29,7 +29,11 @@
  * - Cache layout: cache[num_blocks][num_kv_heads][block_size][head_dim], row-major, so each
  *   (physical block, kv head) tile is contiguous (the pages give no layout; this is the
  *   library's choice). fp8 caches carry float32 scales[num_blocks][num_kv_heads], one per
- *   (block, kv head), separately for K and V: stored value = E4M3(x / scale).
+ *   (block, kv head), separately for K and V: stored value = E4M3(x / scale). int8 caches
+ *   ([KVPaged] "KV quantization: FP8 and INT8": one byte per element with a scale and a
+ *   zero point) carry the same scales plus int32 zero points[num_blocks][num_kv_heads]:
+ *   stored code = clamp(round_half_even(x / scale) + zero, -128, 127), value =
+ *   (code - zero) * scale.
  * - q and out: [num_seqs][num_q_heads][head_dim] row-major. Query head h reads kv head
  *   h / (num_q_heads / num_kv_heads) ([KVPaged] "GQA and MQA": query heads are grouped and
  *   each group shares one KV head).
@@ -42,7 +46,8 @@
  *
  * Supported today: block_size 16; head_dim 64, 128 or 256; num_q_heads a multiple of
  * num_kv_heads with a group of at most 16; (q, kv, out) dtypes (f32, f32, f32),
- * (bf16, bf16, bf16) and (bf16, fp8_e4m3, bf16). Anything else returns PA_ERR_UNSUPPORTED.
+ * (bf16, bf16, bf16), (bf16, fp8_e4m3, bf16) and (bf16, int8, bf16). Anything else returns
+ * PA_ERR_UNSUPPORTED.
  */
 #ifndef PAGEDATTN_H_
 #define PAGEDATTN_H_
@@ -54,7 +59,7 @@
 extern "C" {
 #endif
 
-typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2, PA_INT8 = 3 } pa_dtype;
 
 typedef enum {
   PA_OK = 0,
@@ -102,7 +107,8 @@ size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len
  * with g = h / (Hq/Hkv) and the cached tokens t < context_lens[s]:
  *     z_t = scale * q[s][h] . K_t,   out[s][h] = sum_t softmax(z)_t V_t,
  *     lse_out[s][h] = log sum_t exp(z_t)                    (natural log, float32)
- * fp8 caches are dequantised as E4M3 value * scales[block][g]. Accumulation is float32.
+ * fp8 caches are dequantised as E4M3 value * scales[block][g], int8 caches as
+ * (code - zeros[block][g]) * scales[block][g]. Accumulation is float32.
  * With partition_size > 0 the context is cut into partitions of that many logical tokens,
  * each reduced to (max, sum, unnormalised output) in `workspace`, then combined by a
  * log-sum-exp reduction; the result does not depend on where blocks sit physically.
@@ -110,7 +116,8 @@ size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len
  *   k_cache/v_cache pool in desc->kv_dtype (layout above)
  *   block_tables   int32 [S][max_blocks_per_seq];  context_lens int32 [S]
  *   max_context_len  host int >= every context_lens entry (sizes the grid)
- *   k_scales/v_scales float32 [num_blocks][Hkv], required for fp8, ignored otherwise
+ *   k_scales/v_scales float32 [num_blocks][Hkv], required for fp8 and int8, else ignored
+ *   k_zeros/v_zeros  int32 [num_blocks][Hkv], required for int8, ignored otherwise
  *   lse_out        float32 [S][Hq] or NULL
  *   workspace      device bytes, >= paged_attn_workspace_size(desc, max_context_len),
  *                  16-byte aligned; may be NULL when that size is 0
@@ -120,8 +127,8 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
                             const int32_t* block_tables, const int32_t* context_lens,
                             float scale, void* out, const pa_decode_desc* desc,
                             int max_context_len, const float* k_scales, const float* v_scales,
-                            float* lse_out, void* workspace, size_t workspace_bytes,
-                            void* stream);
+                            const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
+                            void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Largest workspace (bytes) that paged_attn_decode_noalloc can serve from its fixed device
@@ -153,7 +160,8 @@ pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
                                     const int32_t* block_tables, const int32_t* context_lens,
                                     float scale, void* out, const pa_decode_desc* desc,
                                     int max_context_len, const float* k_scales,
-                                    const float* v_scales, float* lse_out, void* stream);
+                                    const float* v_scales, const int32_t* k_zeros,
+                                    const int32_t* v_zeros, float* lse_out, void* stream);
 
 /*
  * Slot-mapped write of new tokens' K and V into the pool ([KVPaged] "PagedAttention: OS
@@ -163,31 +171,37 @@ pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
  *     k_cache[block][h][offset][:] = convert(k[t][h][:])   for every kv head h (same for v)
  * convert: f32->f32 and bf16->bf16 copy bits; f32->bf16 rounds to nearest even; f32 or
  * bf16 -> fp8 stores E4M3(x / scale[block][h]) with an IEEE float32 division, round to
- * nearest even, saturating to +-448. A negative slot is a padding token and is skipped.
+ * nearest even, saturating to +-448; f32 or bf16 -> int8 stores
+ * clamp(round_half_even(x / scale[block][h]) + zero[block][h], -128, 127), same division.
+ * A negative slot is a padding token and is skipped.
  *   k, v             device [num_tokens][Hkv][head_dim] rows, token stride k_stride /
  *                    v_stride elements (>= Hkv*head_dim), in in_dtype
  *   slot_mapping     int64 [num_tokens]
- *   k_scales/v_scales float32 [num_blocks][Hkv], fp8 caches only (read, not written)
+ *   k_scales/v_scales float32 [num_blocks][Hkv], fp8 and int8 caches (read, not written)
+ *   k_zeros/v_zeros  int32 [num_blocks][Hkv], int8 caches only (read, not written)
  * Tokens must map to distinct slots (two writes to one slot race).
  */
 pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,
                             const int64_t* slot_mapping, int num_tokens, int64_t k_stride,
                             int64_t v_stride, int num_kv_heads, int head_dim, int block_size,
                             int num_blocks, pa_dtype in_dtype, pa_dtype cache_dtype,
-                            const float* k_scales, const float* v_scales, void* stream);
+                            const float* k_scales, const float* v_scales,
+                            const int32_t* k_zeros, const int32_t* v_zeros, void* stream);
 
 /*
  * Copy-on-write block copy ([KVPaged] "Prefix sharing and copy-on-write": a shared block is
  * copied before one sharer modifies it; [Ch4PA] "Prefix Caching": copies happen only on
  * write). For each pair i, (src, dst) = (pairs[2i], pairs[2i+1]) (device int32 [n][2]):
  * the K and V tiles of every kv head of block src are copied to block dst, and for fp8
- * caches the scales too (k_scales/v_scales may be NULL otherwise). No dst may appear twice
+ * and int8 caches the scales too (k_scales/v_scales may be NULL otherwise), for int8 also
+ * the zero points (k_zeros/v_zeros may be NULL otherwise). No dst may appear twice
  * or also be a src: such copies race. Enqueue it before the reshape_and_cache that writes
  * into the destination blocks.
  */
 pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_scales,
-                      const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
-                      int block_size, int num_blocks, pa_dtype cache_dtype, void* stream);
+                      int32_t* k_zeros, int32_t* v_zeros, const int32_t* pairs, int num_pairs,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      pa_dtype cache_dtype, void* stream);
 
 /*
  * Reads and clears the device error word of the current device (a bitwise OR of

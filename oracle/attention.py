@@ -8,7 +8,8 @@ attention. [KVPaged] "GQA and MQA": query heads are grouped and every group shar
 head (read: contiguous groups, query head h uses kv head h // (Hq / Hkv)).
 
 The oracle is the plain definition: gather through the block table into contiguous arrays,
-decode every stored element exactly to float64 (fp8: E4M3 value * the block's scale), then
+decode every stored element exactly to float64 (fp8: E4M3 value * the block's scale; int8:
+(code - zero point) * scale), then
 z = scale * q . K_t, p = exp(z - max z) / sum exp(z - max z), out = sum_t p_t V_t and
 lse = max z + log sum exp(z - max z). ``context_lens[s]`` counts the token being decoded.
 """
@@ -34,16 +35,24 @@ def decode_values(codes: np.ndarray, dtype: str) -> np.ndarray:
 
 
 def gather_kv(k_cache, v_cache, block_row, ctx: int, kvh: int, kv_dtype: str,
-              k_scales=None, v_scales=None) -> Tuple[np.ndarray, np.ndarray]:
+              k_scales=None, v_scales=None, k_zeros=None,
+              v_zeros=None) -> Tuple[np.ndarray, np.ndarray]:
     """Contiguous float64 K and V [ctx, d] of one (sequence, kv head), read through the
-    block table row: token t lives in physical block block_row[t // B] at offset t % B."""
+    block table row: token t lives in physical block block_row[t // B] at offset t % B.
+    fp8: E4M3 value * scale; int8: (code - zero) * scale, of the token's block."""
     B = k_cache.shape[2]
     t = np.arange(ctx)
     blk = np.asarray(block_row, dtype=np.int64)[t // B]
     off = t % B
-    K = decode_values(k_cache[blk, kvh, off, :], kv_dtype)
-    V = decode_values(v_cache[blk, kvh, off, :], kv_dtype)
-    if kv_dtype == "fp8":
+    if kv_dtype == "int8":
+        K = k_cache[blk, kvh, off, :].astype(np.float64) - \
+            np.asarray(k_zeros, dtype=np.float64)[blk, kvh][:, None]
+        V = v_cache[blk, kvh, off, :].astype(np.float64) - \
+            np.asarray(v_zeros, dtype=np.float64)[blk, kvh][:, None]
+    else:
+        K = decode_values(k_cache[blk, kvh, off, :], kv_dtype)
+        V = decode_values(v_cache[blk, kvh, off, :], kv_dtype)
+    if kv_dtype in ("fp8", "int8"):
         K = K * np.asarray(k_scales, dtype=np.float64)[blk, kvh][:, None]
         V = V * np.asarray(v_scales, dtype=np.float64)[blk, kvh][:, None]
     return K, V
@@ -53,7 +62,8 @@ def ref_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
                block_tables: np.ndarray, context_lens: np.ndarray, scale: float,
                num_kv_heads: int, q_dtype: str, kv_dtype: str,
                k_scales: Optional[np.ndarray] = None, v_scales: Optional[np.ndarray] = None,
-               seqs: Optional[Iterable[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+               seqs: Optional[Iterable[int]] = None, k_zeros: Optional[np.ndarray] = None,
+               v_zeros: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
     """out [S, Hq, d] and lse [S, Hq] in float64 for the sequences in ``seqs`` (default all;
     rows of other sequences are NaN). ctx = 0 gives out = 0 and lse = -inf."""
     S, Hq, d = q.shape
@@ -70,7 +80,7 @@ def ref_decode(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray,
                 lse[s, hs] = -np.inf
                 continue
             K, V = gather_kv(k_cache, v_cache, block_tables[s], ctx, kvh, kv_dtype,
-                             k_scales, v_scales)
+                             k_scales, v_scales, k_zeros, v_zeros)
             z = scale * (qv[s, hs] @ K.T)          # [G, ctx]
             m = z.max(axis=1, keepdims=True)
             e = np.exp(z - m)

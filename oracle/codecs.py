@@ -81,3 +81,20 @@ def e4m3_encode(y: np.ndarray) -> np.ndarray:
     if nan.any():
         code[nan] = np.uint8(0x7F)
     return code
+
+
+# ---------------------------------------------------------------------------------------
+# INT8 with scale and zero point ([KVPaged] "KV quantization: FP8 and INT8": one byte per
+# element, needs a scale and a zero point). Affine code: value = (code - zero) * scale.
+# ---------------------------------------------------------------------------------------
+def int8_encode(y: np.ndarray, zero) -> np.ndarray:
+    """float32 y = x / scale (already divided) -> int8 code = clip(round(y) + zero, -128, 127),
+    round half to even."""
+    y = np.asarray(y, dtype=np.float32)
+    r = np.rint(y.astype(np.float64)) + np.asarray(zero, dtype=np.float64)
+    return np.clip(r, -128, 127).astype(np.int8)
+
+
+def int8_decode(codes: np.ndarray, zero) -> np.ndarray:
+    """int8 codes -> (code - zero) as float64 (exact); multiply by the scale to dequantise."""
+    return np.asarray(codes, dtype=np.int8).astype(np.float64) - np.asarray(zero, dtype=np.float64)

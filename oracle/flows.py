@@ -37,6 +37,8 @@ class RefState:
     context_lens: np.ndarray
     cow_pairs: List
     step_slots: Dict[int, np.ndarray]
+    k_zeros: Optional[np.ndarray] = None
+    v_zeros: Optional[np.ndarray] = None
 
 
 def max_blocks_per_seq(draw) -> int:
@@ -55,6 +57,18 @@ def _fp8_scales(draw, alloc, seqs, nb, hkv):
     return ks, vs
 
 
+def _int8_params(draw, alloc, seqs, nb, hkv):
+    ks = np.ones((nb, hkv), dtype=np.float32)
+    vs = np.ones((nb, hkv), dtype=np.float32)
+    kz = np.zeros((nb, hkv), dtype=np.int32)
+    vz = np.zeros((nb, hkv), dtype=np.int32)
+    for s in seqs:
+        lks, lkz, lvs, lvz = draw.int8_params_logical(s)
+        row = alloc.block_table(s)
+        ks[row], kz[row], vs[row], vz[row] = lks, lkz, lvs, lvz
+    return ks, vs, kz, vz
+
+
 def build_state(draw, write_seqs: Optional[Sequence[int]] = None, shared: bool = True) -> RefState:
     """Allocate, copy and write the whole workload. K/V is written only for ``write_seqs``
     (default: all), which bounds the work for large workloads checked on a sample; the
@@ -69,7 +83,7 @@ def build_state(draw, write_seqs: Optional[Sequence[int]] = None, shared: bool =
     alloc = RefAllocator(nb, B, order=draw.pool_order if nb == wl.num_blocks else None)
     kc = new_cache(nb, H, B, d, wl.kv_dtype)
     vc = new_cache(nb, H, B, d, wl.kv_dtype)
-    ks = vs = None
+    ks = vs = kz = vz = None
     pairs: List = []
     step_slots: Dict[int, np.ndarray] = {}
     if wl.shared_prefix is not None and shared:
@@ -84,13 +98,16 @@ def build_state(draw, write_seqs: Optional[Sequence[int]] = None, shared: bool =
             pairs += pr
         if wl.kv_dtype == "fp8":
             ks, vs = _fp8_scales(draw, alloc, range(S), nb, H)
+        elif wl.kv_dtype == "int8":
+            ks, vs, kz, vz = _int8_params(draw, alloc, range(S), nb, H)
         k0, v0 = draw.kv(0)
-        ref_reshape_and_cache(k0[:p], v0[:p], kc, vc, slots0, wl.in_dtype, wl.kv_dtype, ks, vs)
-        ref_copy_blocks(kc, vc, pairs, ks, vs)
+        ref_reshape_and_cache(k0[:p], v0[:p], kc, vc, slots0, wl.in_dtype, wl.kv_dtype, ks, vs,
+                              kz, vz)
+        ref_copy_blocks(kc, vc, pairs, ks, vs, kz, vz)
         for s in sorted(write):
             k, v = draw.kv(s)
             ref_reshape_and_cache(k[p:], v[p:], kc, vc, sfx_slots[s], wl.in_dtype, wl.kv_dtype,
-                                  ks, vs)
+                                  ks, vs, kz, vz)
             step_slots[s] = sfx_slots[s]
     else:
         pre = {}
@@ -102,13 +119,17 @@ def build_state(draw, write_seqs: Optional[Sequence[int]] = None, shared: bool =
             step_slots[s] = sl
         if wl.kv_dtype == "fp8":
             ks, vs = _fp8_scales(draw, alloc, write, nb, H)
+        elif wl.kv_dtype == "int8":
+            ks, vs, kz, vz = _int8_params(draw, alloc, write, nb, H)
         for s in sorted(write):
             k, v = draw.kv(s)
-            ref_reshape_and_cache(k[:-1], v[:-1], kc, vc, pre[s], wl.in_dtype, wl.kv_dtype, ks, vs)
+            ref_reshape_and_cache(k[:-1], v[:-1], kc, vc, pre[s], wl.in_dtype, wl.kv_dtype, ks, vs,
+                                  kz, vz)
             ref_reshape_and_cache(k[-1:], v[-1:], kc, vc, step_slots[s], wl.in_dtype,
-                                  wl.kv_dtype, ks, vs)
+                                  wl.kv_dtype, ks, vs, kz, vz)
     tables = alloc.padded_tables(range(S), max_blocks_per_seq(draw))
-    return RefState(alloc, kc, vc, ks, vs, tables, draw.context_lens.copy(), pairs, step_slots)
+    return RefState(alloc, kc, vc, ks, vs, tables, draw.context_lens.copy(), pairs, step_slots,
+                    kz, vz)
 
 
 def ref_outputs(draw, state: RefState, seqs: Optional[Sequence[int]] = None, scale=None):
@@ -117,4 +138,5 @@ def ref_outputs(draw, state: RefState, seqs: Optional[Sequence[int]] = None, sca
     sc = float(np.float32(1.0 / np.sqrt(wl.head_dim) if scale is None else scale))
     return ref_decode(draw.q, state.k_cache, state.v_cache, state.block_tables,
                       state.context_lens, sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype,
-                      state.k_scales, state.v_scales, seqs=seqs)
+                      state.k_scales, state.v_scales, seqs=seqs, k_zeros=state.k_zeros,
+                      v_zeros=state.v_zeros)

@@ -24,7 +24,7 @@ from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
 
-from .codecs import bf16_encode, bf16_decode, e4m3_encode
+from .codecs import bf16_encode, bf16_decode, e4m3_encode, int8_encode
 
 
 class NoBlocks(Exception):
@@ -158,7 +158,7 @@ class RefAllocator:
 # ---------------------------------------------------------------------------------------
 # cache storage
 # ---------------------------------------------------------------------------------------
-_STORE = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}
+_STORE = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8, "int8": np.int8}
 
 
 def new_cache(num_blocks: int, num_kv_heads: int, block_size: int, head_dim: int,
@@ -175,11 +175,13 @@ def _to_f32(x: np.ndarray, in_dtype: str) -> np.ndarray:
     raise ValueError(in_dtype)
 
 
-def _convert(xf: np.ndarray, cache_dtype: str, scale: Optional[np.ndarray]) -> np.ndarray:
+def _convert(xf: np.ndarray, cache_dtype: str, scale: Optional[np.ndarray],
+             zero: Optional[np.ndarray] = None) -> np.ndarray:
     """float32 values -> storage codes of ``cache_dtype``.
 
     fp8: code = E4M3(x / scale) with the division done in IEEE float32 (round to nearest),
-    ``scale`` broadcast over the head dimension."""
+    ``scale`` broadcast over the head dimension. int8: code = clip(rint(x / scale) + zero,
+    -128, 127), same division."""
     if cache_dtype == "f32":
         return xf.astype(np.float32)
     if cache_dtype == "bf16":
@@ -187,19 +189,24 @@ def _convert(xf: np.ndarray, cache_dtype: str, scale: Optional[np.ndarray]) -> n
     if cache_dtype == "fp8":
         y = (xf / scale[..., None].astype(np.float32)).astype(np.float32)
         return e4m3_encode(y)
+    if cache_dtype == "int8":
+        y = (xf / scale[..., None].astype(np.float32)).astype(np.float32)
+        return int8_encode(y, np.asarray(zero)[..., None])
     raise ValueError(cache_dtype)
 
 
 def ref_reshape_and_cache(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,
                           v_cache: np.ndarray, slot_mapping: np.ndarray, in_dtype: str,
                           cache_dtype: str, k_scales: Optional[np.ndarray] = None,
-                          v_scales: Optional[np.ndarray] = None) -> None:
+                          v_scales: Optional[np.ndarray] = None,
+                          k_zeros: Optional[np.ndarray] = None,
+                          v_zeros: Optional[np.ndarray] = None) -> None:
     """Slot-mapped write of new tokens' K and V into the paged cache (in place).
 
     For token t with slot = slot_mapping[t] >= 0: block = slot // B, offset = slot % B and
     ``cache[block][h][offset][:] = convert(x[t][h][:])`` for every kv head h. A negative
     slot marks a padding token and is skipped. fp8 caches use the per-(block, kv head)
-    scale of the destination block.
+    scale of the destination block; int8 caches its scale and zero point.
     """
     B = k_cache.shape[2]
     slots = np.asarray(slot_mapping, dtype=np.int64)
@@ -207,22 +214,25 @@ def ref_reshape_and_cache(k: np.ndarray, v: np.ndarray, k_cache: np.ndarray,
         if slot < 0:
             continue
         blk, off = int(slot // B), int(slot % B)
-        for x, cache, sc in ((k, k_cache, k_scales), (v, v_cache, v_scales)):
+        for x, cache, sc, zp in ((k, k_cache, k_scales, k_zeros), (v, v_cache, v_scales, v_zeros)):
             xf = _to_f32(x[t], in_dtype)  # [Hkv, d]
             s = None if sc is None else sc[blk]  # [Hkv]
-            cache[blk, :, off, :] = _convert(xf, cache_dtype, s)
+            z = None if zp is None else zp[blk]
+            cache[blk, :, off, :] = _convert(xf, cache_dtype, s, z)
 
 
 def ref_copy_blocks(k_cache: np.ndarray, v_cache: np.ndarray,
                     pairs: Sequence[Tuple[int, int]],
                     k_scales: Optional[np.ndarray] = None,
-                    v_scales: Optional[np.ndarray] = None) -> None:
+                    v_scales: Optional[np.ndarray] = None,
+                    k_zeros: Optional[np.ndarray] = None,
+                    v_zeros: Optional[np.ndarray] = None) -> None:
     """Copy-on-write block copy: for each (src, dst) pair, in order, the K and V tiles of
-    every kv head (and the fp8 scales, when given) of ``src`` are copied to ``dst``."""
+    every kv head (and the quantisation scales / zero points, when given) of ``src`` are
+    copied to ``dst``."""
     for src, dst in pairs:
         k_cache[dst] = k_cache[src]
         v_cache[dst] = v_cache[src]
-        if k_scales is not None:
-            k_scales[dst] = k_scales[src]
-        if v_scales is not None:
-            v_scales[dst] = v_scales[src]
+        for arr in (k_scales, v_scales, k_zeros, v_zeros):
+            if arr is not None:
+                arr[dst] = arr[src]

@@ -28,7 +28,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 # ---------------------------------------------------------------------------------------
 # enums (mirror include/pagedattn.h)
 # ---------------------------------------------------------------------------------------
-PA_F32, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+PA_F32, PA_BF16, PA_FP8_E4M3, PA_INT8 = 0, 1, 2, 3
 PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR_WORKSPACE, \
     PA_ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6
 PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_CONTEXT, PA_DEVERR_TIMEOUT = \
@@ -62,12 +62,12 @@ _SIGS = {
     "pa_version": (ctypes.c_char_p, []),
     "paged_attn_workspace_size": (_sz, [_P(pa_decode_desc), _i]),
     "paged_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i, _vp,
-                               _vp, _vp, _vp, _sz, _vp]),
+                               _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "paged_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i,
-                                       _vp, _vp, _vp, _vp]),
+                                       _vp, _vp, _vp, _vp, _vp, _vp]),
     "reshape_and_cache": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _i, _i, _i, _i,
-                               _vp, _vp, _vp]),
-    "copy_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
+                               _vp, _vp, _vp, _vp, _vp]),
+    "copy_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
     "pa_device_error": (_i, [_P(_i), _vp]),
     "pa_alloc_create": (_vp, [_i, _i]),
     "pa_alloc_create_ordered": (_vp, [_i, _i, _vp]),
@@ -116,6 +116,8 @@ def _dtype_code(t) -> int:
         return PA_BF16
     if t in (torch.float8_e4m3fn, torch.uint8):
         return PA_FP8_E4M3
+    if t == torch.int8:
+        return PA_INT8
     raise TypeError(f"unsupported dtype {t}")
 
 
@@ -172,13 +174,15 @@ def decode_desc_for(q, k_cache, block_tables, partition_size: int) -> pa_decode_
 
 def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: float, out, *,
                       max_context_len: int, partition_size: int = 0, k_scales=None,
-                      v_scales=None, lse_out=None, workspace=None, stream=None):
+                      v_scales=None, k_zeros=None, v_zeros=None, lse_out=None, workspace=None,
+                      stream=None):
     """out[s, h] = softmax(scale * q[s, h] K^T) V over the paged cache of sequence s.
 
-    q, out [S, Hq, d] (fp32 or bf16); k_cache/v_cache [NB, Hkv, 16, d] (fp32, bf16 or
-    fp8-e4m3 as float8_e4m3fn/uint8); block_tables int32 [S, MB]; context_lens int32 [S];
-    k_scales/v_scales fp32 [NB, Hkv] for fp8; lse_out fp32 [S, Hq] or None; workspace a
-    uint8 CUDA tensor of at least ``workspace_size(...)`` bytes when partition_size > 0.
+    q, out [S, Hq, d] (fp32 or bf16); k_cache/v_cache [NB, Hkv, 16, d] (fp32, bf16,
+    fp8-e4m3 as float8_e4m3fn/uint8, or int8); block_tables int32 [S, MB]; context_lens
+    int32 [S]; k_scales/v_scales fp32 [NB, Hkv] for fp8 and int8; k_zeros/v_zeros int32
+    [NB, Hkv] for int8; lse_out fp32 [S, Hq] or None; workspace a uint8 CUDA tensor of at
+    least ``workspace_size(...)`` bytes when partition_size > 0.
     """
     torch = _torch()
     desc = decode_desc_for(q, k_cache, block_tables, partition_size)
@@ -190,9 +194,9 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: fl
         raise ValueError("block_tables / context_lens do not match q")
     if lse_out is not None and tuple(lse_out.shape) != tuple(q.shape[:2]):
         raise ValueError("lse_out must be [S, Hq]")
-    for sc in (k_scales, v_scales):
+    for sc in (k_scales, v_scales, k_zeros, v_zeros):
         if sc is not None and tuple(sc.shape) != tuple(k_cache.shape[:2]):
-            raise ValueError("scales must be [num_blocks, num_kv_heads]")
+            raise ValueError("scales / zero points must be [num_blocks, num_kv_heads]")
     ws_need = workspace_size(desc, max_context_len)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = _lib.paged_attn_decode(
@@ -200,6 +204,7 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: fl
         _dev(block_tables, "block_tables", torch.int32), _dev(context_lens, "context_lens", torch.int32),
         ctypes.c_float(scale), _dev(out, "out"), ctypes.byref(desc), int(max_context_len),
         _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(k_zeros, "k_zeros", torch.int32), _dev(v_zeros, "v_zeros", torch.int32),
         _dev(lse_out, "lse_out", torch.float32), _dev(workspace, "workspace"), ws_bytes,
         _stream(stream))
     if st == PA_ERR_WORKSPACE:
@@ -213,7 +218,8 @@ NOALLOC_SCRATCH_BYTES = 32 << 20
 
 def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale: float,
                               out, *, max_context_len: int, partition_size: int = 0,
-                              k_scales=None, v_scales=None, lse_out=None, stream=None):
+                              k_scales=None, v_scales=None, k_zeros=None, v_zeros=None,
+                              lse_out=None, stream=None):
     """paged_attn_decode without a caller workspace: the split-KV scratch comes from a fixed
     array inside the library (at most NOALLOC_SCRATCH_BYTES per GPU), for callers that
     cannot allocate device memory. Overlapping calls on one GPU race on that array."""
@@ -226,15 +232,17 @@ def paged_attn_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, s
         _dev(block_tables, "block_tables", torch.int32), _dev(context_lens, "context_lens", torch.int32),
         ctypes.c_float(scale), _dev(out, "out"), ctypes.byref(desc), int(max_context_len),
         _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(k_zeros, "k_zeros", torch.int32), _dev(v_zeros, "v_zeros", torch.int32),
         _dev(lse_out, "lse_out", torch.float32), _stream(stream))
     _check(st, "paged_attn_decode_noalloc")
     return out
 
 
 def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, *, k_scales=None, v_scales=None,
-                      stream=None):
+                      k_zeros=None, v_zeros=None, stream=None):
     """Writes k, v [T, Hkv, d] (rows may be strided along T) into the cache slots given by
-    slot_mapping int64 [T] (negative = skip)."""
+    slot_mapping int64 [T] (negative = skip); fp8 / int8 caches take the per-(block, kv
+    head) scales (and int8 zero points) of the destination blocks."""
     torch = _torch()
     T, Hkv, d = k.shape
     NB, Hkv2, B, d2 = k_cache.shape
@@ -253,19 +261,23 @@ def reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, *, k_scales=None, v_
         _dev(v_cache, "v_cache"), _dev(slot_mapping, "slot_mapping", torch.int64), T,
         int(k.stride(0)), int(v.stride(0)), Hkv, d, B, NB, _dtype_code(k.dtype),
         _dtype_code(k_cache.dtype), _dev(k_scales, "k_scales", torch.float32),
-        _dev(v_scales, "v_scales", torch.float32), _stream(stream))
+        _dev(v_scales, "v_scales", torch.float32), _dev(k_zeros, "k_zeros", torch.int32),
+        _dev(v_zeros, "v_zeros", torch.int32), _stream(stream))
     _check(st, "reshape_and_cache")
 
 
-def copy_blocks(k_cache, v_cache, pairs, *, k_scales=None, v_scales=None, stream=None):
-    """Copies whole blocks (K, V and fp8 scales) for every (src, dst) row of pairs int32 [n, 2]."""
+def copy_blocks(k_cache, v_cache, pairs, *, k_scales=None, v_scales=None, k_zeros=None,
+                v_zeros=None, stream=None):
+    """Copies whole blocks (K, V and the quantisation scales / zero points) for every
+    (src, dst) row of pairs int32 [n, 2]."""
     torch = _torch()
     NB, Hkv, B, d = k_cache.shape
     if pairs.dim() != 2 or pairs.shape[1] != 2:
         raise ValueError("pairs must be [n, 2]")
     st = _lib.copy_blocks(
         _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"), _dev(k_scales, "k_scales", torch.float32),
-        _dev(v_scales, "v_scales", torch.float32), _dev(pairs, "pairs", torch.int32),
+        _dev(v_scales, "v_scales", torch.float32), _dev(k_zeros, "k_zeros", torch.int32),
+        _dev(v_zeros, "v_zeros", torch.int32), _dev(pairs, "pairs", torch.int32),
         int(pairs.shape[0]), Hkv, d, B, NB, _dtype_code(k_cache.dtype), _stream(stream))
     _check(st, "copy_blocks")
 

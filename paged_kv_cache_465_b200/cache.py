@@ -13,7 +13,7 @@ import numpy as np
 from . import (BlockAllocator, copy_blocks, paged_attn_decode, reshape_and_cache,
                workspace_size, decode_desc_for)
 
-_TORCH_DTYPE = {"f32": "float32", "bf16": "bfloat16", "fp8": "uint8"}
+_TORCH_DTYPE = {"f32": "float32", "bf16": "bfloat16", "fp8": "uint8", "int8": "int8"}
 
 
 class PagedKVCache:
@@ -27,11 +27,16 @@ class PagedKVCache:
         shape = (num_blocks, num_kv_heads, block_size, head_dim)
         self.k_cache = torch.zeros(shape, dtype=dt, device=device)
         self.v_cache = torch.zeros(shape, dtype=dt, device=device)
-        if kv_dtype == "fp8":
+        if kv_dtype in ("fp8", "int8"):
             self.k_scales = torch.ones((num_blocks, num_kv_heads), dtype=torch.float32, device=device)
             self.v_scales = torch.ones((num_blocks, num_kv_heads), dtype=torch.float32, device=device)
         else:
             self.k_scales = self.v_scales = None
+        if kv_dtype == "int8":
+            self.k_zeros = torch.zeros((num_blocks, num_kv_heads), dtype=torch.int32, device=device)
+            self.v_zeros = torch.zeros((num_blocks, num_kv_heads), dtype=torch.int32, device=device)
+        else:
+            self.k_zeros = self.v_zeros = None
         self.alloc = BlockAllocator(num_blocks, block_size, order)
 
     # ---- host bookkeeping ----------------------------------------------------------------
@@ -53,12 +58,14 @@ class PagedKVCache:
     # ---- device operations -------------------------------------------------------------
     def write(self, k, v, slots, stream=None) -> None:
         reshape_and_cache(k, v, self.k_cache, self.v_cache, slots, k_scales=self.k_scales,
-                          v_scales=self.v_scales, stream=stream)
+                          v_scales=self.v_scales, k_zeros=self.k_zeros, v_zeros=self.v_zeros,
+                          stream=stream)
 
     def copy(self, pairs, stream=None) -> None:
         if pairs is not None and pairs.shape[0] > 0:
             copy_blocks(self.k_cache, self.v_cache, pairs, k_scales=self.k_scales,
-                        v_scales=self.v_scales, stream=stream)
+                        v_scales=self.v_scales, k_zeros=self.k_zeros, v_zeros=self.v_zeros,
+                        stream=stream)
 
     def workspace_bytes(self, q, block_tables, max_context_len: int, partition_size: int) -> int:
         return workspace_size(decode_desc_for(q, self.k_cache, block_tables, partition_size),
@@ -69,5 +76,6 @@ class PagedKVCache:
         return paged_attn_decode(q, self.k_cache, self.v_cache, block_tables, context_lens,
                                  scale, out, max_context_len=max_context_len,
                                  partition_size=partition_size, k_scales=self.k_scales,
-                                 v_scales=self.v_scales, lse_out=lse_out, workspace=workspace,
+                                 v_scales=self.v_scales, k_zeros=self.k_zeros,
+                                 v_zeros=self.v_zeros, lse_out=lse_out, workspace=workspace,
                                  stream=stream)

@@ -2,7 +2,9 @@
 //
 // [KVPaged] "PagedAttention: OS virtual-memory style management": new tokens land in the
 // block the block table maps their logical position to. [KVPaged] "Prefix sharing and
-// copy-on-write": a shared block is copied before a sharer writes into it.
+// copy-on-write": a shared block is copied before a sharer writes into it. [KVPaged] "KV
+// quantization: FP8 and INT8": fp8 stores E4M3(x / scale), int8 an affine code with a scale
+// and a zero point, per (block, kv head).
 //
 // Both are pure HBM streams: one CTA per token (write) or per (pair, K|V) (copy), 16-byte
 // vector accesses, no shared memory.
@@ -36,7 +38,9 @@ __global__ void reshape_and_cache_kernel(const void* __restrict__ k, const void*
                                          int64_t k_stride, int64_t v_stride, int num_kv_heads,
                                          int head_dim, int block_size, int num_blocks,
                                          const float* __restrict__ k_scales,
-                                         const float* __restrict__ v_scales) {
+                                         const float* __restrict__ v_scales,
+                                         const int32_t* __restrict__ k_zeros,
+                                         const int32_t* __restrict__ v_zeros) {
   pdl_wait();
   pdl_trigger();
   const int t = blockIdx.x;
@@ -68,6 +72,20 @@ __global__ void reshape_and_cache_kernel(const void* __restrict__ k, const void*
       w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
       w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
       *reinterpret_cast<uint4*>(static_cast<uint16_t*>(cache) + dst) = w;
+    } else if constexpr (CACHE == PA_INT8) {
+      const int64_t sh = blk * num_kv_heads + h;
+      const float s = (is_v ? v_scales : k_scales)[sh];
+      const int z = (is_v ? v_zeros : k_zeros)[sh];
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // round half to even; |y| is clamped first so the sum cannot overflow (the result
+        // is clamped to the int8 range anyway)
+        const float y = fminf(fmaxf(__fdiv_rn(x[j], s), -1024.f), 1024.f);
+        const int c = min(127, max(-128, __float2int_rn(y) + z));
+        w[j >> 2] |= ((uint32_t)c & 0xffu) << (8 * (j & 3));
+      }
+      *reinterpret_cast<uint2*>(static_cast<uint8_t*>(cache) + dst) = make_uint2(w[0], w[1]);
     } else {
       const float s = (is_v ? v_scales : k_scales)[blk * num_kv_heads + h];
       uint16_t b[4];
@@ -85,6 +103,7 @@ __global__ void reshape_and_cache_kernel(const void* __restrict__ k, const void*
 // One CTA per (pair, K|V): copies the whole block (all kv heads) with 16-byte accesses.
 __global__ void copy_blocks_kernel(uint8_t* __restrict__ k_cache, uint8_t* __restrict__ v_cache,
                                    float* __restrict__ k_scales, float* __restrict__ v_scales,
+                                   int32_t* __restrict__ k_zeros, int32_t* __restrict__ v_zeros,
                                    const int32_t* __restrict__ pairs, int64_t block_bytes,
                                    int num_kv_heads, int num_blocks) {
   pdl_wait();
@@ -105,6 +124,10 @@ __global__ void copy_blocks_kernel(uint8_t* __restrict__ k_cache, uint8_t* __res
   if (sc != nullptr)
     for (int h = threadIdx.x; h < num_kv_heads; h += blockDim.x)
       sc[(int64_t)dst * num_kv_heads + h] = sc[(int64_t)src * num_kv_heads + h];
+  int32_t* zp = is_v ? v_zeros : k_zeros;
+  if (zp != nullptr)
+    for (int h = threadIdx.x; h < num_kv_heads; h += blockDim.x)
+      zp[(int64_t)dst * num_kv_heads + h] = zp[(int64_t)src * num_kv_heads + h];
 }
 
 }  // namespace pa

@@ -35,11 +35,18 @@ template <>
 struct KvTraits<PA_BF16> { static constexpr int bytes = 2; };
 template <>
 struct KvTraits<PA_FP8_E4M3> { static constexpr int bytes = 1; };
+template <>
+struct KvTraits<PA_INT8> { static constexpr int bytes = 1; };
 
-// 16 bytes of KV -> 16/bytes floats (raw stored value, scale not applied).
+// 16 bytes of KV -> 16/bytes floats (raw stored value: no scale applied; int8 gives the
+// signed code, the zero point is subtracted by the caller).
 template <pa_dtype KV>
 __device__ __forceinline__ void unpack16(uint4 w, float* x) {
-  if constexpr (KV == PA_F32) {
+  if constexpr (KV == PA_INT8) {
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int j = 0; j < 16; ++j) x[j] = (float)(int8_t)((ws[j >> 2] >> (8 * (j & 3))) & 0xff);
+  } else if constexpr (KV == PA_F32) {
     x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
     x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
   } else if constexpr (KV == PA_BF16) {
@@ -74,6 +81,12 @@ __device__ __forceinline__ void load_vslice(const uint8_t* row, int lane, float*
       uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(p) + j / 2);
       x[j] = bf16_lo(w); x[j + 1] = bf16_hi(w);
     }
+  } else if constexpr (KV == PA_INT8) {
+#pragma unroll
+    for (int j = 0; j < N; j += 2) {
+      uint16_t w = __ldg(reinterpret_cast<const uint16_t*>(p) + j / 2);
+      x[j] = (float)(int8_t)(w & 0xff); x[j + 1] = (float)(int8_t)(w >> 8);
+    }
   } else {
 #pragma unroll
     for (int j = 0; j < N; j += 2) {
@@ -94,6 +107,8 @@ struct DecodeArgs {
   float* lse_out;
   const float* k_scales;
   const float* v_scales;
+  const int32_t* k_zeros;  // int8 caches
+  const int32_t* v_zeros;
   float* part_m;    // [S][Hq][P]   log2-domain running max of each partition
   float* part_l;    // [S][Hq][P]   sum of exp2(z - m)
   float* part_acc;  // [S][Hq][P][D] unnormalised sum of exp2(z - m) V
@@ -200,10 +215,14 @@ decode_simt_kernel(const DecodeArgs a) {
       continue;
     }
     const int64_t tile = ((int64_t)phys * a.num_kv_heads + kvh) * TILE;
-    float ks = 1.f, vs = 1.f;
-    if constexpr (KV == PA_FP8_E4M3) {
+    float ks = 1.f, vs = 1.f, kz = 0.f, vz = 0.f;
+    if constexpr (KV == PA_FP8_E4M3 || KV == PA_INT8) {
       ks = a.k_scales[(int64_t)phys * a.num_kv_heads + kvh];
       vs = a.v_scales[(int64_t)phys * a.num_kv_heads + kvh];
+    }
+    if constexpr (KV == PA_INT8) {
+      kz = (float)a.k_zeros[(int64_t)phys * a.num_kv_heads + kvh];
+      vz = (float)a.v_zeros[(int64_t)phys * a.num_kv_heads + kvh];
     }
     // ---- scores: lane (tok, half) -> partial dot over its half of d ----
     float sc[GP];
@@ -214,6 +233,10 @@ decode_simt_kernel(const DecodeArgs a) {
     for (int c = 0; c < CH; ++c) {
       float kx[EPC];
       unpack16<KV>(__ldg(krow + c), kx);
+      if constexpr (KV == PA_INT8) {
+#pragma unroll
+        for (int e = 0; e < EPC; ++e) kx[e] -= kz;  // exact: small integers
+      }
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         const float* qr = sq + g * QROW + half * (HALF + 4) + c * EPC;
@@ -259,6 +282,10 @@ decode_simt_kernel(const DecodeArgs a) {
     for (int tt = 0; tt < nv; ++tt) {
       float vx[NV];
       load_vslice<KV, D>(vbase + tile + (int64_t)tt * D * ES, lane, vx);
+      if constexpr (KV == PA_INT8) {
+#pragma unroll
+        for (int j = 0; j < NV; ++j) vx[j] -= vz;
+      }
 #pragma unroll
       for (int g = 0; g < GP; ++g) {
         const float pg = sp[warp][tt][g];

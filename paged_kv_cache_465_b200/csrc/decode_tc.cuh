@@ -142,6 +142,27 @@ __device__ __forceinline__ void mma16816(float (&c)[4], const uint32_t (&a)[4], 
   }
 }
 __device__ __forceinline__ uint32_t lo16(uint32_t x) { return x & 0xffffu; }
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+// int8 codes -> exact f16 (code - zero). The byte is made offset-binary (u = code + 128),
+// placed under an f16 exponent of 2^10 (0x64uu = 1024 + u) and (1152 + zero) subtracted:
+// all values are integers below 2048, so every step is exact. `sel` picks the two bytes
+// of `x_ob` (already XORed with 0x80808080); zc = f16x2(1152 + zero, 1152 + zero).
+__device__ __forceinline__ uint32_t i8x2_to_f16x2(uint32_t x_ob, uint32_t sel, uint32_t zc) {
+  return hsub2(__byte_perm(x_ob, 0x64646464u, sel), zc);
+}
+// (K, V) zero points of one block packed as two int16 -> the two subtraction constants.
+__device__ __forceinline__ void zero_consts(uint32_t packed, uint32_t& kzc, uint32_t& vzc) {
+  const float kz = (float)(int16_t)(packed & 0xffffu), vz = (float)(int16_t)(packed >> 16);
+  kzc = pack_f16x2(1152.f + kz, 1152.f + kz);
+  vzc = pack_f16x2(1152.f + vz, 1152.f + vz);
+}
+__device__ __forceinline__ uint32_t pack_zeros(int kz, int vz) {
+  return ((uint32_t)kz & 0xffffu) | ((uint32_t)vz << 16);
+}
 __device__ __forceinline__ uint32_t hi16(uint32_t x) { return x >> 16; }
 
 // Byte address of (row r, 16-byte chunk c) in a tile of 128-byte rows written by TMA with
@@ -160,7 +181,7 @@ __device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void* src, uint
 
 template <pa_dtype KV>
 struct TcCfg {
-  static constexpr bool kFp8 = KV == PA_FP8_E4M3;
+  static constexpr bool kFp8 = KV != PA_BF16;  // one-byte codes (fp8 or int8) -> f16 mma
   static constexpr int kTile = kFp8 ? 2048 : 4096;      // one (block, head) tile of K or V
   static constexpr int kStage = 2 * kTile;              // K + V
   static constexpr int kRows = kTile / 128;             // tensor-map rows per tile
@@ -259,10 +280,12 @@ __device__ __forceinline__ float load_q_frags(const uint16_t* qp, int G, int lan
 // block inside the work item; zs: log2-domain score scale (x fp8 K scale); vs: fp8 V scale.
 // The K products run as two independent accumulation chains and the V fragments are read
 // before the softmax, so a warp has independent work in flight at every step.
-template <bool FP8>
+template <pa_dtype KV>
 __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, float zs,
-                                         float vs, const uint32_t (&qf)[8][2], WarpAcc& w,
-                                         int lane) {
+                                         float vs, uint32_t kzc, uint32_t vzc,
+                                         const uint32_t (&qf)[8][2], WarpAcc& w, int lane) {
+  constexpr bool FP8 = KV != PA_BF16;  // one-byte codes, f16 products
+  constexpr bool I8 = KV == PA_INT8;
   constexpr int TILE = FP8 ? 2048 : 4096;
   const int gq = lane >> 2;
   float pv = 1.f, beta = 1.f;
@@ -303,11 +326,23 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
       for (int cp = 0; cp < 4; ++cp) ldsm_x4(swz(kt, tok, 2 * cp + (mi >> 1)), r[cp]);
 #pragma unroll
       for (int cp = 0; cp < 4; ++cp) {
-        uint32_t x0[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[cp][0])), e4m3x2_to_f16x2((uint16_t)lo16(r[cp][1])),
-                          e4m3x2_to_f16x2((uint16_t)hi16(r[cp][0])), e4m3x2_to_f16x2((uint16_t)hi16(r[cp][1]))};
+        // a register holds 4 consecutive channels of one token: pairs (0,1) and (2,3)
+        uint32_t x0[4], x1[4];
+        if constexpr (I8) {
+          uint32_t u[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) u[e] = r[cp][e] ^ 0x80808080u;
+          x0[0] = i8x2_to_f16x2(u[0], 0x4140, kzc); x0[1] = i8x2_to_f16x2(u[1], 0x4140, kzc);
+          x0[2] = i8x2_to_f16x2(u[0], 0x4342, kzc); x0[3] = i8x2_to_f16x2(u[1], 0x4342, kzc);
+          x1[0] = i8x2_to_f16x2(u[2], 0x4140, kzc); x1[1] = i8x2_to_f16x2(u[3], 0x4140, kzc);
+          x1[2] = i8x2_to_f16x2(u[2], 0x4342, kzc); x1[3] = i8x2_to_f16x2(u[3], 0x4342, kzc);
+        } else {
+          x0[0] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][0])); x0[1] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][1]));
+          x0[2] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][0])); x0[3] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][1]));
+          x1[0] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][2])); x1[1] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][3]));
+          x1[2] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][2])); x1[3] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][3]));
+        }
         mma16816<true>(sa, x0, qf[2 * cp][0], qf[2 * cp][1]);
-        uint32_t x1[4] = {e4m3x2_to_f16x2((uint16_t)lo16(r[cp][2])), e4m3x2_to_f16x2((uint16_t)lo16(r[cp][3])),
-                          e4m3x2_to_f16x2((uint16_t)hi16(r[cp][2])), e4m3x2_to_f16x2((uint16_t)hi16(r[cp][3]))};
         mma16816<true>(sb, x1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
       }
     }
@@ -368,14 +403,25 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
   } else {
 #pragma unroll
     for (int cp = 0; cp < 4; ++cp) {
-      uint32_t y[4];
+      // a register holds channels (2j, 2j+1) of tokens t0 (low half) and t1 (high half):
+      // pairs (t0, t1) at channel 2j are bytes (0, 2), at channel 2j+1 bytes (1, 3)
+      uint32_t ev[4], od[4];
+      if constexpr (I8) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) y[u] = __byte_perm(vr[cp][u], 0, 0x3120);
-      uint32_t ev[4] = {e4m3x2_to_f16x2((uint16_t)lo16(y[0])), e4m3x2_to_f16x2((uint16_t)lo16(y[1])),
-                        e4m3x2_to_f16x2((uint16_t)lo16(y[2])), e4m3x2_to_f16x2((uint16_t)lo16(y[3]))};
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t u = vr[cp][e] ^ 0x80808080u;
+          ev[e] = i8x2_to_f16x2(u, 0x4240, vzc);
+          od[e] = i8x2_to_f16x2(u, 0x4341, vzc);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t y = __byte_perm(vr[cp][e], 0, 0x3120);
+          ev[e] = e4m3x2_to_f16x2((uint16_t)lo16(y));
+          od[e] = e4m3x2_to_f16x2((uint16_t)hi16(y));
+        }
+      }
       mma16816<true>(w.acc[2 * cp], ev, pb0, pb1);
-      uint32_t od[4] = {e4m3x2_to_f16x2((uint16_t)hi16(y[0])), e4m3x2_to_f16x2((uint16_t)hi16(y[1])),
-                        e4m3x2_to_f16x2((uint16_t)hi16(y[2])), e4m3x2_to_f16x2((uint16_t)hi16(y[3]))};
       mma16816<true>(w.acc[2 * cp + 1], od, pb0, pb1);
     }
   }
@@ -477,11 +523,12 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   const int nblk = b_end - b_begin;
   const int nmine = nblk > warp ? (nblk - warp + kNW - 1) / kNW : 0;
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-  auto load_window = [&](int base, int& p, float& ks, float& vs) {
+  auto load_window = [&](int base, int& p, float& ks, float& vs, uint32_t& z) {
     const int k = base + lane;
     p = -2;
     ks = 1.f;
     vs = 1.f;
+    z = 0;
     if (k < nmine) {
       p = bt[b_begin + warp + k * kNW];
       if (p < 0 || p >= a.num_blocks) {
@@ -490,13 +537,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
       } else if constexpr (FP8) {
         ks = a.k_scales[(int64_t)p * a.num_kv_heads + kvh];
         vs = a.v_scales[(int64_t)p * a.num_kv_heads + kvh];
+        if constexpr (KV == PA_INT8)
+          z = pack_zeros(a.k_zeros[(int64_t)p * a.num_kv_heads + kvh],
+                         a.v_zeros[(int64_t)p * a.num_kv_heads + kvh]);
       }
     }
   };
   int cur_p, nxt_p;
   float cur_ks, cur_vs, nxt_ks, nxt_vs;
-  load_window(0, cur_p, cur_ks, cur_vs);
-  load_window(32, nxt_p, nxt_ks, nxt_vs);
+  uint32_t cur_z, nxt_z;
+  load_window(0, cur_p, cur_ks, cur_vs, cur_z);
+  load_window(32, nxt_p, nxt_ks, nxt_vs, nxt_z);
   const uint64_t policy = evict_first_policy();
   auto issue = [&](int k, int wbase, int stage) {
     const int rel = k - wbase;
@@ -526,13 +577,15 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   for (int i = 0; i < nmine; ++i) {
     const int wbase = i & ~31;
     if ((i & 31) == 0 && i > 0) {
-      cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs;
-      load_window(i + 32, nxt_p, nxt_ks, nxt_vs);
+      cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs; cur_z = nxt_z;
+      load_window(i + 32, nxt_p, nxt_ks, nxt_vs, nxt_z);
     }
     const int stage = i % NST;
     const int p = __shfl_sync(0xffffffffu, cur_p, i & 31);
     const float ks = __shfl_sync(0xffffffffu, cur_ks, i & 31);
     const float vs = __shfl_sync(0xffffffffu, cur_vs, i & 31);
+    uint32_t kzc = 0, vzc = 0;
+    if constexpr (KV == PA_INT8) zero_consts(__shfl_sync(0xffffffffu, cur_z, i & 31), kzc, vzc);
     if (!mbar_wait(bars + 8 * stage, (uint32_t)((i / NST) & 1))) {
       if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
       timed_out = true;
@@ -542,7 +595,8 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
     if (p >= 0) {
       const int b = b_begin + warp + i * kNW;
       const uint32_t kt = wtiles + stage * STAGE;
-      tc_block<FP8>(kt, kt + TILE, min(kBS, t1 - b * kBS), zscale * ks, vs, qf, w, lane);
+      tc_block<KV>(kt, kt + TILE, min(kBS, t1 - b * kBS), zscale * ks, vs, kzc, vzc, qf, w,
+                   lane);
     }
     __syncwarp();
     if (i + NST < nmine) issue(i + NST, wbase, stage);
@@ -705,11 +759,12 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
     }
     return v;
   };
-  // block-table window of an item for this warp: lane k holds block k's (phys, ks, vs)
-  auto load_window = [&](const WarpItem& v, int& p, float& ks, float& vs) {
+  // block-table window of an item for this warp: lane k holds block k's (phys, ks, vs, z)
+  auto load_window = [&](const WarpItem& v, int& p, float& ks, float& vs, uint32_t& z) {
     p = -2;
     ks = 1.f;
     vs = 1.f;
+    z = 0;
     if (v.valid && lane < v.nmine) {
       p = a.block_tables[(int64_t)v.s * a.max_blocks_per_seq + v.b_begin + warp + lane * kNW];
       if (p < 0 || p >= a.num_blocks) {
@@ -718,6 +773,8 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       } else if constexpr (FP8) {
         ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
         vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
+        if constexpr (KV == PA_INT8)
+          z = pack_zeros(a.k_zeros[(int64_t)p * Hkv + v.kvh], a.v_zeros[(int64_t)p * Hkv + v.kvh]);
       }
     }
   };
@@ -726,8 +783,9 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
   WarpItem cur = item_view(0), nxt = item_view(1);
   int cur_p, nxt_p;
   float cur_ks, cur_vs, nxt_ks, nxt_vs;
-  load_window(cur, cur_p, cur_ks, cur_vs);
-  load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+  uint32_t cur_z, nxt_z;
+  load_window(cur, cur_p, cur_ks, cur_vs, cur_z);
+  load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
 
   // producer position in this warp's block stream: (pslot 0 = cur / 1 = nxt, pk)
   int pslot = 0, pk = 0;
@@ -775,6 +833,8 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       const int p = __shfl_sync(0xffffffffu, cur_p, i);
       const float ks = __shfl_sync(0xffffffffu, cur_ks, i);
       const float vs = __shfl_sync(0xffffffffu, cur_vs, i);
+      uint32_t kzc = 0, vzc = 0;
+      if constexpr (KV == PA_INT8) zero_consts(__shfl_sync(0xffffffffu, cur_z, i), kzc, vzc);
       const int stage = g_cons % NST;
       if (!dead && !mbar_wait(bars + 8 * stage, (g_cons / NST) & 1)) {
         if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
@@ -783,7 +843,8 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       if (!dead && p >= 0) {
         const int b = cur.b_begin + warp + i * kNW;
         const uint32_t kt = wtiles + stage * STAGE;
-        tc_block<FP8>(kt, kt + TILE, min(kBS, cur.t1 - b * kBS), zscale * ks, vs, qf, w, lane);
+        tc_block<KV>(kt, kt + TILE, min(kBS, cur.t1 - b * kBS), zscale * ks, vs, kzc, vzc, qf,
+                     w, lane);
       }
       __syncwarp();
       ++g_cons;
@@ -813,9 +874,9 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
     // ---- advance: item k+1 becomes current, item k+2 (just fetched) the next ----
     ++k;
     cur = nxt;
-    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs;
+    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs; cur_z = nxt_z;
     nxt = item_view((k + 1) & 1);
-    load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+    load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
     pslot = 0;  // the producer finished item k, so it was positioned in item k+1
     produce();
   }
@@ -908,11 +969,12 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     }
     return v;
   };
-  // lane k holds block k's (phys, ks, vs) of an item
-  auto load_window = [&](const Item& v, int& p, float& ks, float& vs) {
+  // lane k holds block k's (phys, ks, vs, packed zero points) of an item
+  auto load_window = [&](const Item& v, int& p, float& ks, float& vs, uint32_t& z) {
     p = -2;
     ks = 1.f;
     vs = 1.f;
+    z = 0;
     if (v.valid && lane < v.nblk) {
       p = a.block_tables[(int64_t)v.s * a.max_blocks_per_seq + v.b_begin + lane];
       if (p < 0 || p >= a.num_blocks) {
@@ -921,6 +983,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       } else if constexpr (FP8) {
         ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
         vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
+        if constexpr (KV == PA_INT8)
+          z = pack_zeros(a.k_zeros[(int64_t)p * Hkv + v.kvh], a.v_zeros[(int64_t)p * Hkv + v.kvh]);
       }
     }
   };
@@ -942,8 +1006,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   Item nxt = fetch();
   int cur_p, nxt_p;
   float cur_ks, cur_vs, nxt_ks, nxt_vs;
-  load_window(cur, cur_p, cur_ks, cur_vs);
-  load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+  uint32_t cur_z, nxt_z;
+  load_window(cur, cur_p, cur_ks, cur_vs, cur_z);
+  load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
   copy_q(cur);
 
   int pslot = 0, pk = 0;
@@ -997,6 +1062,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       const int p = __shfl_sync(0xffffffffu, cur_p, i);
       const float ks = __shfl_sync(0xffffffffu, cur_ks, i);
       const float vs = __shfl_sync(0xffffffffu, cur_vs, i);
+      uint32_t kzc = 0, vzc = 0;
+      if constexpr (KV == PA_INT8) zero_consts(__shfl_sync(0xffffffffu, cur_z, i), kzc, vzc);
       const int stage = g_cons % NST;
       if (!dead && !mbar_wait(bars + 8 * stage, (g_cons / NST) & 1)) {
         if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
@@ -1004,8 +1071,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       }
       if (!dead && p >= 0) {
         const uint32_t kt = wtiles + stage * STAGE;
-        tc_block<FP8>(kt, kt + TILE, min(kBS, cur.t1 - (cur.b_begin + i) * kBS), zscale * ks, vs,
-                      qf, w, lane);
+        tc_block<KV>(kt, kt + TILE, min(kBS, cur.t1 - (cur.b_begin + i) * kBS), zscale * ks, vs,
+                     kzc, vzc, qf, w, lane);
       }
       __syncwarp();
       ++g_cons;
@@ -1065,9 +1132,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     }
     // ---- advance ----
     cur = nxt;
-    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs;
+    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs; cur_z = nxt_z;
     nxt = fetch();
-    load_window(nxt, nxt_p, nxt_ks, nxt_vs);
+    load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
     pslot = 0;
     produce();
   }
@@ -1102,7 +1169,7 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dtype kv) {
   auto enc = encoder();
   if (enc == nullptr) return false;
-  const bool fp8 = kv == PA_FP8_E4M3;
+  const bool fp8 = kv != PA_BF16;  // one-byte codes (fp8 or int8), copied as raw bytes
   cuuint64_t dims[2] = {(cuuint64_t)(fp8 ? 128 : 64), (cuuint64_t)total_rows};
   cuuint64_t strides[1] = {128};
   cuuint32_t box[2] = {(cuuint32_t)(fp8 ? 128 : 64), (cuuint32_t)(fp8 ? 16 : 32)};
@@ -1185,7 +1252,8 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
 
 inline bool tc_supported(const pa_decode_desc* d) {
   const int G = d->num_q_heads / d->num_kv_heads;
-  if (d->kv_dtype != PA_BF16 && d->kv_dtype != PA_FP8_E4M3) return false;
+  if (d->kv_dtype != PA_BF16 && d->kv_dtype != PA_FP8_E4M3 && d->kv_dtype != PA_INT8)
+    return false;
   if (d->q_dtype != PA_BF16 || d->out_dtype != PA_BF16) return false;
   if (d->head_dim != tc::kD || d->block_size != kBS || G > 8) return false;
   const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * 32;
@@ -1210,6 +1278,7 @@ inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
 inline cudaError_t launch_tc(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
                              const tc::PlanView* pl, tc::TcKind kind, cudaStream_t st) {
   if (d->kv_dtype == PA_BF16) return tc::launch_tc_kv<PA_BF16>(a, d, grid, pl, kind, st);
+  if (d->kv_dtype == PA_INT8) return tc::launch_tc_kv<PA_INT8>(a, d, grid, pl, kind, st);
   return tc::launch_tc_kv<PA_FP8_E4M3>(a, d, grid, pl, kind, st);
 }
 

@@ -41,7 +41,7 @@ bool desc_supported(const pa_decode_desc* d) {
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return false;
   if (G > 16 || G * d->head_dim > 2048) return false;
   if (d->kv_dtype == PA_F32) return d->q_dtype == PA_F32 && d->out_dtype == PA_F32;
-  if (d->kv_dtype == PA_BF16 || d->kv_dtype == PA_FP8_E4M3)
+  if (d->kv_dtype == PA_BF16 || d->kv_dtype == PA_FP8_E4M3 || d->kv_dtype == PA_INT8)
     return d->q_dtype == PA_BF16 && d->out_dtype == PA_BF16;
   return false;
 }
@@ -119,7 +119,7 @@ using namespace pa;
 
 extern "C" {
 
-const char* pa_version(void) { return "pagedattn 0.1 sm_100a"; }
+const char* pa_version(void) { return "pagedattn 0.2 sm_100a"; }
 
 pa_status pa_set_decode_impl(int impl) {
   if (impl < 0 || impl > 5) return PA_ERR_INVALID;
@@ -136,8 +136,8 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
                             const int32_t* block_tables, const int32_t* context_lens,
                             float scale, void* out, const pa_decode_desc* desc,
                             int max_context_len, const float* k_scales, const float* v_scales,
-                            float* lse_out, void* workspace, size_t workspace_bytes,
-                            void* stream) {
+                            const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
   if (!desc_ok(desc) || max_context_len < 0 || !std::isfinite(scale)) return PA_ERR_INVALID;
   if (!desc_supported(desc)) return PA_ERR_UNSUPPORTED;
   if (desc->num_seqs == 0) return PA_OK;
@@ -146,8 +146,9 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     return PA_ERR_INVALID;
   if ((int64_t)desc->max_blocks_per_seq * desc->block_size < (int64_t)max_context_len)
     return PA_ERR_INVALID;
-  const bool fp8 = desc->kv_dtype == PA_FP8_E4M3;
-  if (fp8 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  const bool quant = desc->kv_dtype == PA_FP8_E4M3 || desc->kv_dtype == PA_INT8;
+  if (quant && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  if (desc->kv_dtype == PA_INT8 && (!k_zeros || !v_zeros)) return PA_ERR_INVALID;
   const WorkspaceLayout wl = layout_for(desc, max_context_len);
   if (wl.total > 0 && (workspace == nullptr || workspace_bytes < wl.total || !aligned16(workspace)))
     return PA_ERR_WORKSPACE;
@@ -157,6 +158,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
   a.block_tables = block_tables; a.context_lens = context_lens;
   a.out = out; a.lse_out = lse_out; a.k_scales = k_scales; a.v_scales = v_scales;
+  a.k_zeros = k_zeros; a.v_zeros = v_zeros;
   a.scale_log2 = scale * kLog2e;
   a.num_seqs = desc->num_seqs; a.num_q_heads = desc->num_q_heads;
   a.num_kv_heads = desc->num_kv_heads; a.group = desc->num_q_heads / desc->num_kv_heads;
@@ -196,6 +198,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     switch (desc->kv_dtype) {
       case PA_F32: e = launch_simt_d<PA_F32>(a, D, gp, grid, st); break;
       case PA_BF16: e = launch_simt_d<PA_BF16>(a, D, gp, grid, st); break;
+      case PA_INT8: e = launch_simt_d<PA_INT8>(a, D, gp, grid, st); break;
       default: e = launch_simt_d<PA_FP8_E4M3>(a, D, gp, grid, st); break;
     }
   }
@@ -208,7 +211,8 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
                             const int64_t* slot_mapping, int num_tokens, int64_t k_stride,
                             int64_t v_stride, int num_kv_heads, int head_dim, int block_size,
                             int num_blocks, pa_dtype in_dtype, pa_dtype cache_dtype,
-                            const float* k_scales, const float* v_scales, void* stream) {
+                            const float* k_scales, const float* v_scales,
+                            const int32_t* k_zeros, const int32_t* v_zeros, void* stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || head_dim % 8 != 0 ||
       block_size <= 0 || num_blocks <= 0)
     return PA_ERR_INVALID;
@@ -223,7 +227,9 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
   if (k_stride % align_elems || v_stride % align_elems || !aligned16(k) || !aligned16(v) ||
       !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
-  if (cache_dtype == PA_FP8_E4M3 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  if ((cache_dtype == PA_FP8_E4M3 || cache_dtype == PA_INT8) && (!k_scales || !v_scales))
+    return PA_ERR_INVALID;
+  if (cache_dtype == PA_INT8 && (!k_zeros || !v_zeros)) return PA_ERR_INVALID;
   const cudaStream_t st = as_stream(stream);
   const dim3 grid(num_tokens);
   const int threads = 128;
@@ -231,15 +237,17 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
 #define PA_RC(IN, C)                                                                          \
   e = launch_pdl(reshape_and_cache_kernel<IN, C>, grid, dim3(threads), 0, st, k, v, k_cache,  \
                  v_cache, slot_mapping, k_stride, v_stride, num_kv_heads, head_dim,          \
-                 block_size, num_blocks, k_scales, v_scales)
+                 block_size, num_blocks, k_scales, v_scales, k_zeros, v_zeros)
   if (in_dtype == PA_F32) {
     if (cache_dtype == PA_F32) PA_RC(PA_F32, PA_F32);
     else if (cache_dtype == PA_BF16) PA_RC(PA_F32, PA_BF16);
     else if (cache_dtype == PA_FP8_E4M3) PA_RC(PA_F32, PA_FP8_E4M3);
+    else if (cache_dtype == PA_INT8) PA_RC(PA_F32, PA_INT8);
     else return PA_ERR_UNSUPPORTED;
   } else {
     if (cache_dtype == PA_BF16) PA_RC(PA_BF16, PA_BF16);
     else if (cache_dtype == PA_FP8_E4M3) PA_RC(PA_BF16, PA_FP8_E4M3);
+    else if (cache_dtype == PA_INT8) PA_RC(PA_BF16, PA_INT8);
     else return PA_ERR_UNSUPPORTED;
   }
 #undef PA_RC
@@ -247,25 +255,29 @@ pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v
 }
 
 pa_status copy_blocks(void* k_cache, void* v_cache, float* k_scales, float* v_scales,
-                      const int32_t* pairs, int num_pairs, int num_kv_heads, int head_dim,
-                      int block_size, int num_blocks, pa_dtype cache_dtype, void* stream) {
+                      int32_t* k_zeros, int32_t* v_zeros, const int32_t* pairs, int num_pairs,
+                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                      pa_dtype cache_dtype, void* stream) {
   if (num_pairs < 0 || num_pairs > 65535 * 1024 || num_kv_heads <= 0 || head_dim <= 0 ||
       block_size <= 0 || num_blocks <= 0)
     return PA_ERR_INVALID;
-  if (cache_dtype != PA_F32 && cache_dtype != PA_BF16 && cache_dtype != PA_FP8_E4M3)
+  if (cache_dtype != PA_F32 && cache_dtype != PA_BF16 && cache_dtype != PA_FP8_E4M3 &&
+      cache_dtype != PA_INT8)
     return PA_ERR_UNSUPPORTED;
   if (num_pairs == 0) return PA_OK;
   if (!k_cache || !v_cache || !pairs || !aligned16(k_cache) || !aligned16(v_cache))
     return PA_ERR_INVALID;
   const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * dtype_bytes(cache_dtype);
   if (block_bytes % 16 != 0) return PA_ERR_INVALID;
-  if (cache_dtype == PA_FP8_E4M3 && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  const bool quant = cache_dtype == PA_FP8_E4M3 || cache_dtype == PA_INT8;
+  if (quant && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  if (cache_dtype == PA_INT8 && (!k_zeros || !v_zeros)) return PA_ERR_INVALID;
+  const bool i8 = cache_dtype == PA_INT8;
   const cudaError_t e = launch_pdl(
       copy_blocks_kernel, dim3(num_pairs, 2), dim3(256), 0, as_stream(stream),
       static_cast<uint8_t*>(k_cache), static_cast<uint8_t*>(v_cache),
-      cache_dtype == PA_FP8_E4M3 ? k_scales : nullptr,
-      cache_dtype == PA_FP8_E4M3 ? v_scales : nullptr, pairs, block_bytes, num_kv_heads,
-      num_blocks);
+      quant ? k_scales : nullptr, quant ? v_scales : nullptr, i8 ? k_zeros : nullptr,
+      i8 ? v_zeros : nullptr, pairs, block_bytes, num_kv_heads, num_blocks);
   return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
@@ -287,7 +299,8 @@ pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
                                     const int32_t* block_tables, const int32_t* context_lens,
                                     float scale, void* out, const pa_decode_desc* desc,
                                     int max_context_len, const float* k_scales,
-                                    const float* v_scales, float* lse_out, void* stream) {
+                                    const float* v_scales, const int32_t* k_zeros,
+                                    const int32_t* v_zeros, float* lse_out, void* stream) {
   if (!desc_ok(desc) || max_context_len < 0) return PA_ERR_INVALID;
   const size_t need = paged_attn_workspace_size(desc, max_context_len);
   if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
@@ -306,7 +319,7 @@ pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
     ws = g_noalloc_ptr[dev];
   }
   return paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, desc,
-                           max_context_len, k_scales, v_scales, lse_out, ws,
+                           max_context_len, k_scales, v_scales, k_zeros, v_zeros, lse_out, ws,
                            ws ? (size_t)PA_NOALLOC_SCRATCH_BYTES : 0, stream);
 }
 

@@ -44,10 +44,10 @@ class DeviceScenario:
         self.max_blocks = max(1, _ceil_div(self.max_context_len, B))
         nb = wl.num_blocks
         self.is_shared = wl.shared_prefix is not None and shared
-        if self.is_shared and wl.kv_dtype == "fp8":
+        if self.is_shared and wl.kv_dtype in ("fp8", "int8"):
             # per-block scales must be fixed before a block's first write; a shared partial
             # block is written before its copies exist, so the recipe has no single value
-            raise NotImplementedError("fp8 cache with a shared prefix")
+            raise NotImplementedError("quantised cache with a shared prefix")
         if wl.shared_prefix is not None and not shared:
             nb = max(nb, S * self.max_blocks)
         order = draw.pool_order if nb == wl.num_blocks else None
@@ -88,6 +88,8 @@ class DeviceScenario:
             k, v = self._seq_kv(s)
             if wl.kv_dtype == "fp8":
                 self._set_scales(s, k, v, tables_host[s])
+            elif wl.kv_dtype == "int8":
+                self._set_int8(s, k, v, tables_host[s])
             a, b = pre_range.get(s, (0, 0))
             if b > a:
                 self._write(k[a:b], v[a:b], pre_slots[s])
@@ -158,6 +160,38 @@ class DeviceScenario:
         self.cache.k_scales[idx] = lk
         self.cache.v_scales[idx] = lv
 
+    def _set_int8(self, s, k, v, table_row):
+        """int8 scale / zero point of sequence s per (logical block, kv head): min/max to the
+        int8 range (the workloads' recipe), placed at the block's physical index."""
+        torch = self.torch
+        wl = self.wl
+        if s in self.draw_seqs:
+            lks, lkz, lvs, lvz = [torch.from_numpy(x).to(self.device)
+                                  for x in self.draw.int8_params_logical(s)]
+        else:
+            n, B = k.shape[0], wl.block_size
+            nb = _ceil_div(n, B)
+            res = []
+            for x in (k, v):
+                xf = x.float()
+                pad = nb * B - n
+                if pad:  # pad with the block's first value so min/max cover valid tokens only
+                    last = xf[(nb - 1) * B:(nb - 1) * B + 1].expand(pad, -1, -1)
+                    xf = torch.cat([xf, last])
+                xb = xf.reshape(nb, B, wl.num_kv_heads, wl.head_dim)
+                mn = xb.amin(dim=(1, 3))
+                mx = xb.amax(dim=(1, 3))
+                sc = (mx - mn) / 255.0
+                flat = mx <= mn
+                sc = torch.where(flat, torch.ones_like(sc), sc)
+                zp = torch.clamp(torch.round(-128.0 - mn / sc), -128, 127).to(torch.int32)
+                zp = torch.where(flat, torch.zeros_like(zp), zp)
+                res += [sc, zp]
+            lks, lkz, lvs, lvz = res
+        idx = torch.from_numpy(table_row[: lks.shape[0]].astype(np.int64)).to(self.device)
+        c = self.cache
+        c.k_scales[idx], c.k_zeros[idx], c.v_scales[idx], c.v_zeros[idx] = lks, lkz, lvs, lvz
+
     def _write(self, k, v, slots: np.ndarray):
         sl = self.torch.from_numpy(np.ascontiguousarray(slots, dtype=np.int64)).to(self.device)
         self.cache.write(k.contiguous(), v.contiguous(), sl)
@@ -180,19 +214,19 @@ class DeviceScenario:
     def kv_bytes(self) -> int:
         """K and V bytes decode must read: every cached token of every (seq, kv head)."""
         wl = self.wl
-        es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+        es = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[wl.kv_dtype]
         return int(self.draw.context_lens.astype(np.int64).sum()) * 2 * wl.num_kv_heads * \
             wl.head_dim * es
 
     def step_bytes(self) -> dict:
         wl = self.wl
         S, Hq, Hkv, d, B = wl.num_seqs, wl.num_q_heads, wl.num_kv_heads, wl.head_dim, wl.block_size
-        es = {"f32": 4, "bf16": 2, "fp8": 1}[wl.kv_dtype]
+        es = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[wl.kv_dtype]
         ins = {"f32": 4, "bf16": 2}[wl.in_dtype]
         lens = self.draw.context_lens.astype(np.int64)
         blocks = int(np.sum(-(-lens // B)))
         kv = self.kv_bytes()
-        scales = (blocks * 2 * Hkv * 4) if wl.kv_dtype == "fp8" else 0
+        scales = {"fp8": blocks * 2 * Hkv * 4, "int8": blocks * 2 * Hkv * 8}.get(wl.kv_dtype, 0)
         qo = S * Hq * d * ins * 2
         meta = blocks * 4 + S * 4
         decode = kv + scales + qo + meta

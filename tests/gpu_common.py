@@ -8,6 +8,7 @@ TOL = {
     "f32": dict(max_abs=1e-4, rel_l2=1e-5, lse=1e-3),
     "bf16": dict(max_abs=2e-2, rel_l2=1e-2, lse=1e-3),
     "fp8": dict(max_abs=3e-2, rel_l2=3e-2, lse=1e-3),
+    "int8": dict(max_abs=3e-2, rel_l2=3e-2, lse=1e-3),
 }
 
 

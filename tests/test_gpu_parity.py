@@ -46,7 +46,8 @@ def _bf16_dev(x):
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("in_dt,cache_dt,d", [("f32", "f32", 64), ("f32", "bf16", 128),
                                               ("bf16", "bf16", 128), ("bf16", "fp8", 128),
-                                              ("f32", "fp8", 64), ("bf16", "bf16", 256)])
+                                              ("f32", "fp8", 64), ("bf16", "bf16", 256),
+                                              ("bf16", "int8", 128), ("f32", "int8", 64)])
 def test_reshape_and_cache_bitexact(pa, in_dt, cache_dt, d):
     rng = np.random.default_rng(hash((in_dt, cache_dt, d)) % 2 ** 32)
     NB, H, B, T = 40, 4, 16, 300
@@ -56,9 +57,12 @@ def test_reshape_and_cache_bitexact(pa, in_dt, cache_dt, d):
     slots[::17] = -1
     ks = rng.uniform(0.01, 2.0, (NB, H)).astype(np.float32)
     vs = rng.uniform(0.01, 2.0, (NB, H)).astype(np.float32)
+    kz = rng.integers(-30, 31, (NB, H)).astype(np.int32)
+    vz = rng.integers(-30, 31, (NB, H)).astype(np.int32)
     kref = opaged.new_cache(NB, H, B, d, cache_dt)
     vref = opaged.new_cache(NB, H, B, d, cache_dt)
-    opaged.ref_reshape_and_cache(xin, xin[::-1].copy(), kref, vref, slots, in_dt, cache_dt, ks, vs)
+    opaged.ref_reshape_and_cache(xin, xin[::-1].copy(), kref, vref, slots, in_dt, cache_dt, ks, vs,
+                                 kz, vz)
     # device inputs: rows strided along T (a wider row buffer) to exercise k_stride
     tdt = torch.float32 if in_dt == "f32" else torch.bfloat16
     pad = 8
@@ -67,37 +71,43 @@ def test_reshape_and_cache_bitexact(pa, in_dt, cache_dt, d):
     wide[:, :H * d] = src.reshape(T, H * d)
     k = wide.cuda()[:, :H * d].view(T, H, d)
     v = src.flip(0).contiguous().cuda()
-    cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}[cache_dt]
+    cdt = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8,
+           "int8": torch.int8}[cache_dt]
     kc = torch.zeros((NB, H, B, d), dtype=cdt, device="cuda")
     vc = torch.zeros_like(kc)
     sc = dict(k_scales=torch.from_numpy(ks).cuda(), v_scales=torch.from_numpy(vs).cuda()) \
-        if cache_dt == "fp8" else {}
+        if cache_dt in ("fp8", "int8") else {}
+    if cache_dt == "int8":
+        sc.update(k_zeros=torch.from_numpy(kz).cuda(), v_zeros=torch.from_numpy(vz).cuda())
     pa.reshape_and_cache(k, v, kc, vc, torch.from_numpy(slots).cuda(), **sc)
     assert pa.device_error() == 0
     assert np.array_equal(cache_codes(kc), kref)
     assert np.array_equal(cache_codes(vc), vref)
 
 
-@pytest.mark.parametrize("cache_dt", ["f32", "bf16", "fp8"])
+@pytest.mark.parametrize("cache_dt", ["f32", "bf16", "fp8", "int8"])
 def test_copy_blocks_bitexact(pa, cache_dt):
     rng = np.random.default_rng(5)
     NB, H, B, d = 64, 8, 16, 128
-    store = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}[cache_dt]
+    store = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8, "int8": np.int8}[cache_dt]
     if cache_dt == "f32":
         k0 = rng.standard_normal((NB, H, B, d)).astype(np.float32)
         v0 = rng.standard_normal((NB, H, B, d)).astype(np.float32)
     else:
-        hi = 2 ** 16 if cache_dt == "bf16" else 256
-        k0 = rng.integers(0, hi, (NB, H, B, d)).astype(store)
-        v0 = rng.integers(0, hi, (NB, H, B, d)).astype(store)
+        lo, hi = {"bf16": (0, 2 ** 16), "fp8": (0, 256), "int8": (-128, 128)}[cache_dt]
+        k0 = rng.integers(lo, hi, (NB, H, B, d)).astype(store)
+        v0 = rng.integers(lo, hi, (NB, H, B, d)).astype(store)
+    quant = cache_dt in ("fp8", "int8")
     ks0 = rng.uniform(size=(NB, H)).astype(np.float32)
     vs0 = rng.uniform(size=(NB, H)).astype(np.float32)
+    kz0 = rng.integers(-128, 128, (NB, H)).astype(np.int32)
+    vz0 = rng.integers(-128, 128, (NB, H)).astype(np.int32)
     srcs = rng.choice(NB, 20, replace=False)
     dsts = rng.choice(np.setdiff1d(np.arange(NB), srcs), 20, replace=False)
     pairs = [(int(s), int(t)) for s, t in zip(srcs, dsts)]
-    kr, vr, ksr, vsr = k0.copy(), v0.copy(), ks0.copy(), vs0.copy()
-    opaged.ref_copy_blocks(kr, vr, pairs, ksr if cache_dt == "fp8" else None,
-                           vsr if cache_dt == "fp8" else None)
+    kr, vr, ksr, vsr, kzr, vzr = k0.copy(), v0.copy(), ks0.copy(), vs0.copy(), kz0.copy(), vz0.copy()
+    opaged.ref_copy_blocks(kr, vr, pairs, ksr if quant else None, vsr if quant else None,
+                           kzr if cache_dt == "int8" else None, vzr if cache_dt == "int8" else None)
 
     def dev(x):
         t = torch.from_numpy(x)
@@ -106,12 +116,15 @@ def test_copy_blocks_bitexact(pa, cache_dt):
         return t.cuda()
     kc, vc = dev(k0), dev(v0)
     ksd, vsd = torch.from_numpy(ks0).cuda(), torch.from_numpy(vs0).cuda()
+    kzd, vzd = torch.from_numpy(kz0).cuda(), torch.from_numpy(vz0).cuda()
     pa.copy_blocks(kc, vc, torch.tensor(pairs, dtype=torch.int32, device="cuda"),
-                   k_scales=ksd if cache_dt == "fp8" else None,
-                   v_scales=vsd if cache_dt == "fp8" else None)
+                   k_scales=ksd if quant else None, v_scales=vsd if quant else None,
+                   k_zeros=kzd if cache_dt == "int8" else None,
+                   v_zeros=vzd if cache_dt == "int8" else None)
     assert pa.device_error() == 0
     assert np.array_equal(cache_codes(kc), kr) and np.array_equal(cache_codes(vc), vr)
     assert np.array_equal(ksd.cpu().numpy(), ksr) and np.array_equal(vsd.cpu().numpy(), vsr)
+    assert np.array_equal(kzd.cpu().numpy(), kzr) and np.array_equal(vzd.cpu().numpy(), vzr)
 
 
 # ---------------------------------------------------------------------------------------
@@ -176,8 +189,9 @@ def test_shared_prefix_workload(pa, scen, impl):
 
 @pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("part", [512, 0])
-def test_batch256_fp8_full_size_sampled(pa, scen, impl, part):
-    d = workloads.draw("b256")
+@pytest.mark.parametrize("name", ["b256", "b256_int8"])
+def test_batch256_full_size_sampled(pa, scen, impl, part, name):
+    d = workloads.draw(name)
     lens = d.context_lens
     sample = sorted({int(np.argmax(lens)), int(np.argmin(lens)), 7, 100, 200, 255})
     _run_and_compare(pa, scen, d, impl, draw_seqs=sample, partition_size=part, check_cache=False)
@@ -193,7 +207,8 @@ def test_long_context_full_size_sampled(pa, scen, impl):
 # invariances, needles, closed forms, edge cases
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("impl", SPLIT_IMPLS)
-@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512)])
+@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512),
+                                       ("b256_int8", 512)])
 def test_physical_placement_bit_identical(pa, scen, impl, name, part):
     wl = workloads.WORKLOADS[name].scaled(num_seqs=6)
     pa.set_decode_impl(impl)
@@ -218,6 +233,7 @@ def test_physical_placement_bit_identical(pa, scen, impl, name, part):
     ("b32", 512, [511, 512, 513, 1024, 1025, 3000]),
     ("b256", 512, [16, 17, 500, 512, 2049, 8192]),
     ("b256", 0, [1, 16, 100, 8192]),
+    ("b256_int8", 512, [16, 17, 500, 513, 2049]),
     ("long", 512, [20000, 513]),
 ])
 def test_ragged_lengths_and_needles(pa, scen, impl, name, part, lens):
@@ -247,7 +263,8 @@ def test_zero_query_is_mean_of_values(pa, scen, impl):
                                             (64, 4, 128, "bf16"), (16, 2, 64, "bf16"),
                                             (8, 1, 256, "bf16"), (32, 8, 128, "fp8"),
                                             (64, 8, 128, "fp8"), (8, 2, 128, "f32"),
-                                            (6, 2, 128, "bf16")])
+                                            (6, 2, 128, "bf16"), (32, 8, 128, "int8"),
+                                            (8, 8, 128, "int8"), (16, 2, 64, "int8")])
 def test_head_shapes(pa, scen, impl, hq, hkv, dim, kv):
     in_dt = "f32" if kv == "f32" else "bf16"
     wl = workloads.Workload("shape", 9, 5, hq, hkv, dim, 16, 512, kv, in_dt,

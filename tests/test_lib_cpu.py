@@ -142,34 +142,45 @@ def test_host_validation_without_device(pa):
     ]
     for b in bad:
         st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
-                                   ctypes.byref(b), 40, nul, nul, nul, nul, 0, nul)
+                                   ctypes.byref(b), 40, nul, nul, nul, nul, nul, nul, 0, nul)
         assert st == pa.PA_ERR_INVALID
     uns = pa.make_desc(4, 4, 2, 96, 3, 32, 0, pa.PA_F32, pa.PA_F32, pa.PA_F32)    # head_dim 96
     st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
-                               ctypes.byref(uns), 40, nul, nul, nul, nul, 0, nul)
+                               ctypes.byref(uns), 40, nul, nul, nul, nul, nul, nul, 0, nul)
     assert st == pa.PA_ERR_UNSUPPORTED
     mixed = pa.make_desc(4, 4, 2, 64, 3, 32, 0, pa.PA_F32, pa.PA_BF16, pa.PA_F32)
     st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
-                               ctypes.byref(mixed), 40, nul, nul, nul, nul, 0, nul)
+                               ctypes.byref(mixed), 40, nul, nul, nul, nul, nul, nul, 0, nul)
     assert st == pa.PA_ERR_UNSUPPORTED
     # null pointers with a valid descriptor are rejected before any launch
     st = lib.paged_attn_decode(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
-                               ctypes.byref(d), 40, nul, nul, nul, nul, 0, nul)
+                               ctypes.byref(d), 40, nul, nul, nul, nul, nul, nul, 0, nul)
     assert st == pa.PA_ERR_INVALID
     # split path without workspace
     st = lib.paged_attn_decode(ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256),
                                ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_float(0.1),
                                ctypes.c_void_p(256), ctypes.byref(d2), 40, nul, nul, nul, nul,
-                               0, nul)
+                               nul, nul, 0, nul)
     assert st == pa.PA_ERR_WORKSPACE
     # zero-sized work is a successful no-op
     assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 0, 128, 128, 2, 64, 16, 32,
-                                 pa.PA_F32, pa.PA_F32, nul, nul, nul) == pa.PA_OK
-    assert lib.copy_blocks(nul, nul, nul, nul, nul, 0, 2, 64, 16, 32, pa.PA_BF16, nul) == pa.PA_OK
+                                 pa.PA_F32, pa.PA_F32, nul, nul, nul, nul, nul) == pa.PA_OK
+    assert lib.copy_blocks(nul, nul, nul, nul, nul, nul, nul, 0, 2, 64, 16, 32, pa.PA_BF16,
+                           nul) == pa.PA_OK
     assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 3, 128, 128, 2, 60, 16, 32,
-                                 pa.PA_F32, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_INVALID
+                                 pa.PA_F32, pa.PA_F32, nul, nul, nul, nul, nul) == pa.PA_ERR_INVALID
     assert lib.reshape_and_cache(nul, nul, nul, nul, nul, 3, 128, 128, 2, 64, 16, 32,
-                                 pa.PA_BF16, pa.PA_F32, nul, nul, nul) == pa.PA_ERR_UNSUPPORTED
+                                 pa.PA_BF16, pa.PA_F32, nul, nul, nul, nul,
+                                 nul) == pa.PA_ERR_UNSUPPORTED
+    # int8 caches need scales and zero points
+    one = ctypes.c_void_p(256)
+    assert lib.reshape_and_cache(one, one, one, one, one, 3, 128, 128, 2, 64, 16, 32,
+                                 pa.PA_BF16, pa.PA_INT8, one, one, nul, nul,
+                                 nul) == pa.PA_ERR_INVALID
+    i8 = pa.make_desc(4, 4, 2, 128, 3, 32, 0, pa.PA_BF16, pa.PA_INT8, pa.PA_BF16)
+    st = lib.paged_attn_decode(one, one, one, one, one, ctypes.c_float(0.1), one, ctypes.byref(i8),
+                               40, one, one, nul, nul, nul, nul, 0, nul)
+    assert st == pa.PA_ERR_INVALID
     assert lib.pa_set_decode_impl(6) == pa.PA_ERR_INVALID
     assert lib.pa_set_decode_impl(-1) == pa.PA_ERR_INVALID
     assert lib.pa_set_decode_impl(0) == pa.PA_OK

@@ -113,3 +113,46 @@ def test_e4m3_roundtrip_all_finite_codes():
     codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
     vals = codecs.e4m3_decode(codes).astype(np.float32)
     assert np.array_equal(codecs.e4m3_encode(vals), codes)
+
+
+def _brute_int8(y, zero):
+    """Nearest code c in [-128, 127] to y + zero with ties to an even (c - zero), then clip."""
+    out = []
+    for yy, z in zip(np.asarray(y, np.float64).ravel(), np.broadcast_to(zero, np.shape(y)).ravel()):
+        lo = int(np.floor(yy))
+        cands = [lo, lo + 1]
+        best = min(cands, key=lambda c: (abs(yy - c), c % 2))
+        out.append(min(127, max(-128, best + int(z))))
+    return np.array(out, dtype=np.int8).reshape(np.shape(y))
+
+
+def test_int8_encode_brute_force_ties_and_clipping():
+    rng = np.random.default_rng(3)
+    y = np.concatenate([rng.uniform(-140, 140, 3000), np.arange(-130, 130) + 0.5,
+                        [0.0, -0.0, 0.5, -0.5, 1.5, -1.5, 2.5, 1e9, -1e9]]).astype(np.float32)
+    zero = rng.integers(-20, 21, y.shape).astype(np.int32)
+    got = codecs.int8_encode(y, zero)
+    assert np.array_equal(got, _brute_int8(y, zero))
+    # ties go to the even integer before the zero point is added
+    assert list(codecs.int8_encode(np.array([0.5, 1.5, 2.5, -0.5, -1.5], np.float32), 3)) == \
+        [3, 5, 5, 3, 1]
+    assert list(codecs.int8_encode(np.array([1e9, -1e9], np.float32), 0)) == [127, -128]
+
+
+def test_int8_roundtrip_and_affine_decode():
+    codes = np.arange(-128, 128).astype(np.int8)
+    for zero in (-128, -7, 0, 9, 127):
+        vals = codecs.int8_decode(codes, zero)            # code - zero, exact
+        assert np.array_equal(vals, np.arange(-128, 128) - zero)
+        assert np.array_equal(codecs.int8_encode(vals.astype(np.float32), zero), codes)
+    # a block quantised with the min/max recipe maps its min and max to the range ends and
+    # every value to within half a step of itself
+    import workloads
+    rng = np.random.default_rng(4)
+    for _ in range(50):
+        x = (rng.standard_normal((16, 128)) * rng.uniform(0.01, 50)).astype(np.float32)
+        scale, zero = workloads._int8_params(x)
+        c = codecs.int8_encode((x / scale).astype(np.float32), zero)
+        back = codecs.int8_decode(c, zero) * float(scale)
+        assert np.abs(back - x).max() <= 0.5 * float(scale) * (1 + 1e-5) + 1e-7
+        assert c.min() <= -127 and c.max() >= 126

@@ -28,7 +28,8 @@ def _call_noalloc(pa, sc, out, lse):
     st = pa._lib.paged_attn_decode_noalloc(
         _ptr(sc.q), _ptr(c.k_cache), _ptr(c.v_cache), _ptr(sc.block_tables),
         _ptr(sc.context_lens), ctypes.c_float(sc.scale), _ptr(out), ctypes.byref(desc),
-        int(sc.max_context_len), _ptr(c.k_scales), _ptr(c.v_scales), _ptr(lse),
+        int(sc.max_context_len), _ptr(c.k_scales), _ptr(c.v_scales), _ptr(c.k_zeros),
+        _ptr(c.v_zeros), _ptr(lse),
         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
     return st, desc
 
@@ -66,5 +67,6 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     assert pa.workspace_size(big, 131072) > pa.NOALLOC_SCRATCH_BYTES
     nul = ctypes.c_void_p(0)
     st = pa._lib.paged_attn_decode_noalloc(nul, nul, nul, nul, nul, ctypes.c_float(0.1), nul,
-                                           ctypes.byref(big), 131072, nul, nul, nul, nul)
+                                           ctypes.byref(big), 131072, nul, nul, nul, nul, nul,
+                                           nul)
     assert st == pa.PA_ERR_WORKSPACE

@@ -19,6 +19,10 @@ Recipe (stated once, used everywhere):
 * fp8 scales: per (sequence, logical block, kv head), ``absmax / 448`` over the bf16 values
   of the block's valid tokens (all ``d`` channels), separately for K and V, computed in
   float32; 1.0 where the absmax is 0. They are inputs of the fp8 cache write, not outputs.
+* int8 scale / zero point: per (sequence, logical block, kv head), from the min and max of
+  the same values: ``scale = (max - min) / 255`` and ``zero = rint(-128 - min / scale)``
+  clipped to [-128, 127] (float32 arithmetic), so that min and max map to the ends of the
+  int8 range; ``scale = 1, zero = 0`` where max == min.
 """
 from __future__ import annotations
 
@@ -43,7 +47,7 @@ class Workload:
     head_dim: int
     block_size: int
     num_blocks: int
-    kv_dtype: str  # "f32" | "bf16" | "fp8"
+    kv_dtype: str  # "f32" | "bf16" | "fp8" | "int8"
     in_dtype: str  # dtype of q and of the new K/V handed to the cache write: "f32" | "bf16"
     lens: Tuple  # ("fixed", [..]) | ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi) | ("const", n)
     partition_size: int = 0  # split-KV partition in tokens; 0 = one pass per (seq, kv head)
@@ -72,6 +76,9 @@ WORKLOADS: Dict[str, Workload] = {
     # 256 seqs, ctx lognormal(median 1024, sigma 1) clipped [16, 8192], fp8 KV, bf16 q/out.
     "b256": Workload("b256", 3, 256, 32, 8, 128, 16, 32768, "fp8", "bf16",
                      ("lognormal", 1024, 1.0, 16, 8192), partition_size=512),
+    # the batch-256 workload with an int8 cache (scale + zero point per block and kv head)
+    "b256_int8": Workload("b256_int8", 3, 256, 32, 8, 128, 16, 32768, "int8", "bf16",
+                          ("lognormal", 1024, 1.0, 16, 8192), partition_size=512),
     # 8 seqs x 131072 tokens, 64q/8kv, d 128, bf16, split into 512-token partitions.
     "long": Workload("long", 4, 8, 64, 8, 128, 16, 65536, "bf16", "bf16", ("const", 131072),
                      partition_size=512),
@@ -96,6 +103,7 @@ def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
 
 
 def _bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    bits = np.asarray(bits)
     return (bits.astype(np.uint32) << 16).view(np.float32)
 
 
@@ -204,6 +212,35 @@ class Draw:
             sc[am == 0] = 1.0
             out.append(sc)
         return out[0], out[1]
+
+    def int8_params_logical(self, s: int):
+        """Per (logical block, kv head) int8 (k_scale, k_zero, v_scale, v_zero) of seq s."""
+        wl = self.wl
+        k, v = self.kv(s)
+        n = int(self.context_lens[s])
+        nb = -(-n // wl.block_size)
+        res = []
+        for x in (k, v):
+            xf = self._as_f32(x)
+            sc = np.ones((nb, wl.num_kv_heads), np.float32)
+            zp = np.zeros((nb, wl.num_kv_heads), np.int32)
+            for b in range(nb):
+                blk = xf[b * wl.block_size:min(n, (b + 1) * wl.block_size)]
+                for h in range(wl.num_kv_heads):
+                    sc[b, h], zp[b, h] = _int8_params(blk[:, h, :])
+            res += [sc, zp]
+        return tuple(res)
+
+
+def _int8_params(x: np.ndarray):
+    """scale, zero of one block's values x (float32 array): min/max to the int8 range."""
+    mn = np.float32(x.min())
+    mx = np.float32(x.max())
+    if mx <= mn:
+        return np.float32(1.0), np.int32(0)
+    scale = np.float32((mx - mn) / np.float32(255.0))
+    zero = np.clip(np.rint(np.float32(-128.0) - mn / scale), -128, 127).astype(np.int32)
+    return scale, zero
 
 
 def draw(name_or_wl, **kw) -> Draw:
