@@ -269,6 +269,37 @@ int pa_alloc_seq_len(const pa_allocator* a, int seq_id);
 /* Writes the free queue front-to-back into out (at most cap entries); returns its size. */
 int pa_alloc_free_queue(const pa_allocator* a, int32_t* out, int cap);
 
+/* ------------------------------------------------------------------------------------- */
+/* Automatic prefix caching ([Ch4PA] "Prefix Caching": a SHA-256 hash of the prefix       */
+/* identifies identical blocks and hits raise ref_count; [KVPaged] "Prefix cache lifetime */
+/* and invalidation": a hit skips recomputing the prefix KV, eviction is least recently   */
+/* used; [KVFail] Key Points: a cached block is evicted when the free queue hands it out). */
+/* Every full block i of a sequence added with its tokens gets the chained hash           */
+/*   h_i = SHA-256(h_{i-1} || tokens of block i as little-endian int32), h_{-1} empty.    */
+/* ------------------------------------------------------------------------------------- */
+/*
+ * New sequence of num_tokens token ids (host int32 tokens[num_tokens]). Its longest run of
+ * leading full blocks whose hashes are cached is reused (ref_count + 1; a cached block
+ * waiting in the free queue is taken out of it); the remaining blocks are popped from the
+ * queue front (a popped block loses any cache entry it had: eviction) and its other full
+ * blocks are registered in the cache. slots_out[num_tokens] receives every token's slot;
+ * *cached_tokens_out (may be NULL) the number of leading tokens whose K/V is already in
+ * the cache (the caller writes only the tokens after them). A freed block keeps its entry
+ * while it waits in the free queue. PA_ERR_NO_BLOCKS (nothing changed) when the free queue,
+ * minus the cached blocks this call reuses, is too short.
+ */
+pa_status pa_alloc_add_seq_tokens(pa_allocator* a, int seq_id, const int32_t* tokens,
+                                  int num_tokens, int64_t* slots_out, int* cached_tokens_out);
+/* Number of blocks with a prefix-cache entry (in use or waiting in the free queue). */
+int pa_alloc_num_cached(const pa_allocator* a);
+/* Totals since creation: blocks reused by hits, cache entries evicted. */
+pa_status pa_alloc_cache_stats(const pa_allocator* a, int64_t* hit_blocks, int64_t* evictions);
+/* Copies block's chained hash (32 bytes) into out32 and returns 1, or returns 0 when the
+ * block has no cache entry. */
+int pa_alloc_block_hash(const pa_allocator* a, int block, uint8_t* out32);
+/* SHA-256 (FIPS 180-4) of len bytes at data into out32: the hash the prefix cache uses. */
+void pa_sha256(const void* data, size_t len, uint8_t* out32);
+
 #ifdef __cplusplus
 }
 #endif

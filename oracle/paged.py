@@ -19,6 +19,7 @@ shared block is copied only when a writer modifies it.
 """
 from __future__ import annotations
 
+import hashlib
 from collections import deque
 from typing import Dict, List, Optional, Sequence, Tuple
 
@@ -55,6 +56,17 @@ class RefAllocator:
       new 16-token boundary crossed. A full shared block is never written, so it is never
       copied. At most one copy pair per call;
     * every call checks first and changes nothing when it fails.
+
+    Automatic prefix caching ([Ch4PA] "Prefix Caching": a SHA-256 hash of the prefix
+    identifies identical blocks, hits raise ref_count; [KVPaged] "Prefix cache lifetime and
+    invalidation": hits skip recomputation, eviction is least recently used; [KVFail] Key
+    Points: a cached block is evicted when the free queue hands it out again):
+    * full block i of a sequence added with ``add_seq_tokens`` has the chained hash
+      h_i = sha256(h_{i-1} + little-endian int32 tokens of block i), h_{-1} = b"";
+    * the longest run of leading full blocks with cached hashes is reused (a waiting block
+      is taken out of the free queue), the other blocks are popped, the new full blocks
+      registered;
+    * a freed block keeps its entry while it waits in the free queue; popping it evicts it.
     """
 
     def __init__(self, num_blocks: int, block_size: int = 16,
@@ -72,6 +84,10 @@ class RefAllocator:
         self.refs: List[int] = [0] * num_blocks
         self.tables: Dict[int, List[int]] = {}
         self.lens: Dict[int, int] = {}
+        self.cache: Dict[bytes, int] = {}        # chained hash -> block
+        self.block_hash: Dict[int, bytes] = {}   # block -> its hash
+        self.hit_blocks = 0
+        self.evictions = 0
 
     # -- queries ------------------------------------------------------------------------
     def num_free(self) -> int:
@@ -89,8 +105,51 @@ class RefAllocator:
     # -- mutations ----------------------------------------------------------------------
     def _pop(self) -> int:
         b = self.free.popleft()
+        if b in self.block_hash:                 # handed out again: evict its entry
+            del self.cache[self.block_hash.pop(b)]
+            self.evictions += 1
         self.refs[b] = 1
         return b
+
+    @staticmethod
+    def chain_hash(parent: Optional[bytes], tokens: Sequence[int]) -> bytes:
+        m = hashlib.sha256()
+        if parent is not None:
+            m.update(parent)
+        m.update(np.asarray(tokens, dtype="<i4").tobytes())
+        return m.digest()
+
+    def add_seq_tokens(self, seq: int, tokens: Sequence[int]) -> Tuple[np.ndarray, int]:
+        if seq in self.tables:
+            raise InvalidCall("add_seq_tokens")
+        B = self.block_size
+        n = len(tokens)
+        nfull, nblk = n // B, -(-n // B)
+        hashes: List[bytes] = []
+        hits: List[int] = []
+        for i in range(nfull):
+            hashes.append(self.chain_hash(hashes[-1] if i else None, tokens[i * B:(i + 1) * B]))
+            if len(hits) == i and hashes[i] in self.cache:
+                hits.append(self.cache[hashes[i]])
+        waiting = sum(1 for b in hits if self.refs[b] == 0)
+        if nblk - len(hits) > len(self.free) - waiting:
+            raise NoBlocks()
+        row = []
+        for b in hits:
+            if self.refs[b] == 0:
+                self.free.remove(b)
+            self.refs[b] += 1
+            row.append(b)
+        for i in range(len(hits), nblk):
+            b = self._pop()
+            row.append(b)
+            if i < nfull:
+                self.cache[hashes[i]] = b
+                self.block_hash[b] = hashes[i]
+        self.hit_blocks += len(hits)
+        self.tables[seq] = row
+        self.lens[seq] = n
+        return self._slots(seq, 0, n), len(hits) * B
 
     def _slots(self, seq: int, start: int, n: int) -> np.ndarray:
         row = self.tables[seq]

@@ -82,6 +82,11 @@ _SIGS = {
     "pa_alloc_seq_len": (_i, [_vp, _i]),
     "pa_alloc_free_queue": (_i, [_vp, _vp, _i]),
     "pa_set_decode_impl": (_i, [_i]),
+    "pa_alloc_add_seq_tokens": (_i, [_vp, _i, _vp, _i, _vp, _P(_i)]),
+    "pa_alloc_num_cached": (_i, [_vp]),
+    "pa_alloc_cache_stats": (_i, [_vp, _P(_i64), _P(_i64)]),
+    "pa_alloc_block_hash": (_i, [_vp, _i, _vp]),
+    "pa_sha256": (None, [_vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -291,6 +296,14 @@ def device_error(stream=None) -> int:
     return bits.value
 
 
+def sha256(data: bytes) -> bytes:
+    """SHA-256 computed by the library (the hash its prefix cache chains)."""
+    buf = (ctypes.c_uint8 * 32)()
+    b = bytes(data)
+    _lib.pa_sha256(ctypes.c_char_p(b), len(b), buf)
+    return bytes(buf)
+
+
 class BlockAllocator:
     """Host block allocator (FIFO free queue, ref_count, fork, append with copy-on-write)."""
 
@@ -325,6 +338,32 @@ class BlockAllocator:
         _check(_lib.pa_alloc_add_seq(self._h, int(seq), int(num_tokens),
                                      slots.ctypes.data_as(ctypes.c_void_p)), "pa_alloc_add_seq")
         return slots
+
+    def add_seq_tokens(self, seq: int, tokens) -> Tuple[np.ndarray, int]:
+        """New sequence with token ids (prefix caching): returns (slots, cached_tokens)."""
+        tok = np.ascontiguousarray(tokens, dtype=np.int32)
+        slots = np.empty(tok.size, dtype=np.int64)
+        cached = ctypes.c_int(0)
+        _check(_lib.pa_alloc_add_seq_tokens(self._h, int(seq), tok.ctypes.data_as(ctypes.c_void_p),
+                                            int(tok.size), slots.ctypes.data_as(ctypes.c_void_p),
+                                            ctypes.byref(cached)), "pa_alloc_add_seq_tokens")
+        return slots, cached.value
+
+    def num_cached(self) -> int:
+        return _lib.pa_alloc_num_cached(self._h)
+
+    def cache_stats(self) -> Tuple[int, int]:
+        """(blocks reused by hits, cache entries evicted) since creation."""
+        h, e = ctypes.c_int64(0), ctypes.c_int64(0)
+        _check(_lib.pa_alloc_cache_stats(self._h, ctypes.byref(h), ctypes.byref(e)),
+               "pa_alloc_cache_stats")
+        return h.value, e.value
+
+    def block_hash(self, block: int) -> Optional[bytes]:
+        buf = (ctypes.c_uint8 * 32)()
+        if not _lib.pa_alloc_block_hash(self._h, int(block), buf):
+            return None
+        return bytes(buf)
 
     def fork(self, parent: int, child: int) -> None:
         _check(_lib.pa_alloc_fork(self._h, int(parent), int(child)), "pa_alloc_fork")
