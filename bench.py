@@ -347,16 +347,27 @@ def _traffic_note(name, version):
     return e.get("bytes_per_launch")
 
 
+def _last_block_waste(lens, block_size):
+    """Idle slots in the last blocks / allocated slots over the batch."""
+    lens = np.asarray(lens, dtype=np.int64)
+    alloc = int(((lens + block_size - 1) // block_size).sum()) * block_size
+    return (alloc - int(lens.sum())) / alloc if alloc else 0.0
+
+
 def _extra_workloads(torch, pa, args, flush):
     from paged_kv_cache_465_b200.scenario import DeviceScenario
     peak, _ = _peaks()
     out = {}
-    for name in ("tiny", "b32", "shared", "b256", "long", "b256_int8"):
-        if name == args.workload:
-            continue
-        draw = workloads.draw(name)
-        sc = DeviceScenario(draw, draw_seqs=[] if name in ("b256", "long", "b32", "b256_int8")
-                            else None)
+    # the named workloads, then the batch-256 fp8 workload with 8- and 32-token blocks (the
+    # block-size trade-off: last-block waste against table length and tile size)
+    runs = [(n, workloads.WORKLOADS[n]) for n in ("tiny", "b32", "shared", "b256", "long",
+                                                   "b256_int8") if n != args.workload]
+    base = workloads.WORKLOADS["b256"]
+    runs += [(f"b256_bs{B}", base.scaled(block_size=B, num_blocks=base.num_blocks * 16 // B))
+             for B in (8, 32)]
+    for name, wl in runs:
+        draw = workloads.draw(wl)
+        sc = DeviceScenario(draw, draw_seqs=[] if name not in ("tiny", "shared") else None)
         for _ in range(3):
             flush()
             sc.step()
@@ -370,7 +381,10 @@ def _extra_workloads(torch, pa, args, flush):
                      "decode_ms": round(dec * 1e3, 5),
                      "decode_gbs": round(b["decode"] / dec / 1e9, 2),
                      "tokens_per_s": round(draw.wl.num_seqs / (total / steps), 1),
-                     "partition_size": sc.partition_size, "steps": steps}
+                     "partition_size": sc.partition_size, "block_size": wl.block_size,
+                     "last_block_waste": round(_last_block_waste(draw.context_lens,
+                                                                 wl.block_size), 6),
+                     "steps": steps}
         del sc
         torch.cuda.empty_cache()
     return out

@@ -1,8 +1,8 @@
 /*
  * pagedattn.h — C ABI of libpagedattn.so, paged decode attention for NVIDIA B200 (sm_100a).
  *
- * Scope: the decode-step hot path of PagedAttention. The KV cache is cut into fixed
- * 16-token blocks scattered through a physical block pool; a per-sequence block table maps
+ * Scope: the decode-step hot path of PagedAttention. The KV cache is cut into fixed-size
+ * blocks (8, 16 or 32 tokens; 16 by default) scattered through a physical block pool; a per-sequence block table maps
  * logical blocks to physical ones; sequences with a common prefix share physical blocks,
  * counted by ref_count, and a shared block is copied before it is written (copy-on-write).
  * Sources (page title, section):
@@ -38,13 +38,15 @@
  *   h / (num_q_heads / num_kv_heads) ([KVPaged] "GQA and MQA": query heads are grouped and
  *   each group shares one KV head).
  * - block_tables: int32 [num_seqs][max_blocks_per_seq]; entry b of row s is the physical
- *   block holding logical tokens [16b, 16b+16) of sequence s; entries at or beyond
+ *   block holding logical tokens [B*b, B*b+B) of sequence s (B = block_size); entries at or beyond
  *   ceil(context_lens[s] / block_size) are never read ([Ch4PA] "PagedAttention algorithm":
  *   the block table maps logical block ids to physical blocks that need not be contiguous).
  * - context_lens[s] counts every cached token of sequence s, including the token being
  *   decoded (whose K/V must have been written by reshape_and_cache first).
  *
- * Supported today: block_size 16; head_dim 64, 128 or 256; num_q_heads a multiple of
+ * Supported today: block_size 8, 16 or 32 ([KVPaged] "the block-size knob" and [Ch4PA]
+ * "Theorem 1, fragmentation bound": smaller blocks waste less of the last block, larger
+ * ones need shorter tables; 16 is the usual default); head_dim 64, 128 or 256; num_q_heads a multiple of
  * num_kv_heads with a group of at most 16; (q, kv, out) dtypes (f32, f32, f32),
  * (bf16, bf16, bf16), (bf16, fp8_e4m3, bf16) and (bf16, int8, bf16). Anything else returns
  * PA_ERR_UNSUPPORTED.
@@ -84,10 +86,11 @@ typedef struct {
   int num_q_heads;         /* Hq                                                       */
   int num_kv_heads;        /* Hkv; Hq % Hkv == 0                                       */
   int head_dim;            /* d                                                        */
-  int block_size;          /* tokens per block (16)                                    */
+  int block_size;          /* tokens per block: 8, 16 or 32                            */
   int max_blocks_per_seq;  /* row stride of block_tables                               */
   int num_blocks;          /* physical blocks in the pool (bounds check)               */
-  int partition_size;      /* split-KV partition in tokens, a multiple of block_size;  */
+  int partition_size;      /* split-KV partition in tokens, a multiple of block_size   */
+                           /* and of 16;                                               */
                            /* 0 = one pass over the whole context per (seq, kv head)   */
   pa_dtype q_dtype, kv_dtype, out_dtype;
 } pa_decode_desc;

@@ -25,7 +25,9 @@
 namespace pa {
 
 constexpr int kSimtWarps = 4;
-constexpr int kBS = 16;  // tokens per block (template constant of the whole library)
+// Tokens per sub-tile: the unit every decode kernel steps through. A block of 32 tokens is
+// two sub-tiles, a block of 8 tokens half of one.
+constexpr int kSub = 16;
 
 template <pa_dtype KV>
 struct KvTraits;
@@ -115,7 +117,8 @@ struct DecodeArgs {
   float scale_log2;  // scale * log2(e)
   int num_seqs, num_q_heads, num_kv_heads, group;
   int max_blocks_per_seq, num_blocks;
-  int part_tokens;   // tokens per work item (a multiple of 16)
+  int block_size;    // tokens per physical block: 8, 16 or 32
+  int part_tokens;   // tokens per work item (a multiple of 16 and of the block size)
   int max_parts;     // P: partitions per sequence in the workspace
   int max_context_len;
   int final_pass;    // 1: one item covers the whole context, write out directly
@@ -169,10 +172,9 @@ decode_simt_kernel(const DecodeArgs a) {
   constexpr int CH = HALF / EPC;            // chunks per lane per token row
   constexpr int NV = D / 32;                // channels per lane in the P.V phase
   constexpr int QROW = D + 4;               // padded q row (floats); halves in different banks
-  constexpr int TILE = kBS * D * ES;        // bytes of one (block, head) tile
 
   __shared__ __align__(16) float sq[GP * QROW];
-  __shared__ __align__(16) float sp[kSimtWarps][kBS][GP];
+  __shared__ __align__(16) float sp[kSimtWarps][kSub][GP];
   __shared__ float sm[kSimtWarps][GP], sl[kSimtWarps][GP];
   __shared__ __align__(16) float sacc[kSimtWarps][GP][D];
 
@@ -202,56 +204,68 @@ decode_simt_kernel(const DecodeArgs a) {
     for (int j = 0; j < NV; ++j) acc[g][j] = 0.f;
   }
 
+  // Tokens are taken in 16-token chunks of logical positions (any block size): lane
+  // (tok, half) owns token 16c + tok of chunk c, looks its block up in the table and reads
+  // its row at ((block * Hkv + kvh) * block_size + offset) * D elements.
   const int tok = lane & 15, half = lane >> 4;
-  const int b_begin = t0 / kBS, b_end = (t1 + kBS - 1) / kBS;
+  const int BS = a.block_size;
+  const int c_begin = t0 / kSub, c_end = (t1 + kSub - 1) / kSub;
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
   const uint8_t* kbase = static_cast<const uint8_t*>(a.k_cache);
   const uint8_t* vbase = static_cast<const uint8_t*>(a.v_cache);
 
-  for (int b = b_begin + warp; b < b_end; b += kSimtWarps) {
-    int phys = bt[b];
-    if (phys < 0 || phys >= a.num_blocks) {
-      if (lane == 0) flag_error(PA_DEVERR_BLOCK_ID);
-      continue;
-    }
-    const int64_t tile = ((int64_t)phys * a.num_kv_heads + kvh) * TILE;
+  for (int c = c_begin + warp; c < c_end; c += kSimtWarps) {
+    const int t = c * kSub + tok;
+    bool valid = t >= t0 && t < t1;
+    int64_t row = -1;  // byte offset of the token's K / V row, -1 when not read
     float ks = 1.f, vs = 1.f, kz = 0.f, vz = 0.f;
-    if constexpr (KV == PA_FP8_E4M3 || KV == PA_INT8) {
-      ks = a.k_scales[(int64_t)phys * a.num_kv_heads + kvh];
-      vs = a.v_scales[(int64_t)phys * a.num_kv_heads + kvh];
+    if (valid) {
+      const int phys = bt[t / BS];
+      if (phys < 0 || phys >= a.num_blocks) {
+        if (half == 0) flag_error(PA_DEVERR_BLOCK_ID);
+        valid = false;
+      } else {
+        const int64_t bh = (int64_t)phys * a.num_kv_heads + kvh;
+        row = (bh * BS + t % BS) * D * ES;
+        if constexpr (KV == PA_FP8_E4M3 || KV == PA_INT8) {
+          ks = a.k_scales[bh];
+          vs = a.v_scales[bh];
+        }
+        if constexpr (KV == PA_INT8) {
+          kz = (float)a.k_zeros[bh];
+          vz = (float)a.v_zeros[bh];
+        }
+      }
     }
-    if constexpr (KV == PA_INT8) {
-      kz = (float)a.k_zeros[(int64_t)phys * a.num_kv_heads + kvh];
-      vz = (float)a.v_zeros[(int64_t)phys * a.num_kv_heads + kvh];
-    }
+    if (!__any_sync(0xffffffffu, valid)) continue;
     // ---- scores: lane (tok, half) -> partial dot over its half of d ----
     float sc[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) sc[g] = 0.f;
-    const uint4* krow = reinterpret_cast<const uint4*>(kbase + tile + (int64_t)tok * D * ES + half * HALF * ES);
+    if (valid) {
+      const uint4* krow = reinterpret_cast<const uint4*>(kbase + row + half * HALF * ES);
 #pragma unroll
-    for (int c = 0; c < CH; ++c) {
-      float kx[EPC];
-      unpack16<KV>(__ldg(krow + c), kx);
-      if constexpr (KV == PA_INT8) {
+      for (int cc = 0; cc < CH; ++cc) {
+        float kx[EPC];
+        unpack16<KV>(__ldg(krow + cc), kx);
+        if constexpr (KV == PA_INT8) {
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) kx[e] -= kz;  // exact: small integers
-      }
+          for (int e = 0; e < EPC; ++e) kx[e] -= kz;  // exact: small integers
+        }
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        const float* qr = sq + g * QROW + half * (HALF + 4) + c * EPC;
+        for (int g = 0; g < GP; ++g) {
+          const float* qr = sq + g * QROW + half * (HALF + 4) + cc * EPC;
 #pragma unroll
-        for (int e = 0; e < EPC; e += 4) {
-          float4 qv = *reinterpret_cast<const float4*>(qr + e);
-          sc[g] = fmaf(qv.x, kx[e], sc[g]);
-          sc[g] = fmaf(qv.y, kx[e + 1], sc[g]);
-          sc[g] = fmaf(qv.z, kx[e + 2], sc[g]);
-          sc[g] = fmaf(qv.w, kx[e + 3], sc[g]);
+          for (int e = 0; e < EPC; e += 4) {
+            float4 qv = *reinterpret_cast<const float4*>(qr + e);
+            sc[g] = fmaf(qv.x, kx[e], sc[g]);
+            sc[g] = fmaf(qv.y, kx[e + 1], sc[g]);
+            sc[g] = fmaf(qv.z, kx[e + 2], sc[g]);
+            sc[g] = fmaf(qv.w, kx[e + 3], sc[g]);
+          }
         }
       }
     }
-    const int t = b * kBS + tok;
-    const bool valid = t >= t0 && t < t1;
     float p[GP];
 #pragma unroll
     for (int g = 0; g < GP; ++g) {
@@ -262,7 +276,7 @@ decode_simt_kernel(const DecodeArgs a) {
       bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
       bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
       bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-      const float mn = fmaxf(m[g], bm);   // finite: the block holds a valid token
+      const float mn = fmaxf(m[g], bm);   // finite: the chunk holds a valid token
       const float alpha = fast_exp2(m[g] - mn);
       m[g] = mn;
       p[g] = valid ? fast_exp2(z - mn) : 0.f;
@@ -276,15 +290,19 @@ decode_simt_kernel(const DecodeArgs a) {
     }
     __syncwarp();
     // ---- P.V: lane -> channels [lane*NV, lane*NV + NV) ----
-    // tokens past the context are skipped: their slots may hold anything (even NaN)
-    const int nv = min(kBS, t1 - b * kBS);
+    // tokens past the item or in an unreadable block are skipped (their rows may hold
+    // anything, even NaN)
+    const int nv = min(kSub, t1 - c * kSub);
 #pragma unroll 4
     for (int tt = 0; tt < nv; ++tt) {
+      const int64_t r = __shfl_sync(0xffffffffu, row, tt);
+      if (r < 0) continue;
       float vx[NV];
-      load_vslice<KV, D>(vbase + tile + (int64_t)tt * D * ES, lane, vx);
+      load_vslice<KV, D>(vbase + r, lane, vx);
       if constexpr (KV == PA_INT8) {
+        const float z = __shfl_sync(0xffffffffu, vz, tt);
 #pragma unroll
-        for (int j = 0; j < NV; ++j) vx[j] -= vz;
+        for (int j = 0; j < NV; ++j) vx[j] -= z;
       }
 #pragma unroll
       for (int g = 0; g < GP; ++g) {

@@ -37,6 +37,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <type_traits>
+
 #include "decode_simt.cuh"
 
 namespace pa {
@@ -280,24 +282,34 @@ __device__ __forceinline__ float load_q_frags(const uint16_t* qp, int G, int lan
 // block inside the work item; zs: log2-domain score scale (x fp8 K scale); vs: fp8 V scale.
 // The K products run as two independent accumulation chains and the V fragments are read
 // before the softmax, so a warp has independent work in flight at every step.
+// Per-half dequantisation parameters of a 16-token sub-tile: tokens 0-7 come from one
+// block and 8-15 from another when blocks hold 8 tokens; otherwise both halves are equal.
+struct HalfParams {
+  float zs0, zs1;              // log2-domain score scale (x K scale) of each half
+  float vs0, vs1;              // V scale of each half
+  uint32_t kzc0, kzc1;         // int8: f16x2 (1152 + K zero point) of each half
+  uint32_t vzc0, vzc1;         // int8: f16x2 (1152 + V zero point) of each half
+};
+
 template <pa_dtype KV>
-__device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, float zs,
-                                         float vs, uint32_t kzc, uint32_t vzc,
-                                         const uint32_t (&qf)[8][2], WarpAcc& w, int lane) {
+__device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid,
+                                         const HalfParams& hp, const uint32_t (&qf)[8][2],
+                                         WarpAcc& w, int lane) {
   constexpr bool FP8 = KV != PA_BF16;  // one-byte codes, f16 products
   constexpr bool I8 = KV == PA_INT8;
   constexpr int TILE = FP8 ? 2048 : 4096;
   const int gq = lane >> 2;
-  float pv = 1.f, beta = 1.f;
+  float pv0 = 1.f, pv1 = 1.f, beta = 1.f;
   if constexpr (FP8) {
-    const float vnew = fmaxf(w.vref, vs);
+    const float vnew = fmaxf(w.vref, fmaxf(hp.vs0, hp.vs1));
     beta = w.vref > 0.f ? w.vref / vnew : 1.f;
-    pv = vnew > 0.f ? vs / vnew : 0.f;
+    pv0 = vnew > 0.f ? hp.vs0 / vnew : 0.f;
+    pv1 = vnew > 0.f ? hp.vs1 / vnew : 0.f;
     w.vref = vnew;
   }
   // rows of tokens past the item may hold anything (even NaN): zero them before P.V reads
-  if (nvalid < kBS) {
-    const int bytes_per_tok = TILE / kBS;
+  if (nvalid < kSub) {
+    const int bytes_per_tok = TILE / kSub;
     for (int o = nvalid * bytes_per_tok + lane * 16; o < TILE; o += 32 * 16)
       asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(vt + o), "r"(0) : "memory");
     __syncwarp();
@@ -329,13 +341,14 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
         // a register holds 4 consecutive channels of one token: pairs (0,1) and (2,3)
         uint32_t x0[4], x1[4];
         if constexpr (I8) {
+          // registers 0 and 2 hold tokens 0-7, registers 1 and 3 tokens 8-15
           uint32_t u[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) u[e] = r[cp][e] ^ 0x80808080u;
-          x0[0] = i8x2_to_f16x2(u[0], 0x4140, kzc); x0[1] = i8x2_to_f16x2(u[1], 0x4140, kzc);
-          x0[2] = i8x2_to_f16x2(u[0], 0x4342, kzc); x0[3] = i8x2_to_f16x2(u[1], 0x4342, kzc);
-          x1[0] = i8x2_to_f16x2(u[2], 0x4140, kzc); x1[1] = i8x2_to_f16x2(u[3], 0x4140, kzc);
-          x1[2] = i8x2_to_f16x2(u[2], 0x4342, kzc); x1[3] = i8x2_to_f16x2(u[3], 0x4342, kzc);
+          x0[0] = i8x2_to_f16x2(u[0], 0x4140, hp.kzc0); x0[1] = i8x2_to_f16x2(u[1], 0x4140, hp.kzc1);
+          x0[2] = i8x2_to_f16x2(u[0], 0x4342, hp.kzc0); x0[3] = i8x2_to_f16x2(u[1], 0x4342, hp.kzc1);
+          x1[0] = i8x2_to_f16x2(u[2], 0x4140, hp.kzc0); x1[1] = i8x2_to_f16x2(u[3], 0x4140, hp.kzc1);
+          x1[2] = i8x2_to_f16x2(u[2], 0x4342, hp.kzc0); x1[3] = i8x2_to_f16x2(u[3], 0x4342, hp.kzc1);
         } else {
           x0[0] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][0])); x0[1] = e4m3x2_to_f16x2((uint16_t)lo16(r[cp][1]));
           x0[2] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][0])); x0[3] = e4m3x2_to_f16x2((uint16_t)hi16(r[cp][1]));
@@ -364,8 +377,10 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
   }
   // ---- online softmax (log2 domain); thread holds tokens gq, gq+8 x heads 2tq, 2tq+1 ----
   const bool va = gq < nvalid, vb = gq + 8 < nvalid;
-  const float z0 = va ? (sa[0] + sb[0]) * zs : -INFINITY, z1 = va ? (sa[1] + sb[1]) * zs : -INFINITY;
-  const float z2 = vb ? (sa[2] + sb[2]) * zs : -INFINITY, z3 = vb ? (sa[3] + sb[3]) * zs : -INFINITY;
+  const float z0 = va ? (sa[0] + sb[0]) * hp.zs0 : -INFINITY;
+  const float z1 = va ? (sa[1] + sb[1]) * hp.zs0 : -INFINITY;
+  const float z2 = vb ? (sa[2] + sb[2]) * hp.zs1 : -INFINITY;
+  const float z3 = vb ? (sa[3] + sb[3]) * hp.zs1 : -INFINITY;
   float bm0 = fmaxf(z0, z2), bm1 = fmaxf(z1, z3);
 #pragma unroll
   for (int o = 4; o < 32; o <<= 1) {
@@ -390,8 +405,8 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
   // P^T as B fragments: pack [token][head] pairs, transpose 8x8 in registers
   uint32_t pb0, pb1;
   if constexpr (FP8) {
-    pb0 = movm_t(pack_f16x2(p0 * pv, p1 * pv));
-    pb1 = movm_t(pack_f16x2(p2 * pv, p3 * pv));
+    pb0 = movm_t(pack_f16x2(p0 * pv0, p1 * pv0));
+    pb1 = movm_t(pack_f16x2(p2 * pv1, p3 * pv1));
   } else {
     pb0 = movm_t(pack_bf16x2(p0, p1));
     pb1 = movm_t(pack_bf16x2(p2, p3));
@@ -408,10 +423,10 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid, f
       uint32_t ev[4], od[4];
       if constexpr (I8) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 4; ++e) {  // registers 0, 1: tokens 0-7; 2, 3: tokens 8-15
           const uint32_t u = vr[cp][e] ^ 0x80808080u;
-          ev[e] = i8x2_to_f16x2(u, 0x4240, vzc);
-          od[e] = i8x2_to_f16x2(u, 0x4341, vzc);
+          ev[e] = i8x2_to_f16x2(u, 0x4240, e < 2 ? hp.vzc0 : hp.vzc1);
+          od[e] = i8x2_to_f16x2(u, 0x4341, e < 2 ? hp.vzc0 : hp.vzc1);
         }
       } else {
 #pragma unroll
@@ -482,9 +497,131 @@ __device__ __forceinline__ void combine_warps(const float* sacc, const float* sm
 }
 
 // =======================================================================================
-// Single pass: one CTA per (sequence, kv head) work item, grid (1, Hkv, S).
+// Block-table view of 16-token sub-tiles (any block size: 8, 16 or 32 tokens)
 // =======================================================================================
+// Sub-tile c covers logical tokens [16c, 16c + 16). Blocks of 16 or 32 tokens hold one or
+// two whole sub-tiles (contiguous in the (block, kv head) region); with 8-token blocks a
+// sub-tile has two halves from two blocks, each with its own scales.
+struct SubWin {
+  int p0, p1;          // physical blocks of the halves; p1 = -3: second half absent
+  float ks0, vs0, ks1, vs1;
+  uint32_t z0, z1;     // int8: packed (K, V) zero points
+};
+
+template <pa_dtype KV, int BS>
+__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
+                                         int t1, int kvh, SubWin& w) {
+  auto one = [&](int blk, int& p, float& ks, float& vs, uint32_t& z) {
+    p = btrow[blk];
+    ks = 1.f;
+    vs = 1.f;
+    z = 0;
+    if (p < 0 || p >= a.num_blocks) {
+      flag_error(PA_DEVERR_BLOCK_ID);
+      p = -1;
+      return;
+    }
+    if constexpr (KV != PA_BF16) {
+      const int64_t bh = (int64_t)p * a.num_kv_heads + kvh;
+      ks = a.k_scales[bh];
+      vs = a.v_scales[bh];
+      if constexpr (KV == PA_INT8) z = pack_zeros(a.k_zeros[bh], a.v_zeros[bh]);
+    }
+  };
+  if constexpr (BS == 8) {
+    one(2 * c, w.p0, w.ks0, w.vs0, w.z0);
+    if (c * kSub + 8 < t1) {
+      one(2 * c + 1, w.p1, w.ks1, w.vs1, w.z1);
+    } else {
+      w.p1 = -3; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
+    }
+  } else {
+    one(c * kSub / BS, w.p0, w.ks0, w.vs0, w.z0);
+    w.p1 = w.p0; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
+  }
+}
+
+__device__ __forceinline__ void empty_sub(SubWin& w) {
+  w.p0 = -2; w.p1 = -3; w.ks0 = w.vs0 = w.ks1 = w.vs1 = 1.f; w.z0 = w.z1 = 0;
+}
+
+// Lane k's window entry, broadcast to the warp.
+template <int BS>
+__device__ __forceinline__ SubWin shfl_sub(const SubWin& w, int k) {
+  SubWin r;
+  r.p0 = __shfl_sync(0xffffffffu, w.p0, k);
+  r.ks0 = __shfl_sync(0xffffffffu, w.ks0, k);
+  r.vs0 = __shfl_sync(0xffffffffu, w.vs0, k);
+  r.z0 = __shfl_sync(0xffffffffu, w.z0, k);
+  if constexpr (BS == 8) {
+    r.p1 = __shfl_sync(0xffffffffu, w.p1, k);
+    r.ks1 = __shfl_sync(0xffffffffu, w.ks1, k);
+    r.vs1 = __shfl_sync(0xffffffffu, w.vs1, k);
+    r.z1 = __shfl_sync(0xffffffffu, w.z1, k);
+  } else {
+    r.p1 = r.p0; r.ks1 = r.ks0; r.vs1 = r.vs0; r.z1 = r.z0;
+  }
+  return r;
+}
+
+// A sub-tile the consumer can use: its blocks exist and are in range.
+__device__ __forceinline__ bool sub_ok(const SubWin& w) { return w.p0 >= 0 && w.p1 != -1; }
+
+// Lane 0: TMA copies of sub-tile c's K and V tiles into the stage at dst (V at dst + TILE),
+// completing on bar; a plain arrive when the sub-tile is skipped.
+template <pa_dtype KV, int BS>
+__device__ __forceinline__ void issue_sub(uint32_t dst, const CUtensorMap* kmap,
+                                          const CUtensorMap* vmap, uint32_t bar,
+                                          uint64_t policy, const SubWin& w, int c, int kvh,
+                                          int Hkv) {
+  constexpr int TILE = TcCfg<KV>::kTile, R16 = TcCfg<KV>::kRows;
+  // the stage was last read (and maybe written) through the generic proxy
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (!sub_ok(w)) {
+    mbar_arrive(bar);  // completes the phase; the consumer skips the sub-tile
+    return;
+  }
+  if constexpr (BS == 8) {
+    constexpr int HALF = TILE / 2, R8 = R16 / 2;
+    const bool two = w.p1 >= 0;
+    mbar_arrive_tx(bar, (two ? 4u : 2u) * HALF);
+    const int r0 = (w.p0 * Hkv + kvh) * R8;
+    tma_load_2d(dst, kmap, 0, r0, bar, policy);
+    tma_load_2d(dst + TILE, vmap, 0, r0, bar, policy);
+    if (two) {
+      const int r1 = (w.p1 * Hkv + kvh) * R8;
+      tma_load_2d(dst + HALF, kmap, 0, r1, bar, policy);
+      tma_load_2d(dst + TILE + HALF, vmap, 0, r1, bar, policy);
+    }
+  } else {
+    constexpr int PER = BS / kSub;  // sub-tiles per block
+    const int row = ((w.p0 * Hkv + kvh) * PER + c % PER) * R16;
+    mbar_arrive_tx(bar, 2 * TILE);
+    tma_load_2d(dst, kmap, 0, row, bar, policy);
+    tma_load_2d(dst + TILE, vmap, 0, row, bar, policy);
+  }
+}
+
 template <pa_dtype KV>
+__device__ __forceinline__ HalfParams half_params(const SubWin& w, float zscale) {
+  HalfParams h;
+  h.zs0 = zscale * w.ks0;
+  h.zs1 = zscale * w.ks1;
+  h.vs0 = w.vs0;
+  h.vs1 = w.vs1;
+  h.kzc0 = h.kzc1 = h.vzc0 = h.vzc1 = 0;
+  if constexpr (KV == PA_INT8) {
+    zero_consts(w.z0, h.kzc0, h.vzc0);
+    zero_consts(w.z1, h.kzc1, h.vzc1);
+  }
+  return h;
+}
+
+// =======================================================================================
+// One CTA per work item, grid (partitions, Hkv, S): warp w takes the item's sub-tiles
+// w, w+4, ... through its own TMA ring; warps merge through shared memory at the end.
+// =======================================================================================
+template <pa_dtype KV, int BS>
 __global__ void __launch_bounds__(kNW * 32)
 decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
                  const __grid_constant__ CUtensorMap vmap) {
@@ -518,55 +655,27 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
       static_cast<const uint16_t*>(a.q) + ((int64_t)s * a.num_q_heads + kvh * G) * kD, G, lane,
       a.scale_log2, qf);
 
-  // ---- this warp's blocks and its block-table windows (32 entries per register) ----
-  const int b_begin = t0 / kBS, b_end = (t1 + kBS - 1) / kBS;
-  const int nblk = b_end - b_begin;
-  const int nmine = nblk > warp ? (nblk - warp + kNW - 1) / kNW : 0;
+  // ---- this warp's sub-tiles and their block-table windows (32 per register set) ----
+  const int c_begin = t0 / kSub, c_end = (t1 + kSub - 1) / kSub;
+  const int nsub = c_end - c_begin;
+  const int nmine = nsub > warp ? (nsub - warp + kNW - 1) / kNW : 0;
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
-  auto load_window = [&](int base, int& p, float& ks, float& vs, uint32_t& z) {
+  auto sub_of = [&](int k) { return c_begin + warp + k * kNW; };
+  auto load_window = [&](int base, SubWin& w) {
     const int k = base + lane;
-    p = -2;
-    ks = 1.f;
-    vs = 1.f;
-    z = 0;
-    if (k < nmine) {
-      p = bt[b_begin + warp + k * kNW];
-      if (p < 0 || p >= a.num_blocks) {
-        flag_error(PA_DEVERR_BLOCK_ID);
-        p = -1;
-      } else if constexpr (FP8) {
-        ks = a.k_scales[(int64_t)p * a.num_kv_heads + kvh];
-        vs = a.v_scales[(int64_t)p * a.num_kv_heads + kvh];
-        if constexpr (KV == PA_INT8)
-          z = pack_zeros(a.k_zeros[(int64_t)p * a.num_kv_heads + kvh],
-                         a.v_zeros[(int64_t)p * a.num_kv_heads + kvh]);
-      }
-    }
+    if (k < nmine) load_sub<KV, BS>(a, bt, sub_of(k), t1, kvh, w);
+    else empty_sub(w);
   };
-  int cur_p, nxt_p;
-  float cur_ks, cur_vs, nxt_ks, nxt_vs;
-  uint32_t cur_z, nxt_z;
-  load_window(0, cur_p, cur_ks, cur_vs, cur_z);
-  load_window(32, nxt_p, nxt_ks, nxt_vs, nxt_z);
+  SubWin cur, nxt;
+  load_window(0, cur);
+  load_window(32, nxt);
   const uint64_t policy = evict_first_policy();
   auto issue = [&](int k, int wbase, int stage) {
     const int rel = k - wbase;
-    const int p = rel < 32 ? __shfl_sync(0xffffffffu, cur_p, rel)
-                           : __shfl_sync(0xffffffffu, nxt_p, rel - 32);
-    if (lane == 0) {
-      const uint32_t bar = bars + 8 * stage;
-      // the stage was last read (and maybe written) through the generic proxy
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      if (p >= 0) {
-        const int row = (p * a.num_kv_heads + kvh) * C::kRows;
-        const uint32_t dst = wtiles + stage * STAGE;
-        mbar_arrive_tx(bar, STAGE);
-        tma_load_2d(dst, &kmap, 0, row, bar, policy);
-        tma_load_2d(dst + TILE, &vmap, 0, row, bar, policy);
-      } else {
-        mbar_arrive(bar);  // completes the phase; the consumer skips the block
-      }
-    }
+    const SubWin w = rel < 32 ? shfl_sub<BS>(cur, rel) : shfl_sub<BS>(nxt, rel - 32);
+    if (lane == 0)
+      issue_sub<KV, BS>(wtiles + stage * STAGE, &kmap, &vmap, bars + 8 * stage, policy, w,
+                        sub_of(k), kvh, a.num_kv_heads);
   };
   for (int k = 0; k < NST && k < nmine; ++k) issue(k, 0, k);
 
@@ -577,25 +686,21 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
   for (int i = 0; i < nmine; ++i) {
     const int wbase = i & ~31;
     if ((i & 31) == 0 && i > 0) {
-      cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs; cur_z = nxt_z;
-      load_window(i + 32, nxt_p, nxt_ks, nxt_vs, nxt_z);
+      cur = nxt;
+      load_window(i + 32, nxt);
     }
     const int stage = i % NST;
-    const int p = __shfl_sync(0xffffffffu, cur_p, i & 31);
-    const float ks = __shfl_sync(0xffffffffu, cur_ks, i & 31);
-    const float vs = __shfl_sync(0xffffffffu, cur_vs, i & 31);
-    uint32_t kzc = 0, vzc = 0;
-    if constexpr (KV == PA_INT8) zero_consts(__shfl_sync(0xffffffffu, cur_z, i & 31), kzc, vzc);
+    const SubWin sw = shfl_sub<BS>(cur, i & 31);
     if (!mbar_wait(bars + 8 * stage, (uint32_t)((i / NST) & 1))) {
       if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
       timed_out = true;
       break;
     }
     consumed = i + 1;
-    if (p >= 0) {
-      const int b = b_begin + warp + i * kNW;
+    if (sub_ok(sw)) {
+      const int c = sub_of(i);
       const uint32_t kt = wtiles + stage * STAGE;
-      tc_block<KV>(kt, kt + TILE, min(kBS, t1 - b * kBS), zscale * ks, vs, kzc, vzc, qf, w,
+      tc_block<KV>(kt, kt + TILE, min(kSub, t1 - c * kSub), half_params<KV>(sw, zscale), qf, w,
                    lane);
     }
     __syncwarp();
@@ -637,7 +742,7 @@ struct PlanView {
   int2* list;
 };
 
-// One CTA of 1024 threads: counts partitions per size (blocks per item), orders them
+// One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
 // largest first (full partitions, then partial ones by size), writes the list, zeroes the
 // fetch counter, and writes out = 0 / lse = -inf for empty sequences.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
@@ -645,7 +750,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   pdl_wait();
   pdl_trigger();
   const int P = a.part_tokens;
-  const int nbk = P / kBS;  // blocks of a full partition (<= 128)
+  const int nbk = P / kSub;  // sub-tiles of a full partition (<= 128)
   for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
@@ -660,7 +765,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
     }
     const int full = ctx / P, rem = ctx % P;
     if (full) atomicAdd(&cnt[nbk], full);
-    if (rem) atomicAdd(&cnt[(rem + kBS - 1) / kBS], 1);
+    if (rem) atomicAdd(&cnt[(rem + kSub - 1) / kSub], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -680,7 +785,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       const int base = atomicAdd(&off[nbk], full);
       for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
     }
-    if (rem) pl.list[atomicAdd(&off[(rem + kBS - 1) / kBS], 1)] = make_int2(s, full);
+    if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
   }
 }
 
@@ -689,6 +794,7 @@ struct ItemSlot {
   int valid, s, part, kvh;
 };
 
+// Persistent CTAs: 16-token blocks only (a block is one sub-tile).
 template <pa_dtype KV>
 __global__ void __launch_bounds__(kNW * 32)
 decode_tc_persistent(const DecodeArgs a, const PlanView pl,
@@ -752,8 +858,8 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       const int ctx = checked_ctx(a, x.s);
       const int t0 = x.part * P;
       v.t1 = min(ctx, t0 + P);
-      v.b_begin = t0 / kBS;
-      const int nblk = (v.t1 + kBS - 1) / kBS - v.b_begin;
+      v.b_begin = t0 / kSub;
+      const int nblk = (v.t1 + kSub - 1) / kSub - v.b_begin;
       v.nmine = nblk > warp ? (nblk - warp + kNW - 1) / kNW : 0;
       v.np = (ctx + P - 1) / P;
     }
@@ -843,8 +949,8 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       if (!dead && p >= 0) {
         const int b = cur.b_begin + warp + i * kNW;
         const uint32_t kt = wtiles + stage * STAGE;
-        tc_block<KV>(kt, kt + TILE, min(kBS, cur.t1 - b * kBS), zscale * ks, vs, kzc, vzc, qf,
-                     w, lane);
+        const HalfParams hp{zscale * ks, zscale * ks, vs, vs, kzc, kzc, vzc, vzc};
+        tc_block<KV>(kt, kt + TILE, min(kSub, cur.t1 - b * kSub), hp, qf, w, lane);
       }
       __syncwarp();
       ++g_cons;
@@ -917,7 +1023,7 @@ struct TcwCfg {
       kWW * kNStage * TcCfg<KV>::kStage + kWW * kQBytes + kWW * (kNStage + 1) * 8 + 1024;
 };
 
-template <pa_dtype KV>
+template <pa_dtype KV, int BS>
 __global__ void __launch_bounds__(kWW * 32, PA_TCW_MIN_WARPS / kWW)
 decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap) {
@@ -946,8 +1052,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   const uint32_t total = pl.counters[1];
   const uint64_t policy = evict_first_policy();
 
+  // an item's sub-tiles are c_begin + k, k < nsub (<= 32)
   struct Item {
-    int valid, s, kvh, part, t1, b_begin, nblk, np;
+    int valid, s, kvh, part, t1, c_begin, nsub, np;
   };
   auto fetch = [&]() {
     uint32_t it = 0;
@@ -963,30 +1070,19 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       v.kvh = (int)(it % Hkv);
       v.part = sp.y;
       v.t1 = min(ctx, t0 + P);
-      v.b_begin = t0 / kBS;
-      v.nblk = (v.t1 + kBS - 1) / kBS - v.b_begin;
+      v.c_begin = t0 / kSub;
+      v.nsub = (v.t1 + kSub - 1) / kSub - v.c_begin;
       v.np = (ctx + P - 1) / P;
     }
     return v;
   };
-  // lane k holds block k's (phys, ks, vs, packed zero points) of an item
-  auto load_window = [&](const Item& v, int& p, float& ks, float& vs, uint32_t& z) {
-    p = -2;
-    ks = 1.f;
-    vs = 1.f;
-    z = 0;
-    if (v.valid && lane < v.nblk) {
-      p = a.block_tables[(int64_t)v.s * a.max_blocks_per_seq + v.b_begin + lane];
-      if (p < 0 || p >= a.num_blocks) {
-        flag_error(PA_DEVERR_BLOCK_ID);
-        p = -1;
-      } else if constexpr (FP8) {
-        ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
-        vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
-        if constexpr (KV == PA_INT8)
-          z = pack_zeros(a.k_zeros[(int64_t)p * Hkv + v.kvh], a.v_zeros[(int64_t)p * Hkv + v.kvh]);
-      }
-    }
+  // lane k holds sub-tile k's blocks, scales and zero points of an item
+  auto load_window = [&](const Item& v, SubWin& w) {
+    if (v.valid && lane < v.nsub)
+      load_sub<KV, BS>(a, a.block_tables + (int64_t)v.s * a.max_blocks_per_seq, v.c_begin + lane,
+                       v.t1, v.kvh, w);
+    else
+      empty_sub(w);
   };
   // lane 0: copy an item's q group (G rows, contiguous) into this warp's q buffer
   uint32_t qwaits = 0;  // q copies waited for (barrier phase)
@@ -1004,11 +1100,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
 
   Item cur = fetch();
   Item nxt = fetch();
-  int cur_p, nxt_p;
-  float cur_ks, cur_vs, nxt_ks, nxt_vs;
-  uint32_t cur_z, nxt_z;
-  load_window(cur, cur_p, cur_ks, cur_vs, cur_z);
-  load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
+  SubWin cur_w, nxt_w;
+  load_window(cur, cur_w);
+  load_window(nxt, nxt_w);
   copy_q(cur);
 
   int pslot = 0, pk = 0;
@@ -1016,25 +1110,14 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   bool dead = false;
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
-      if (pslot == 0 && pk >= cur.nblk) { pslot = 1; pk = 0; }
-      if (pslot == 1 && (!nxt.valid || pk >= nxt.nblk)) break;
-      const int kvh = pslot == 0 ? cur.kvh : nxt.kvh;
-      const int p = __shfl_sync(0xffffffffu, pslot == 0 ? cur_p : nxt_p, pk);
+      if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
+      if (pslot == 1 && (!nxt.valid || pk >= nxt.nsub)) break;
+      const Item& v = pslot == 0 ? cur : nxt;
+      const SubWin sw = shfl_sub<BS>(pslot == 0 ? cur_w : nxt_w, pk);
       const int stage = g_iss % NST;
-      if (lane == 0) {
-        const uint32_t bar = bars + 8 * stage;
-        // the stage was last read (and maybe written) through the generic proxy
-        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-        if (p >= 0) {
-          const int row = (p * Hkv + kvh) * C::kRows;
-          const uint32_t dst = wtiles + stage * STAGE;
-          mbar_arrive_tx(bar, STAGE);
-          tma_load_2d(dst, &kmap, 0, row, bar, policy);
-          tma_load_2d(dst + TILE, &vmap, 0, row, bar, policy);
-        } else {
-          mbar_arrive(bar);  // completes the phase; the consumer skips the block
-        }
-      }
+      if (lane == 0)
+        issue_sub<KV, BS>(wtiles + stage * STAGE, &kmap, &vmap, bars + 8 * stage, policy, sw,
+                          v.c_begin + pk, v.kvh, Hkv);
       ++g_iss;
       ++pk;
     }
@@ -1058,21 +1141,17 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     __syncwarp();
     if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
     w.reset();
-    for (int i = 0; i < cur.nblk; ++i) {
-      const int p = __shfl_sync(0xffffffffu, cur_p, i);
-      const float ks = __shfl_sync(0xffffffffu, cur_ks, i);
-      const float vs = __shfl_sync(0xffffffffu, cur_vs, i);
-      uint32_t kzc = 0, vzc = 0;
-      if constexpr (KV == PA_INT8) zero_consts(__shfl_sync(0xffffffffu, cur_z, i), kzc, vzc);
+    for (int i = 0; i < cur.nsub; ++i) {
+      const SubWin sw = shfl_sub<BS>(cur_w, i);
       const int stage = g_cons % NST;
       if (!dead && !mbar_wait(bars + 8 * stage, (g_cons / NST) & 1)) {
         if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
         dead = true;
       }
-      if (!dead && p >= 0) {
+      if (!dead && sub_ok(sw)) {
         const uint32_t kt = wtiles + stage * STAGE;
-        tc_block<KV>(kt, kt + TILE, min(kBS, cur.t1 - (cur.b_begin + i) * kBS), zscale * ks, vs,
-                     kzc, vzc, qf, w, lane);
+        tc_block<KV>(kt, kt + TILE, min(kSub, cur.t1 - (cur.c_begin + i) * kSub),
+                     half_params<KV>(sw, zscale), qf, w, lane);
       }
       __syncwarp();
       ++g_cons;
@@ -1132,9 +1211,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     }
     // ---- advance ----
     cur = nxt;
-    cur_p = nxt_p; cur_ks = nxt_ks; cur_vs = nxt_vs; cur_z = nxt_z;
+    cur_w = nxt_w;
     nxt = fetch();
-    load_window(nxt, nxt_p, nxt_ks, nxt_vs, nxt_z);
+    load_window(nxt, nxt_w);
     pslot = 0;
     produce();
   }
@@ -1165,14 +1244,17 @@ inline PFN_cuTensorMapEncodeTiled_v12000 encoder() {
   return fn;
 }
 
-// The pool seen as rows of 128 bytes: a (block, head) tile is kRows consecutive rows.
-inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dtype kv) {
+// The pool seen as rows of 128 bytes: a token's K (or V) is one row (one-byte codes) or
+// two (bf16); a box is one 16-token sub-tile, or half of one for 8-token blocks.
+inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dtype kv,
+                     int block_size) {
   auto enc = encoder();
   if (enc == nullptr) return false;
   const bool fp8 = kv != PA_BF16;  // one-byte codes (fp8 or int8), copied as raw bytes
+  const int box_tokens = block_size < kSub ? block_size : kSub;
   cuuint64_t dims[2] = {(cuuint64_t)(fp8 ? 128 : 64), (cuuint64_t)total_rows};
   cuuint64_t strides[1] = {128};
-  cuuint32_t box[2] = {(cuuint32_t)(fp8 ? 128 : 64), (cuuint32_t)(fp8 ? 16 : 32)};
+  cuuint32_t box[2] = {(cuuint32_t)(fp8 ? 128 : 64), (cuuint32_t)(box_tokens * (fp8 ? 1 : 2))};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(base), dims, strides, box, estr,
@@ -1205,21 +1287,21 @@ inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
   return e;
 }
 
-template <pa_dtype KV>
+template <pa_dtype KV, int BS>
 inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
                                 const PlanView* pl, TcKind kind, cudaStream_t st) {
   using C = TcCfg<KV>;
-  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * C::kRows;
+  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * BS * (C::kFp8 ? 1 : 2);
   CUtensorMap km, vm;
-  if (!make_map(&km, a.k_cache, rows, KV) || !make_map(&vm, a.v_cache, rows, KV))
+  if (!make_map(&km, a.k_cache, rows, KV, BS) || !make_map(&vm, a.v_cache, rows, KV, BS))
     return cudaErrorInvalidValue;
   if (kind == kTcGrid) {
     static int per_sm = 0;
     if (per_sm == 0) {
-      cudaError_t e = occupancy(decode_tc_kernel<KV>, kNW * 32, C::kSmem, &per_sm);
+      cudaError_t e = occupancy(decode_tc_kernel<KV, BS>, kNW * 32, C::kSmem, &per_sm);
       if (e != cudaSuccess) { per_sm = 0; return e; }
     }
-    decode_tc_kernel<KV><<<grid, kNW * 32, C::kSmem, st>>>(a, km, vm);
+    decode_tc_kernel<KV, BS><<<grid, kNW * 32, C::kSmem, st>>>(a, km, vm);
     return cudaGetLastError();
   }
   const int sms = sm_count();
@@ -1227,6 +1309,7 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, a, *pl);
   if (e != cudaSuccess) return e;
   if (kind == kTcCta) {
+    if constexpr (BS != kSub) return cudaErrorInvalidValue;
     static int per_sm = 0;
     if (per_sm == 0) {
       e = occupancy(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, &per_sm);
@@ -1238,11 +1321,11 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   } else {
     static int per_sm = 0;
     if (per_sm == 0) {
-      e = occupancy(decode_tc_warps<KV>, kWW * 32, TcwCfg<KV>::kSmem, &per_sm);
+      e = occupancy(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, &per_sm);
       if (e != cudaSuccess) { per_sm = 0; return e; }
     }
-    e = launch_pdl(decode_tc_warps<KV>, dim3(sms * per_sm), dim3(kWW * 32), TcwCfg<KV>::kSmem,
-                   st, a, *pl, km, vm);
+    e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32),
+                   TcwCfg<KV>::kSmem, st, a, *pl, km, vm);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();
@@ -1255,19 +1338,21 @@ inline bool tc_supported(const pa_decode_desc* d) {
   if (d->kv_dtype != PA_BF16 && d->kv_dtype != PA_FP8_E4M3 && d->kv_dtype != PA_INT8)
     return false;
   if (d->q_dtype != PA_BF16 || d->out_dtype != PA_BF16) return false;
-  if (d->head_dim != tc::kD || d->block_size != kBS || G > 8) return false;
-  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * 32;
+  if (d->head_dim != tc::kD || G > 8) return false;
+  if (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) return false;
+  const int64_t rows = (int64_t)d->num_blocks * d->num_kv_heads * d->block_size * 2;
   return rows < (int64_t)1 << 31;
 }
 
 // Which tensor-core kernel runs a call. impl: 2 = automatic, 3 = grid, 4 = persistent
 // CTAs, 5 = persistent warps. The persistent kernels need the split path (a workspace for
-// the plan) and keep one partition's blocks per warp in 32-entry register windows:
-// persistent CTAs up to 32 * 4 blocks (2048 tokens), warp workers up to 32 blocks (512).
+// the plan) and keep one partition's 16-token sub-tiles per warp in 32-entry register
+// windows: persistent CTAs (16-token blocks only) up to 32 * 4 sub-tiles (2048 tokens),
+// warp workers up to 32 sub-tiles (512 tokens).
 inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
   const int P = d->partition_size;
-  const bool cta_ok = split && P <= 32 * tc::kNW * kBS;
-  const bool warps_ok = split && P <= 32 * kBS;
+  const bool cta_ok = split && d->block_size == kSub && P <= 32 * tc::kNW * kSub;
+  const bool warps_ok = split && P <= 32 * kSub;
   if (impl == 3) return tc::kTcGrid;
   if (impl == 4) return cta_ok ? tc::kTcCta : tc::kTcGrid;
   if (impl == 5) return warps_ok ? tc::kTcWarps : (cta_ok ? tc::kTcCta : tc::kTcGrid);
@@ -1277,9 +1362,15 @@ inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
 
 inline cudaError_t launch_tc(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
                              const tc::PlanView* pl, tc::TcKind kind, cudaStream_t st) {
-  if (d->kv_dtype == PA_BF16) return tc::launch_tc_kv<PA_BF16>(a, d, grid, pl, kind, st);
-  if (d->kv_dtype == PA_INT8) return tc::launch_tc_kv<PA_INT8>(a, d, grid, pl, kind, st);
-  return tc::launch_tc_kv<PA_FP8_E4M3>(a, d, grid, pl, kind, st);
+  auto by_bs = [&](auto kv) -> cudaError_t {
+    constexpr pa_dtype KV = decltype(kv)::value;
+    if (d->block_size == 8) return tc::launch_tc_kv<KV, 8>(a, d, grid, pl, kind, st);
+    if (d->block_size == 32) return tc::launch_tc_kv<KV, 32>(a, d, grid, pl, kind, st);
+    return tc::launch_tc_kv<KV, 16>(a, d, grid, pl, kind, st);
+  };
+  if (d->kv_dtype == PA_BF16) return by_bs(std::integral_constant<pa_dtype, PA_BF16>{});
+  if (d->kv_dtype == PA_INT8) return by_bs(std::integral_constant<pa_dtype, PA_INT8>{});
+  return by_bs(std::integral_constant<pa_dtype, PA_FP8_E4M3>{});
 }
 
 }  // namespace pa

@@ -37,7 +37,8 @@ bool desc_ok(const pa_decode_desc* d) {
 
 bool desc_supported(const pa_decode_desc* d) {
   const int G = d->num_q_heads / d->num_kv_heads;
-  if (d->block_size != kBS) return false;
+  if (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) return false;
+  if (d->partition_size % kSub != 0) return false;  // partitions start on 16-token sub-tiles
   if (d->head_dim != 64 && d->head_dim != 128 && d->head_dim != 256) return false;
   if (G > 16 || G * d->head_dim > 2048) return false;
   if (d->kv_dtype == PA_F32) return d->q_dtype == PA_F32 && d->out_dtype == PA_F32;
@@ -119,7 +120,7 @@ using namespace pa;
 
 extern "C" {
 
-const char* pa_version(void) { return "pagedattn 0.2 sm_100a"; }
+const char* pa_version(void) { return "pagedattn 0.3 sm_100a"; }
 
 pa_status pa_set_decode_impl(int impl) {
   if (impl < 0 || impl > 5) return PA_ERR_INVALID;
@@ -163,6 +164,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   a.num_seqs = desc->num_seqs; a.num_q_heads = desc->num_q_heads;
   a.num_kv_heads = desc->num_kv_heads; a.group = desc->num_q_heads / desc->num_kv_heads;
   a.max_blocks_per_seq = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
+  a.block_size = desc->block_size;
   a.max_context_len = max_context_len;
   a.q_dtype = desc->q_dtype; a.out_dtype = desc->out_dtype;
   const bool split = wl.total > 0;
@@ -175,7 +177,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     a.max_parts = wl.parts;
     a.final_pass = 0;
   } else {
-    a.part_tokens = (int)round_up((size_t)(max_context_len > 0 ? max_context_len : 1), kBS);
+    a.part_tokens = (int)round_up((size_t)(max_context_len > 0 ? max_context_len : 1), kSub);
     a.max_parts = 1;
     a.final_pass = 1;
   }

@@ -316,3 +316,95 @@ def test_empty_context_and_error_flags(pa):
     assert torch.equal(kc[1:], before[1:]) and torch.equal(kc[0, :, 6:], before[0, :, 6:])
     pa.copy_blocks(kc, vc, torch.tensor([[0, NB]], dtype=torch.int32, device="cuda"))
     assert pa.device_error() & pa.PA_DEVERR_PAIR
+
+
+# ---------------------------------------------------------------------------------------
+# block sizes 8 and 32 ("the block-size knob"; Theorem 1 trade-off note)
+# ---------------------------------------------------------------------------------------
+def _bs(name, B, **kw):
+    wl = workloads.WORKLOADS[name]
+    return wl.scaled(block_size=B, num_blocks=wl.num_blocks * 16 // B, **kw)
+
+
+@pytest.mark.parametrize("B", [8, 32])
+@pytest.mark.parametrize("impl", ["simt", "auto"])
+def test_block_sizes_tiny_and_shared(pa, scen, B, impl):
+    _run_and_compare(pa, scen, workloads.draw(_bs("tiny", B)), impl)
+    d = workloads.draw(_bs("shared", B, num_seqs=20))
+    sc, _ = _run_and_compare(pa, scen, d, impl)
+    # a 200-token prefix fills 25 blocks of 8 exactly (nothing to copy); with 32-token
+    # blocks its last block holds 8 tokens and every child copies it before appending
+    assert len(sc.cow_pairs) == (0 if B == 8 else 19)
+
+
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
+@pytest.mark.parametrize("B", [8, 32])
+@pytest.mark.parametrize("name,part,seqs", [("b32", 0, 32), ("b32", 512, 32), ("b256", 512, 12),
+                                            ("b256", 0, 6), ("b256_int8", 512, 12)])
+def test_block_sizes_workloads(pa, scen, impl, B, name, part, seqs):
+    _run_and_compare(pa, scen, workloads.draw(_bs(name, B, num_seqs=seqs)), impl,
+                     partition_size=part)
+
+
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
+@pytest.mark.parametrize("B", [8, 32])
+@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512),
+                                       ("b256_int8", 512)])
+def test_block_sizes_ragged_needles_and_placement(pa, scen, impl, B, name, part):
+    lens = [1, 7, 8, 9, 15, 16, 17, 24, 31, 32, 33, 40, 511, 513, 1000]
+    wl = _bs(name, B, num_seqs=len(lens))
+    for needle in (False, True):
+        _run_and_compare(pa, scen, workloads.draw(wl, lens_override=lens, needle=needle), impl,
+                         partition_size=part)
+    pa.set_decode_impl(impl)
+    try:
+        d1 = workloads.draw(wl, lens_override=lens)
+        s1 = scen(d1, partition_size=part)
+        s1.step()
+        d2 = workloads.draw(wl, lens_override=lens)
+        d2.pool_order = np.roll(d2.pool_order[::-1], 5).copy()
+        s2 = scen(d2, partition_size=part)
+        s2.step()
+        torch.cuda.synchronize()
+        assert not torch.equal(s1.block_tables, s2.block_tables)
+        assert torch.equal(s1.out, s2.out) and torch.equal(s1.lse, s2.lse)
+    finally:
+        pa.set_decode_impl("auto")
+
+
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
+@pytest.mark.parametrize("B", [8, 32])
+@pytest.mark.parametrize("hq,hkv,dim,kv", [(64, 4, 128, "bf16"), (8, 1, 256, "bf16"),
+                                            (32, 8, 128, "fp8"), (16, 2, 64, "int8"),
+                                            (8, 2, 128, "f32")])
+def test_block_sizes_head_shapes(pa, scen, impl, B, hq, hkv, dim, kv):
+    in_dt = "f32" if kv == "f32" else "bf16"
+    wl = workloads.Workload("shape", 9, 5, hq, hkv, dim, B, 8192 // B, kv, in_dt,
+                            ("fixed", [1, 9, 100, 700, 1500]))
+    for part in (0, 256, 1024):
+        _run_and_compare(pa, scen, workloads.draw(wl), impl, partition_size=part)
+
+
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
+def test_block_size_8_bad_second_half_is_flagged(pa, impl):
+    """A 16-token sub-tile of 8-token blocks whose second block id is out of range: that
+    block is skipped and flagged, the rest of the context still decodes."""
+    S, Hq, Hkv, d, B, NB = 2, 8, 2, 128, 8, 16
+    q = torch.randn(S, Hq, d, device="cuda").to(torch.bfloat16)
+    kc = torch.randn(NB, Hkv, B, d, device="cuda").to(torch.bfloat16)
+    vc = torch.randn(NB, Hkv, B, d, device="cuda").to(torch.bfloat16)
+    bt = torch.tensor([[0, 1_000_000, 2, 3], [4, 5, 6, 7]], dtype=torch.int32, device="cuda")
+    out = torch.empty_like(q)
+    pa.set_decode_impl(impl)
+    try:
+        for part in (0, 16):
+            ws = torch.empty(1 << 20, dtype=torch.uint8, device="cuda")
+            pa.paged_attn_decode(q, kc, vc, bt, torch.tensor([30, 30], dtype=torch.int32,
+                                                             device="cuda"),
+                                 0.1, out, max_context_len=32, partition_size=part,
+                                 workspace=ws)
+            assert pa.device_error() & pa.PA_DEVERR_BLOCK_ID
+            assert pa.device_error() == 0
+            assert torch.isfinite(out.float()).all()
+    finally:
+        pa.set_decode_impl("auto")

@@ -22,8 +22,9 @@ def _contig(draw, s):
     return dec(k), dec(v), dec(draw.q[s])
 
 
-def test_tiny_against_textbook_loops():
-    d = workloads.draw("tiny")
+@pytest.mark.parametrize("B,nb", [(16, 32), (8, 64), (32, 16)])
+def test_tiny_against_textbook_loops(B, nb):
+    d = workloads.draw(workloads.WORKLOADS["tiny"].scaled(block_size=B, num_blocks=nb))
     st = flows.build_state(d)
     out, lse = flows.ref_outputs(d, st)
     wl = d.wl
@@ -37,8 +38,10 @@ def test_tiny_against_textbook_loops():
             assert lse[s, h] == pytest.approx(l, abs=1e-12)
 
 
-def test_lse_matches_scipy():
-    d = workloads.draw(workloads.WORKLOADS["b32"].scaled(num_seqs=3, num_blocks=1024),
+@pytest.mark.parametrize("B", [16, 8, 32])
+def test_lse_matches_scipy(B):
+    d = workloads.draw(workloads.WORKLOADS["b32"].scaled(num_seqs=3, num_blocks=16384 // B,
+                                                        block_size=B),
                        lens_override=[7, 300, 1000])
     st = flows.build_state(d)
     out, lse = flows.ref_outputs(d, st)
@@ -130,8 +133,9 @@ def test_shared_prefix_matches_unshared_copies():
     assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
 
 
-def test_fp8_dequant_is_code_times_scale():
-    wl = workloads.WORKLOADS["b256"].scaled(num_seqs=3, num_blocks=256)
+@pytest.mark.parametrize("B", [16, 8, 32])
+def test_fp8_dequant_is_code_times_scale(B):
+    wl = workloads.WORKLOADS["b256"].scaled(num_seqs=3, num_blocks=4096 // B, block_size=B)
     d = workloads.draw(wl, lens_override=[16, 33, 500])
     st = flows.build_state(d)
     out, lse = flows.ref_outputs(d, st)
@@ -142,7 +146,7 @@ def test_fp8_dequant_is_code_times_scale():
         K, V = attention.gather_kv(st.k_cache, st.v_cache, st.block_tables[s],
                                    int(d.context_lens[s]), 2, "fp8", st.k_scales, st.v_scales)
         err = np.abs(K - kf[:, 2])
-        blk = np.arange(len(K)) // 16
+        blk = np.arange(len(K)) // B
         sc = st.k_scales[st.block_tables[s][blk], 2][:, None]
         # relative step of E4M3 is 2^-3 for normals -> half-step error <= 2^-4 |x|,
         # subnormal step 2^-9 * scale

@@ -80,3 +80,19 @@ def test_sharing_savings(golden):
     b = facts.block_table_bytes(o["requests"], 2048)
     assert b == 131072
     assert abs(b - o["printed_bytes_approx"]) / o["printed_bytes_approx"] < 0.01
+
+
+@pytest.mark.parametrize("B", [8, 32])
+def test_fragmentation_bound_other_block_sizes(B):
+    """[Ch4PA] Theorem 1 trade-off note: halving the block size halves the bound, doubling
+    doubles it; the proof's step (at most B - 1 idle slots per request) holds for any B."""
+    T = 2048
+    assert facts.waste_bound(T, B) == facts.waste_bound(T, 16) * B / 16
+    rng = np.random.default_rng(B)
+    for _ in range(200):
+        lens = rng.integers(T, 4 * T, size=rng.integers(1, 64)).tolist()
+        assert facts.paged_waste_fraction(lens, B) < facts.waste_bound(T, B)
+        for t in lens:
+            assert 0 <= facts.blocks_for_tokens(t, B) * B - t <= B - 1
+    # every request one token past a boundary: B - 1 idle slots each
+    assert facts.paged_waste_fraction([T + 1] * 7, B) == pytest.approx((B - 1) / (T + B))

@@ -41,15 +41,16 @@ def test_block_table_example_and_slots(golden):
     check_invariants(a)
 
 
-def test_theorem1_slack_on_growth():
-    a = RefAllocator(4096, 16)
+@pytest.mark.parametrize("B", [16, 8, 32])
+def test_theorem1_slack_on_growth(B):
+    a = RefAllocator(65536 // B, B)
     rng = np.random.default_rng(3)
     lens = rng.integers(1, 3000, 40)
     for s, n in enumerate(lens):
         a.add_seq(s, int(n) // 2)
         a.append(s, int(n) - int(n) // 2)
-        assert len(a.block_table(s)) == -(-int(n) // 16)
-        assert len(a.block_table(s)) * 16 - int(n) <= 15
+        assert len(a.block_table(s)) == -(-int(n) // B)
+        assert len(a.block_table(s)) * B - int(n) <= B - 1
     check_invariants(a)
 
 
