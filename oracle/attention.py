@@ -1,4 +1,4 @@
-"""Decode attention over the paged cache, float64 (test infrastructure only).
+"""Decode and prefill attention over the paged cache, float64 (test infrastructure only).
 
 [KVPaged] "Core principle: what is the KV cache": attention(Q, K, V) = softmax(Q K^T /
 sqrt(d_k)) V; at decode one new query attends to the cached keys and values of all earlier
@@ -100,3 +100,52 @@ def brute_force_attention(q_vec, keys, values, scale: float):
     d = len(values[0])
     return [sum(w[t] * float(values[t][j]) for t in range(len(keys))) / tot for j in range(d)], \
         math.log(tot)
+
+
+def ref_prefill(q: np.ndarray, query_start: np.ndarray, k_cache: np.ndarray,
+                v_cache: np.ndarray, block_tables: np.ndarray, context_lens: np.ndarray,
+                scale: float, num_kv_heads: int, q_dtype: str, kv_dtype: str,
+                k_scales: Optional[np.ndarray] = None, v_scales: Optional[np.ndarray] = None,
+                k_zeros: Optional[np.ndarray] = None, v_zeros: Optional[np.ndarray] = None,
+                seqs: Optional[Iterable[int]] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """Causal attention of a step's new tokens over the paged cache (prefill).
+
+    [KVPaged] "Core principle: what is the KV cache": the prompt's K and V are computed
+    once and cached, each token attending to itself and every earlier token; "Prefix
+    sharing and copy-on-write": a shared prefix's KV is computed once, so a step may bring
+    only the tokens after a cached prefix. Reading: sequence s brings
+    n_s = query_start[s+1] - query_start[s] new tokens (rows query_start[s].. of q
+    [T, Hq, d]) whose K/V were written into the cache first, as the last n_s of its
+    context_lens[s] positions. Row i of the sequence sits at position
+    p = context_lens[s] - n_s + i and attends to positions 0..p through the block table:
+    z_t = scale * q . K_t for t <= p, out = sum_t softmax(z)_t V_t, lse = log sum_t e^z_t.
+    Returns out [T, Hq, d] and lse [T, Hq] in float64; rows of sequences outside ``seqs``
+    are NaN.
+    """
+    T, Hq, d = q.shape
+    G = Hq // num_kv_heads
+    qv = decode_values(q, q_dtype)
+    out = np.full((T, Hq, d), np.nan)
+    lse = np.full((T, Hq), np.nan)
+    S = len(context_lens)
+    for s in (range(S) if seqs is None else seqs):
+        r0, r1 = int(query_start[s]), int(query_start[s + 1])
+        n, ctx = r1 - r0, int(context_lens[s])
+        if n == 0:
+            continue
+        assert 0 < n <= ctx
+        pos = ctx - n + np.arange(n)                       # position of each new token
+        allowed = np.arange(ctx)[None, :] <= pos[:, None]  # [n, ctx]
+        for kvh in range(num_kv_heads):
+            K, V = gather_kv(k_cache, v_cache, block_tables[s], ctx, kvh, kv_dtype,
+                             k_scales, v_scales, k_zeros, v_zeros)
+            for g in range(G):
+                h = kvh * G + g
+                z = scale * (qv[r0:r1, h] @ K.T)            # [n, ctx]
+                z = np.where(allowed, z, -np.inf)
+                m = z.max(axis=1, keepdims=True)
+                e = np.exp(z - m)
+                l = e.sum(axis=1, keepdims=True)
+                out[r0:r1, h] = (e @ V) / l
+                lse[r0:r1, h] = (m + np.log(l))[:, 0]
+    return out, lse

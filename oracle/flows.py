@@ -9,6 +9,9 @@ Flows (readings of the pages, stated once):
   sequence is added with ctx-1 tokens (in sequence order), then every sequence appends its
   decode token (ctx includes the token being decoded); all K/V is written through the
   slot mapping, then attention runs.
+* prefill workloads: every sequence is added with its cached tokens (ctx - n), in
+  sequence order, then every sequence appends its n new tokens; all K/V is written through
+  the slot mapping, then the new tokens attend causally.
 * shared-prefix workload ([KVPaged] "Prefix sharing and copy-on-write", [Ch4PA] "Prefix
   Caching"): sequence 0 is added with the prefix and the prefix K/V written once; it is
   forked to every other sequence; every sequence then appends its private suffix in
@@ -23,7 +26,7 @@ from typing import Dict, List, Optional, Sequence
 import numpy as np
 
 from .paged import RefAllocator, new_cache, ref_copy_blocks, ref_reshape_and_cache
-from .attention import ref_decode
+from .attention import ref_decode, ref_prefill
 
 
 @dataclasses.dataclass
@@ -140,3 +143,46 @@ def ref_outputs(draw, state: RefState, seqs: Optional[Sequence[int]] = None, sca
                       state.context_lens, sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype,
                       state.k_scales, state.v_scales, seqs=seqs, k_zeros=state.k_zeros,
                       v_zeros=state.v_zeros)
+
+
+def build_prefill_state(draw, write_seqs: Optional[Sequence[int]] = None) -> RefState:
+    """Allocate and write a prefill step: cached tokens first (add_seq), then the step's
+    new tokens (append); K/V written only for ``write_seqs`` (default all)."""
+    wl = draw.wl
+    S, B, H, d = wl.num_seqs, wl.block_size, wl.num_kv_heads, wl.head_dim
+    write = set(range(S) if write_seqs is None else write_seqs)
+    nb = wl.num_blocks
+    alloc = RefAllocator(nb, B, order=draw.pool_order)
+    kc = new_cache(nb, H, B, d, wl.kv_dtype)
+    vc = new_cache(nb, H, B, d, wl.kv_dtype)
+    ks = vs = kz = vz = None
+    pre, new = {}, {}
+    for s in range(S):
+        pre[s] = alloc.add_seq(s, int(draw.context_lens[s] - draw.query_lens[s]))
+    for s in range(S):
+        sl, pr = alloc.append(s, int(draw.query_lens[s]))
+        assert not pr
+        new[s] = sl
+    if wl.kv_dtype == "fp8":
+        ks, vs = _fp8_scales(draw, alloc, write, nb, H)
+    elif wl.kv_dtype == "int8":
+        ks, vs, kz, vz = _int8_params(draw, alloc, write, nb, H)
+    for s in sorted(write):
+        k, v = draw.kv(s)
+        c = int(draw.context_lens[s] - draw.query_lens[s])
+        ref_reshape_and_cache(k[:c], v[:c], kc, vc, pre[s], wl.in_dtype, wl.kv_dtype, ks, vs,
+                              kz, vz)
+        ref_reshape_and_cache(k[c:], v[c:], kc, vc, new[s], wl.in_dtype, wl.kv_dtype, ks, vs,
+                              kz, vz)
+    tables = alloc.padded_tables(range(S), max_blocks_per_seq(draw))
+    return RefState(alloc, kc, vc, ks, vs, tables, draw.context_lens.copy(), [], new, kz, vz)
+
+
+def ref_prefill_outputs(draw, state: RefState, seqs: Optional[Sequence[int]] = None,
+                        scale=None):
+    wl = draw.wl
+    sc = float(np.float32(1.0 / np.sqrt(wl.head_dim) if scale is None else scale))
+    return ref_prefill(draw.q, draw.query_start, state.k_cache, state.v_cache,
+                       state.block_tables, state.context_lens, sc, wl.num_kv_heads,
+                       wl.in_dtype, wl.kv_dtype, state.k_scales, state.v_scales,
+                       state.k_zeros, state.v_zeros, seqs=seqs)

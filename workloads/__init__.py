@@ -246,3 +246,110 @@ def _int8_params(x: np.ndarray):
 def draw(name_or_wl, **kw) -> Draw:
     wl = WORKLOADS[name_or_wl] if isinstance(name_or_wl, str) else name_or_wl
     return Draw(wl, **kw)
+
+
+# ---------------------------------------------------------------------------------------
+# prefill: a step that brings many new tokens per sequence
+# ---------------------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class PrefillWorkload:
+    """Shape and length recipe of one synthetic prefill step (one attention layer).
+
+    Sequence s holds context_lens[s] tokens after the step; the last query_lens[s] of them
+    are the step's new tokens (their K/V are written, then they attend causally), the
+    earlier ones were cached by earlier steps (a chunked prompt or a cached prefix).
+    """
+
+    name: str
+    seed: int
+    num_seqs: int
+    num_q_heads: int
+    num_kv_heads: int
+    head_dim: int
+    block_size: int
+    num_blocks: int
+    kv_dtype: str
+    in_dtype: str
+    lens: Tuple       # context lengths, same forms as Workload.lens
+    new: Tuple        # ("full",) every token new | ("chunk", n) the last min(n, ctx) tokens
+                      # | ("uniform", lo, hi) a uniform count, at most ctx
+    shared_prefix = None  # K/V of every sequence drawn independently
+
+    @property
+    def group(self) -> int:
+        return self.num_q_heads // self.num_kv_heads
+
+    def scaled(self, **kw) -> "PrefillWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+PREFILL_WORKLOADS: Dict[str, PrefillWorkload] = {
+    # 3 seqs: two whole prompts and a 7-token chunk after 33 cached tokens; fp32, d 64.
+    "prefill_tiny": PrefillWorkload("prefill_tiny", 10, 3, 4, 2, 64, 16, 32, "f32", "f32",
+                                    ("fixed", [5, 16, 40]), ("chunk", 16)),
+    # 8 prompts of 2048 tokens prefilled whole: 32q/8kv, d 128, bf16.
+    "prefill": PrefillWorkload("prefill", 11, 8, 32, 8, 128, 16, 8192, "bf16", "bf16",
+                               ("const", 2048), ("full",)),
+    # 16 sequences, 512-token chunks after cached contexts of U{512..3584}: 32q/8kv, bf16.
+    "chunked": PrefillWorkload("chunked", 12, 16, 32, 8, 128, 16, 8192, "bf16", "bf16",
+                               ("uniform", 1024, 4096), ("chunk", 512)),
+}
+
+
+class PrefillDraw(Draw):
+    """All random inputs of one prefill step: lengths, pool order, q of the new tokens
+    [T, Hq, d] (rows grouped by sequence), K/V of every context token of every sequence."""
+
+    def __init__(self, wl: PrefillWorkload, lens_override: Optional[List[int]] = None,
+                 new_override: Optional[List[int]] = None):
+        self.wl = wl
+        self.needle = False
+        ss = np.random.SeedSequence(wl.seed)
+        c_lens, c_pool, c_q, c_kv, c_new = ss.spawn(5)
+        self._kv_seq = c_kv.spawn(wl.num_seqs + 1)
+        S = wl.num_seqs
+        rng = np.random.Generator(np.random.PCG64(c_lens))
+        kind = wl.lens[0]
+        if lens_override is not None:
+            lens = np.asarray(lens_override, dtype=np.int64)
+        elif kind == "fixed":
+            lens = np.asarray(wl.lens[1], dtype=np.int64)
+        elif kind == "const":
+            lens = np.full(S, wl.lens[1], dtype=np.int64)
+        elif kind == "uniform":
+            lens = rng.integers(wl.lens[1], wl.lens[2] + 1, size=S)
+        else:
+            raise ValueError(kind)
+        self.context_lens = lens.astype(np.int32)
+        assert self.context_lens.shape == (S,)
+        nrng = np.random.Generator(np.random.PCG64(c_new))
+        if new_override is not None:
+            qn = np.asarray(new_override, dtype=np.int64)
+        elif wl.new[0] == "full":
+            qn = lens.copy()
+        elif wl.new[0] == "chunk":
+            qn = np.minimum(lens, wl.new[1])
+        elif wl.new[0] == "uniform":
+            qn = np.minimum(lens, nrng.integers(wl.new[1], wl.new[2] + 1, size=S))
+        else:
+            raise ValueError(wl.new[0])
+        assert np.all((qn >= 0) & (qn <= lens))
+        self.query_lens = qn.astype(np.int32)
+        self.query_start = np.concatenate([[0], np.cumsum(qn)]).astype(np.int32)
+        prng = np.random.Generator(np.random.PCG64(c_pool))
+        self.pool_order = prng.permutation(wl.num_blocks).astype(np.int32)
+        qrng = np.random.Generator(np.random.PCG64(c_q))
+        T = int(self.query_start[-1])
+        self.q = self._typed(qrng.standard_normal((T, wl.num_q_heads, wl.head_dim),
+                                                  dtype=np.float32))
+        self._qf = None
+        self._cache = {}
+
+    @property
+    def num_tokens(self) -> int:
+        return int(self.query_start[-1])
+
+
+def draw_prefill(name_or_wl, **kw) -> PrefillDraw:
+    wl = PREFILL_WORKLOADS[name_or_wl] if isinstance(name_or_wl, str) else name_or_wl
+    return PrefillDraw(wl, **kw)
