@@ -79,6 +79,8 @@ typedef enum {
 #define PA_DEVERR_PAIR 0x4       /* copy_blocks pair outside [0, num_blocks)            */
 #define PA_DEVERR_CONTEXT 0x8    /* context_lens entry < 0 or > max_context_len         */
 #define PA_DEVERR_TIMEOUT 0x10   /* a bounded wait on an asynchronous copy gave up      */
+#define PA_DEVERR_QUERY 0x20     /* prefill query_start not ascending, past num_tokens, */
+                                 /* or more new tokens than context (or max_query_len)  */
 
 /* Shape and dtypes of one paged decode-attention call. */
 typedef struct {
@@ -132,6 +134,40 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
                             int max_context_len, const float* k_scales, const float* v_scales,
                             const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
                             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Prefill attention over the paged cache: the new tokens of a step attend causally to
+ * their sequence's cached tokens ([KVPaged] "Core principle: what is the KV cache": the
+ * prompt's K/V is computed once and cached, each token attending to itself and all earlier
+ * tokens; "Prefix sharing and copy-on-write": a cached prefix's K/V is computed once, so
+ * a step may bring only the tokens after it, as may a prompt cut into chunks). Sequence s
+ * brings n_s = query_start[s+1] - query_start[s] new tokens, rows query_start[s] .. of q,
+ * whose K/V were written by reshape_and_cache first as the last n_s of its
+ * context_lens[s] positions. Row i of sequence s sits at position p = context_lens[s] -
+ * n_s + i; for query head h (kv head g = h / (Hq/Hkv)):
+ *     z_t = scale * q[row][h] . K_t (t <= p),  out[row][h] = sum_t softmax(z)_t V_t,
+ *     lse_out[row][h] = log sum_t exp(z_t)              (natural log, float32)
+ * with fp8 / int8 dequantisation as in paged_attn_decode. Accumulation is float32.
+ *   q, out        [num_tokens][Hq][d] in desc->q_dtype / desc->out_dtype
+ *   query_start   int32 [num_seqs + 1], ascending, query_start[0] = 0,
+ *                 query_start[num_seqs] = num_tokens
+ *   max_query_len host int >= every n_s (sizes the grid); max_context_len >= every
+ *                 context_lens entry and >= max_query_len
+ *   block_tables, context_lens, k/v scales and zeros, lse_out: as in paged_attn_decode
+ *   desc          as in paged_attn_decode with partition_size 0
+ * bf16 caches with head_dim 128 and a group of 1, 2, 4, 8 or 16 run on the tensor cores
+ * (tcgen05, accumulators in tensor memory); every other supported shape, or
+ * pa_set_decode_impl(1), runs one CUDA-core pass per new token. No workspace.
+ * A sequence whose query range is inconsistent (descending, past num_tokens, more new
+ * tokens than context or than max_query_len) is skipped and PA_DEVERR_QUERY recorded.
+ */
+pa_status paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             const int32_t* query_start, int num_tokens, int max_query_len,
+                             float scale, void* out, const pa_decode_desc* desc,
+                             int max_context_len, const float* k_scales, const float* v_scales,
+                             const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
+                             void* stream);
 
 /*
  * Largest workspace (bytes) that paged_attn_decode_noalloc can serve from its fixed device

@@ -33,6 +33,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR
     PA_ERR_DEVICE = 0, -1, -2, -3, -4, -5, -6
 PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_CONTEXT, PA_DEVERR_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
+PA_DEVERR_QUERY = 0x20
 _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_CUDA",
            -4: "PA_ERR_NO_BLOCKS", -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_DEVICE"}
 
@@ -65,6 +66,8 @@ _SIGS = {
                                _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "paged_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i,
                                        _vp, _vp, _vp, _vp, _vp, _vp]),
+    "paged_attn_prefill": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _f, _vp,
+                                _P(pa_decode_desc), _i, _vp, _vp, _vp, _vp, _vp, _vp]),
     "reshape_and_cache": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i64, _i64, _i, _i, _i, _i, _i, _i,
                                _vp, _vp, _vp, _vp, _vp]),
     "copy_blocks": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp]),
@@ -218,6 +221,50 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: fl
     return out
 
 
+def paged_attn_prefill(q, k_cache, v_cache, block_tables, context_lens, query_start,
+                       scale: float, out, *, max_query_len: int, max_context_len: int,
+                       k_scales=None, v_scales=None, k_zeros=None, v_zeros=None, lse_out=None,
+                       stream=None):
+    """Causal attention of a step's new tokens over the paged cache.
+
+    q, out [T, Hq, d]: the new tokens of every sequence, sequence s owning rows
+    query_start[s] .. query_start[s+1]-1 (query_start int32 [S+1]); their K/V must already
+    be in the cache as the last tokens of context_lens[s]. Row i of sequence s attends to
+    positions 0 .. context_lens[s] - n_s + i. Other arguments as in paged_attn_decode.
+    """
+    torch = _torch()
+    T, Hq, d = q.shape
+    NB, Hkv, B, d2 = k_cache.shape
+    if d2 != d:
+        raise ValueError("head_dim of q and cache differ")
+    S = block_tables.shape[0]
+    if tuple(context_lens.shape) != (S,) or tuple(query_start.shape) != (S + 1,):
+        raise ValueError("context_lens must be [S] and query_start [S + 1]")
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache differ")
+    if tuple(out.shape) != tuple(q.shape) or out.dtype != q.dtype:
+        raise ValueError("out must match q")
+    if lse_out is not None and tuple(lse_out.shape) != (T, Hq):
+        raise ValueError("lse_out must be [T, Hq]")
+    for sc in (k_scales, v_scales, k_zeros, v_zeros):
+        if sc is not None and tuple(sc.shape) != tuple(k_cache.shape[:2]):
+            raise ValueError("scales / zero points must be [num_blocks, num_kv_heads]")
+    qd = _dtype_code(q.dtype)
+    desc = make_desc(S, Hq, Hkv, d, block_tables.shape[1], NB, 0, qd, _dtype_code(k_cache.dtype),
+                     qd, block_size=B)
+    st = _lib.paged_attn_prefill(
+        _dev(q, "q"), _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache"),
+        _dev(block_tables, "block_tables", torch.int32),
+        _dev(context_lens, "context_lens", torch.int32),
+        _dev(query_start, "query_start", torch.int32), int(T), int(max_query_len),
+        ctypes.c_float(scale), _dev(out, "out"), ctypes.byref(desc), int(max_context_len),
+        _dev(k_scales, "k_scales", torch.float32), _dev(v_scales, "v_scales", torch.float32),
+        _dev(k_zeros, "k_zeros", torch.int32), _dev(v_zeros, "v_zeros", torch.int32),
+        _dev(lse_out, "lse_out", torch.float32), _stream(stream))
+    _check(st, "paged_attn_prefill")
+    return out
+
+
 NOALLOC_SCRATCH_BYTES = 32 << 20
 
 
@@ -323,7 +370,7 @@ class BlockAllocator:
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h:
+        if h and _lib is not None:  # module globals may already be gone at interpreter exit
             _lib.pa_alloc_destroy(h)
             self._h = None
 

@@ -53,7 +53,7 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     cmds = [
         [nvcc, *ARCH, "-lineinfo", *common, "-Xptxas", "-v" if verbose else "-O3",
          "-c", os.path.join(CSRC, "pagedattn.cu"), "-o", cu_obj] + list(extra or []),
-        [nvcc, *common, "-x", "c++", "-c", os.path.join(CSRC, "allocator.cpp"), "-o", cpp_obj],
+        [nvcc, *common, "-Wno-deprecated-gpu-targets", "-x", "c++", "-c", os.path.join(CSRC, "allocator.cpp"), "-o", cpp_obj],
         [nvcc, *ARCH, "-shared", "-cudart", "static", cu_obj, cpp_obj, "-o", LIB + ".tmp"],
     ]
     for c in cmds:

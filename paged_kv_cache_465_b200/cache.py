@@ -10,8 +10,8 @@ from typing import Iterable, List, Optional, Sequence, Tuple
 
 import numpy as np
 
-from . import (BlockAllocator, copy_blocks, paged_attn_decode, reshape_and_cache,
-               workspace_size, decode_desc_for)
+from . import (BlockAllocator, copy_blocks, paged_attn_decode, paged_attn_prefill,
+               reshape_and_cache, workspace_size, decode_desc_for)
 
 _TORCH_DTYPE = {"f32": "float32", "bf16": "bfloat16", "fp8": "uint8", "int8": "int8"}
 
@@ -79,3 +79,11 @@ class PagedKVCache:
                                  v_scales=self.v_scales, k_zeros=self.k_zeros,
                                  v_zeros=self.v_zeros, lse_out=lse_out, workspace=workspace,
                                  stream=stream)
+
+    def prefill(self, q, block_tables, context_lens, query_start, scale: float, out, *,
+                max_query_len: int, max_context_len: int, lse_out=None, stream=None):
+        return paged_attn_prefill(q, self.k_cache, self.v_cache, block_tables, context_lens,
+                                  query_start, scale, out, max_query_len=max_query_len,
+                                  max_context_len=max_context_len, k_scales=self.k_scales,
+                                  v_scales=self.v_scales, k_zeros=self.k_zeros,
+                                  v_zeros=self.v_zeros, lse_out=lse_out, stream=stream)

@@ -124,6 +124,10 @@ struct DecodeArgs {
   int final_pass;    // 1: one item covers the whole context, write out directly
   int skip_single;   // split path: single-partition sequences were written directly
   pa_dtype q_dtype, out_dtype;
+  // prefill rows (CUDA-core kernel only): work row s is new token s; the tokens of
+  // sequence q are rows query_start[q] .. query_start[q+1]-1, the last ones of its context
+  const int32_t* query_start;  // [num_seqs + 1], or null for decode rows
+  int num_tokens;
 };
 
 __device__ __forceinline__ float load_q(const void* q, pa_dtype t, int64_t i) {
@@ -144,6 +148,28 @@ __device__ __forceinline__ int checked_ctx(const DecodeArgs& a, int s) {
     c = c < 0 ? 0 : a.max_context_len;
   }
   return c;
+}
+
+// Work row s of a prefill call: its sequence (block-table row) and the number of keys it
+// sees (its position + 1). A row whose sequence has an inconsistent query range (not
+// ascending, past num_tokens, more new tokens than context) sees no key and is flagged.
+struct RowView {
+  int ctx, seq;
+};
+__device__ __forceinline__ RowView prefill_row(const DecodeArgs& a, int t) {
+  int lo = 0, hi = a.num_seqs;  // largest q with query_start[q] <= t
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (a.query_start[mid] <= t) lo = mid;
+    else hi = mid;
+  }
+  const int q0 = a.query_start[lo], q1 = a.query_start[lo + 1];
+  const int c = a.context_lens[lo];
+  if (q0 < 0 || q0 > t || t >= q1 || q1 > a.num_tokens || c < q1 - q0 || c > a.max_context_len) {
+    if (threadIdx.x == 0) flag_error(PA_DEVERR_QUERY);
+    return RowView{0, lo};
+  }
+  return RowView{c - (q1 - t) + 1, lo};
 }
 
 // Writes the merged state of a work item: either out/lse (final) or the partial.
@@ -178,8 +204,11 @@ decode_simt_kernel(const DecodeArgs a) {
   __shared__ float sm[kSimtWarps][GP], sl[kSimtWarps][GP];
   __shared__ __align__(16) float sacc[kSimtWarps][GP][D];
 
-  const int part = blockIdx.x, kvh = blockIdx.y, s = blockIdx.z;
-  const int ctx = checked_ctx(a, s);
+  // decode: grid (partitions, Hkv, S); prefill: grid (new tokens, Hkv, 1), one pass
+  const bool pre = a.query_start != nullptr;
+  const int part = pre ? 0 : blockIdx.x, kvh = blockIdx.y, s = pre ? blockIdx.x : blockIdx.z;
+  const RowView rv = pre ? prefill_row(a, s) : RowView{checked_ctx(a, s), s};
+  const int ctx = rv.ctx;
   const int t0 = part * a.part_tokens;
   if (!a.final_pass && t0 >= ctx) return;  // empty partition: nothing to write
   const int t1 = min(ctx, t0 + a.part_tokens);
@@ -210,7 +239,7 @@ decode_simt_kernel(const DecodeArgs a) {
   const int tok = lane & 15, half = lane >> 4;
   const int BS = a.block_size;
   const int c_begin = t0 / kSub, c_end = (t1 + kSub - 1) / kSub;
-  const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+  const int32_t* bt = a.block_tables + (int64_t)rv.seq * a.max_blocks_per_seq;
   const uint8_t* kbase = static_cast<const uint8_t*>(a.k_cache);
   const uint8_t* vbase = static_cast<const uint8_t*>(a.v_cache);
 

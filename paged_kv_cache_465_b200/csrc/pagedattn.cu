@@ -9,6 +9,7 @@
 #include "cache_ops.cuh"
 #include "decode_simt.cuh"
 #include "decode_tc.cuh"
+#include "prefill_tc.cuh"
 
 namespace pa {
 namespace {
@@ -207,6 +208,73 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   if (e != cudaSuccess) return PA_ERR_CUDA;
   if (split && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
+}
+
+pa_status paged_attn_prefill(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* context_lens,
+                             const int32_t* query_start, int num_tokens, int max_query_len,
+                             float scale, void* out, const pa_decode_desc* desc,
+                             int max_context_len, const float* k_scales, const float* v_scales,
+                             const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
+                             void* stream) {
+  if (!desc_ok(desc) || desc->partition_size != 0 || num_tokens < 0 || max_query_len < 0 ||
+      max_context_len < max_query_len || !std::isfinite(scale))
+    return PA_ERR_INVALID;
+  if (!desc_supported(desc)) return PA_ERR_UNSUPPORTED;
+  if (desc->num_seqs == 0 || num_tokens == 0) return PA_OK;
+  if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !query_start || !out)
+    return PA_ERR_INVALID;
+  if (!aligned16(k_cache) || !aligned16(v_cache) || !aligned16(q) || !aligned16(out))
+    return PA_ERR_INVALID;
+  if ((int64_t)desc->max_blocks_per_seq * desc->block_size < (int64_t)max_context_len)
+    return PA_ERR_INVALID;
+  const bool quant = desc->kv_dtype == PA_FP8_E4M3 || desc->kv_dtype == PA_INT8;
+  if (quant && (!k_scales || !v_scales)) return PA_ERR_INVALID;
+  if (desc->kv_dtype == PA_INT8 && (!k_zeros || !v_zeros)) return PA_ERR_INVALID;
+  const cudaStream_t st = as_stream(stream);
+  if (max_query_len == 0) return PA_OK;
+  cudaError_t e;
+  if (g_decode_impl != 1 && prefill_tc_supported(desc)) {
+    pf::PrefillArgs a;
+    a.block_tables = block_tables; a.context_lens = context_lens; a.query_start = query_start;
+    a.out = out; a.lse_out = lse_out;
+    a.scale_log2 = scale * kLog2e;
+    a.num_seqs = desc->num_seqs; a.num_tokens = num_tokens;
+    a.num_q_heads = desc->num_q_heads; a.num_kv_heads = desc->num_kv_heads;
+    a.group = desc->num_q_heads / desc->num_kv_heads;
+    a.max_blocks_per_seq = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
+    a.max_context_len = max_context_len; a.max_query_len = max_query_len;
+    e = launch_prefill_tc(a, desc->block_size, q, k_cache, v_cache, st);
+  } else {
+    // CUDA-core path: every new token is one work row of the single-pass decode kernel
+    DecodeArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q; a.k_cache = k_cache; a.v_cache = v_cache;
+    a.block_tables = block_tables; a.context_lens = context_lens;
+    a.out = out; a.lse_out = lse_out; a.k_scales = k_scales; a.v_scales = v_scales;
+    a.k_zeros = k_zeros; a.v_zeros = v_zeros;
+    a.scale_log2 = scale * kLog2e;
+    a.num_seqs = desc->num_seqs; a.num_q_heads = desc->num_q_heads;
+    a.num_kv_heads = desc->num_kv_heads; a.group = desc->num_q_heads / desc->num_kv_heads;
+    a.max_blocks_per_seq = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
+    a.block_size = desc->block_size;
+    a.max_context_len = max_context_len;
+    a.q_dtype = desc->q_dtype; a.out_dtype = desc->out_dtype;
+    a.part_tokens = (int)round_up((size_t)(max_context_len > 0 ? max_context_len : 1), kSub);
+    a.max_parts = 1;
+    a.final_pass = 1;
+    a.query_start = query_start;
+    a.num_tokens = num_tokens;
+    const dim3 grid(num_tokens, desc->num_kv_heads, 1);
+    const int gp = pad_group(a.group);
+    switch (desc->kv_dtype) {
+      case PA_F32: e = launch_simt_d<PA_F32>(a, desc->head_dim, gp, grid, st); break;
+      case PA_BF16: e = launch_simt_d<PA_BF16>(a, desc->head_dim, gp, grid, st); break;
+      case PA_INT8: e = launch_simt_d<PA_INT8>(a, desc->head_dim, gp, grid, st); break;
+      default: e = launch_simt_d<PA_FP8_E4M3>(a, desc->head_dim, gp, grid, st); break;
+    }
+  }
+  return e == cudaSuccess ? PA_OK : PA_ERR_CUDA;
 }
 
 pa_status reshape_and_cache(const void* k, const void* v, void* k_cache, void* v_cache,

@@ -1,0 +1,577 @@
+// Prefill attention on the fifth-generation tensor cores: the new tokens of a step attend
+// causally to their sequence's cached keys through the block table.
+//
+// [KVPaged] "Core principle: what is the KV cache" (each token attends to itself and every
+// earlier token; the prompt's K/V is computed once and cached) and "Prefix sharing and
+// copy-on-write" (a cached prefix's K/V is computed once, so a step may bring only the
+// tokens after it); [Ch4PA] "PagedAttention algorithm" (keys and values are gathered from
+// non-contiguous blocks through the block table).
+//
+// One CTA per (128-row query tile, kv head, sequence). A tile row is a (new token, query
+// head of the kv head's group) pair, so one key/value tile serves the whole group. Keys are
+// taken 128 at a time:
+//   warp 5 (one lane)   TMA: Q once; K and V of key tile j into stage j % 2, one box per
+//                       (block, 64-channel half) straight from the paged pool;
+//   warp 4 (one lane)   tcgen05.mma: S_j = Q K_j^T into tensor memory (two S buffers, so
+//                       S_{j+1} runs while S_j is in softmax), then O += P_j V_j;
+//   warps 0-3           softmax, one thread per tile row (= tensor-memory lane): causal
+//                       mask, running max (rescaling O in tensor memory only when the max
+//                       grows by more than 2^8), P_j as bf16 into shared memory; finally
+//                       O / l to `out` and the log-sum-exp to `lse_out`.
+// Operands sit in shared memory in the 128-byte-swizzled layouts the tensor core reads:
+// Q, K and P K-major (rows of 64 channels / keys, 128 B), V MN-major (rows of keys).
+// Every wait is bounded; a CTA that gives up flags PA_DEVERR_TIMEOUT, lets its issued
+// copies and products finish, and releases its tensor memory.
+#pragma once
+
+#include "decode_tc.cuh"
+
+namespace pa {
+namespace pf {
+
+using tc::evict_first_policy;
+using tc::mbar_arrive;
+using tc::mbar_arrive_tx;
+using tc::mbar_init;
+using tc::mbar_wait;
+using tc::smem_u32;
+
+constexpr int kBM = 128;                  // tile rows: (new token, head) pairs
+constexpr int kBN = 128;                  // keys per key tile
+constexpr int kD = 128;                   // head dimension
+constexpr int kThreads = 192;             // warps 0-3 softmax, 4 MMA, 5 TMA
+constexpr int kMmaWarp = 4, kTmaWarp = 5;
+constexpr int kSlab = 128 * 128;          // 64 channels (128 B) x 128 rows
+constexpr int kTile = 2 * kSlab;          // 128 rows x 128 bf16
+constexpr int kOffQ = 0;
+constexpr int kOffK = kOffQ + kTile;      // 2 stages
+constexpr int kOffV = kOffK + 2 * kTile;  // 2 stages
+constexpr int kOffP = kOffV + 2 * kTile;
+constexpr int kOffBar = kOffP + kTile;
+constexpr int kSmem = kOffBar + 256 + 1024;  // + barriers, + alignment slack
+constexpr uint32_t kTmemCols = 512;       // S buffers at columns 0 / 128, O at 256
+constexpr uint32_t kOCol = 256;
+
+// barrier indices
+enum { kBarQ = 0, kBarKF = 1, kBarVF = 3, kBarKVE = 5, kBarSF = 7, kBarP = 9, kBarO = 10,
+       kBarFin = 11, kNumBars = 12 };
+
+// Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
+// S = Q K^T: A and B K-major, N = 128 keys. O += P V: B (V) MN-major, N = 128 channels.
+constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                             ((uint32_t)(kBM >> 4) << 24);
+constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                              ((uint32_t)(kD >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+// Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride
+// byte offsets (16-byte units), descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+  return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w),
+        "r"(bar), "l"(policy)
+      : "memory");
+}
+
+// ---- tensor memory and tcgen05 ----
+__device__ __forceinline__ void tmem_alloc(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+               ::"r"(dst_smem), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+               ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Arrives on `bar` once every tcgen05 operation this thread issued so far has completed.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+               ::"r"(bar) : "memory");
+}
+// D (tensor memory) = A B (+ D when acc != 0), A and B from shared-memory descriptors.
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {"
+               "%0, %1, %2, %3, %4, %5, %6, %7,"
+               "%8, %9, %10, %11, %12, %13, %14, %15,"
+               "%16, %17, %18, %19, %20, %21, %22, %23,"
+               "%24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]),
+                 "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                 "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
+                 "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+                 "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+                 "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                 "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                 "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {"
+               "%1, %2, %3, %4, %5, %6, %7, %8,"
+               "%9, %10, %11, %12, %13, %14, %15, %16,"
+               "%17, %18, %19, %20, %21, %22, %23, %24,"
+               "%25, %26, %27, %28, %29, %30, %31, %32};"
+               :: "r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+                 "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                 "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+                 "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+                 "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+                 "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+                 "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+                 "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+// tcgen05.wait::ld that also "rewrites" the loaded registers, so no use of them can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]),
+                 "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                 "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]),
+                 "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+                 "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                 "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+               :: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+struct PrefillArgs {
+  const int32_t* block_tables;  // [S][max_blocks_per_seq]
+  const int32_t* context_lens;  // [S]
+  const int32_t* query_start;   // [S + 1]
+  void* out;                    // [T][Hq][128] bf16
+  float* lse_out;               // [T][Hq] or null
+  float scale_log2;             // scale * log2(e)
+  int num_seqs, num_tokens, num_q_heads, num_kv_heads, group;
+  int max_blocks_per_seq, num_blocks, max_context_len, max_query_len;
+};
+
+// The new tokens of sequence s: rows [q0, q0 + n) of q, positions ctx - n .. ctx - 1.
+// False (and flagged by thread 0) when the ranges are inconsistent.
+__device__ __forceinline__ bool seq_rows(const PrefillArgs& a, int s, int& q0, int& n,
+                                         int& ctx) {
+  q0 = a.query_start[s];
+  const int q1 = a.query_start[s + 1];
+  n = q1 - q0;
+  ctx = a.context_lens[s];
+  const bool ok = q0 >= 0 && n >= 0 && q1 <= a.num_tokens && n <= ctx &&
+                  ctx <= a.max_context_len && n <= a.max_query_len;
+  if (!ok && threadIdx.x == 0) flag_error(PA_DEVERR_QUERY);
+  return ok;
+}
+
+template <int BS>
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
+                  const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap) {
+  static_assert(kBN % BS == 0 && kBN / BS <= 32, "block size");
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = a.group, TM = kBM / G;  // new tokens per tile
+  const int s = blockIdx.z, kvh = blockIdx.y;
+  const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // longest tiles (most keys) first
+
+  int q0, n, ctx;
+  if (!seq_rows(a, s, q0, n, ctx) || qt * TM >= n) return;  // before any set-up
+  const int pos0 = ctx - n;                     // position of the sequence's first new token
+  const int tok0 = qt * TM;                     // first new token of the tile
+  const int ntok = min(TM, n - tok0);           // new tokens in the tile
+  const int pos_min = pos0 + tok0;              // smallest position of a tile row
+  const int kv_end = pos_min + ntok;            // keys 0 .. kv_end-1 are seen by some row
+  const int ntiles = (kv_end + kBN - 1) / kBN;
+
+  const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK);
+  const uint32_t sV = smem_u32(smem + kOffV), sP = smem_u32(smem + kOffP);
+  const uint32_t bar0 = smem_u32(smem + kOffBar);
+  auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + 8 * kNumBars);
+  volatile int* dead = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(kBarQ), 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(kBarKF + i), 1);
+      mbar_init(bar(kBarVF + i), 1);
+      mbar_init(bar(kBarKVE + i), 1);
+      mbar_init(bar(kBarSF + i), 1);
+    }
+    mbar_init(bar(kBarP), kBM);
+    mbar_init(bar(kBarO), 1);
+    mbar_init(bar(kBarFin), 1);
+    *dead = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0) {
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == kTmaWarp) {
+    // ---------------- producer: Q once, then K / V tiles through two stages ----------------
+    if (lane == 0) {
+      mbar_arrive_tx(bar(kBarQ), kTile);
+      const uint64_t pol = evict_first_policy();
+      for (int h = 0; h < 2; ++h)
+        tma_load_4d(sQ + h * kSlab, &qmap, 0, h, kvh * G, q0 + tok0, bar(kBarQ), pol);
+      int last[2] = {-1, -1};
+      for (int j = 0; j < ntiles && !*dead; ++j) {
+        const int st = j & 1;
+        if (j >= 2 && !mbar_wait(bar(kBarKVE + st), ((j >> 1) - 1) & 1)) {
+          flag_error(PA_DEVERR_TIMEOUT);
+          *dead = 1;
+          break;
+        }
+        const int t0 = j * kBN;
+        const int nblk = (min(kBN, kv_end - t0) + BS - 1) / BS;
+        int nvalid = 0;
+        for (int b = 0; b < nblk; ++b) {
+          const int p = bt[t0 / BS + b];
+          if (p >= 0 && p < a.num_blocks) ++nvalid;
+          else flag_error(PA_DEVERR_BLOCK_ID);
+        }
+        const uint32_t bytes = (uint32_t)nvalid * 2u * BS * 128u;
+        for (int kv = 0; kv < 2; ++kv) {
+          const uint32_t fb = bar((kv ? kBarVF : kBarKF) + st);
+          const uint32_t dst = (kv ? sV : sK) + st * kTile;
+          const CUtensorMap* map = kv ? &vmap : &kmap;
+          mbar_arrive_tx(fb, bytes);
+          for (int b = 0; b < nblk; ++b) {
+            const int p = bt[t0 / BS + b];
+            if (p < 0 || p >= a.num_blocks) continue;
+            const int row = (p * a.num_kv_heads + kvh) * BS;
+            for (int h = 0; h < 2; ++h) tma_load_3d(dst + h * kSlab + b * BS * 128, map, 0, h, row, fb);
+          }
+        }
+        last[st] = j;
+      }
+      if (*dead) {
+        // copies still in flight complete before the CTA's shared memory is released
+        for (int st = 0; st < 2; ++st)
+          if (last[st] >= 0) {
+            mbar_wait(bar(kBarKF + st), (last[st] >> 1) & 1);
+            mbar_wait(bar(kBarVF + st), (last[st] >> 1) & 1);
+          }
+        mbar_wait(bar(kBarQ), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      auto issue_s = [&](int j) {
+        const uint32_t kst = sK + (j & 1) * kTile;
+        const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
+          umma_bf16(d, sdesc(sQ + off, 16, 1024), sdesc(kst + off, 16, 1024), kIdescS, kk > 0);
+        }
+        umma_commit(bar(kBarSF + (j & 1)));
+      };
+      auto issue_pv = [&](int j) {
+        const uint32_t vst = sV + (j & 1) * kTile;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * kSlab + (kk & 3) * 32;
+          umma_bf16(tmem + kOCol, sdesc(sP + aoff, 16, 1024),
+                    sdesc(vst + kk * 16 * 128, kSlab, 1024), kIdescPV, (j > 0 || kk > 0));
+        }
+        umma_commit(bar(kBarO));
+        umma_commit(bar(kBarKVE + (j & 1)));
+      };
+      bool live = mbar_wait(bar(kBarQ), 0) && mbar_wait(bar(kBarKF), 0);
+      if (live) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int j = 0; live && j < ntiles; ++j) {
+        if (j + 1 < ntiles) {
+          if (!mbar_wait(bar(kBarKF + ((j + 1) & 1)), ((j + 1) >> 1) & 1)) { live = false; break; }
+          issue_s(j + 1);
+        }
+        if (!mbar_wait(bar(kBarP), j & 1) || !mbar_wait(bar(kBarVF + (j & 1)), (j >> 1) & 1)) {
+          live = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(j);
+        if (*dead) live = false;
+      }
+      if (!live) {
+        flag_error(PA_DEVERR_TIMEOUT);
+        *dead = 1;
+      }
+      // every product of the CTA completes before tensor memory is released
+      umma_commit(bar(kBarFin));
+      mbar_wait(bar(kBarFin), 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- softmax: thread r owns tile row r (tensor-memory lane r) ----------------
+    const int r = threadIdx.x;
+    const int tr = r / G, g = r - tr * G;
+    const bool row_valid = tr < ntok;
+    const int prow = pos_min + min(tr, ntok - 1);       // this row's position
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    // waits are made warp-uniform: the tcgen05.ld / st below are warp-collective
+    auto wait_all = [&](uint32_t b, uint32_t parity) {
+      const bool w = !*dead && mbar_wait(b, parity);
+      return __all_sync(0xffffffffu, w);
+    };
+    for (int j = 0; j < ntiles; ++j) {
+      if (!wait_all(bar(kBarSF + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
+      tc_fence_after();
+      const int t0 = j * kBN;
+      const int vlim = min(kBN, kv_end - t0);             // keys of the tile that exist
+      // blocks of the tile with an out-of-range id: skipped by the producer, masked here
+      uint32_t badm = 0;
+      {
+        const int nblk = (vlim + BS - 1) / BS;
+        bool bad = false;
+        if (lane < nblk) {
+          const int p = bt[t0 / BS + lane];
+          bad = p < 0 || p >= a.num_blocks;
+        }
+        badm = __ballot_sync(0xffffffffu, bad);
+      }
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + (uint32_t)((j & 1) * kBN + c * 32), sv[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
+      const bool need_mask = t0 + kBN - 1 > pos_min || badm != 0;  // uniform in the CTA
+      const int lim = prow - t0;                                  // visible: key <= lim
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int col = c * 32 + e;
+          float x = __uint_as_float(sv[c][e]) * a.scale_log2;
+          if (need_mask && (col > lim || ((badm >> (col / BS)) & 1u))) x = -INFINITY;
+          sv[c][e] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      const float m_new = fmaxf(m_used, mx);
+      float alpha = 1.f;
+      if (m_new > m_used + 8.f) {  // lazy rescale: P stays below 2^8 otherwise
+        alpha = fast_exp2(m_used - m_new);
+        m_used = m_new;
+      }
+      const float mref = m_used == -INFINITY ? 0.f : m_used;
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const float p0 = fast_exp2(__uint_as_float(sv[c][e]) - mref);
+          const float p1 = fast_exp2(__uint_as_float(sv[c][e + 1]) - mref);
+          rs += p0 + p1;
+          pk[(c * 32 + e) >> 1] = pack_bf16x2(p0, p1);
+        }
+      l = l * alpha + rs;
+      if (j > 0) {
+        // P_{j-1} and O are free once the previous product has completed
+        if (!wait_all(bar(kBarO), (j - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + kOCol + c * 32, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(lane_addr + kOCol + c * 32, o);
+          }
+          tmem_wait_st();
+        }
+      }
+      // P_j, K-major with the 128-byte swizzle: keys 64h.. in slab h, row r
+#pragma unroll
+      for (int k = 0; k < 16; ++k) {
+        const uint32_t addr = sP + (k >> 3) * kSlab + r * 128 + (((k & 7) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                     ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]), "r"(pk[4 * k + 2]),
+                       "r"(pk[4 * k + 3]) : "memory");
+      }
+      // rows of V past the keys that exist or in a skipped block may hold anything (NaN):
+      // zero them before the product reads them
+      if (vlim < kBN || badm != 0) {
+        if (!wait_all(bar(kBarVF + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
+        if (r >= vlim || ((badm >> (r / BS)) & 1u)) {
+          const uint32_t vrow = sV + (j & 1) * kTile + r * 128;
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};"
+                           ::"r"(vrow + h * kSlab + k * 16), "r"(0) : "memory");
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      tc_fence_before();
+      mbar_arrive(bar(kBarP));
+    }
+    if (ok) ok = wait_all(bar(kBarO), (ntiles - 1) & 1);
+    if (ok) {
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t orow = (int64_t)(q0 + tok0 + tr) * a.num_q_heads + kvh * G + g;
+      uint16_t* op = static_cast<uint16_t*>(a.out) + orow * kD;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        uint32_t o[32];
+        tmem_ld32(lane_addr + kOCol + c * 32, o);
+        tmem_wait_ld(o);
+        if (row_valid) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            uint4 w;
+            w.x = pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv, __uint_as_float(o[8 * k + 1]) * inv);
+            w.y = pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv, __uint_as_float(o[8 * k + 3]) * inv);
+            w.z = pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv, __uint_as_float(o[8 * k + 5]) * inv);
+            w.w = pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv, __uint_as_float(o[8 * k + 7]) * inv);
+            *reinterpret_cast<uint4*>(op + c * 32 + 8 * k) = w;
+          }
+        }
+      }
+      if (row_valid && a.lse_out != nullptr)
+        a.lse_out[orow] = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
+    } else {
+      if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
+      *dead = 1;
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------------------
+// q [T][Hq][128] bf16 as (64 channels, half, head, token); a box is the tile's rows of one
+// half: G heads x (128 / G) tokens, rows (token, head) of 128 B.
+inline bool make_q_map(CUtensorMap* m, const void* q, int num_tokens, int hq, int group) {
+  auto enc = tc::encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[4] = {64, 2, (cuuint64_t)hq, (cuuint64_t)num_tokens};
+  cuuint64_t strides[3] = {128, 256, (cuuint64_t)hq * 256};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)group, (cuuint32_t)(kBM / group)};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(q), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// A bf16 pool [NB][Hkv][BS][128] as (64 channels, half, token row); a box is one block's
+// tokens of one half.
+inline bool make_kv_map(CUtensorMap* m, const void* pool, int64_t token_rows, int bs) {
+  auto enc = tc::encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[3] = {64, 2, (cuuint64_t)token_rows};
+  cuuint64_t strides[2] = {128, 256};
+  cuuint32_t box[3] = {64, 1, (cuuint32_t)bs};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pool), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int BS>
+inline cudaError_t launch_bs(const PrefillArgs& a, const void* q, const void* kc, const void* vc,
+                             cudaStream_t st) {
+  CUtensorMap qm, km, vm;
+  const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
+  if (!make_q_map(&qm, q, a.num_tokens, a.num_q_heads, a.group) ||
+      !make_kv_map(&km, kc, rows, BS) || !make_kv_map(&vm, vc, rows, BS))
+    return cudaErrorInvalidValue;
+  static bool attr = false;
+  if (!attr) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<BS>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    attr = true;
+  }
+  const int tiles = (a.max_query_len * a.group + kBM - 1) / kBM;
+  const dim3 grid(tiles, a.num_kv_heads, a.num_seqs);
+  prefill_tc_kernel<BS><<<grid, kThreads, kSmem, st>>>(a, qm, km, vm);
+  return cudaGetLastError();
+}
+
+}  // namespace pf
+
+// Shapes the tensor-core prefill kernel takes: bf16 everywhere, head_dim 128, a group that
+// divides the 128 tile rows, blocks of 8, 16 or 32 tokens.
+inline bool prefill_tc_supported(const pa_decode_desc* d) {
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (d->kv_dtype != PA_BF16 || d->q_dtype != PA_BF16 || d->out_dtype != PA_BF16) return false;
+  if (d->head_dim != pf::kD) return false;
+  if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return false;
+  if (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) return false;
+  return (int64_t)d->num_blocks * d->num_kv_heads * d->block_size < ((int64_t)1 << 31);
+}
+
+inline cudaError_t launch_prefill_tc(const pf::PrefillArgs& a, int block_size, const void* q,
+                                     const void* kc, const void* vc, cudaStream_t st) {
+  if (block_size == 8) return pf::launch_bs<8>(a, q, kc, vc, st);
+  if (block_size == 32) return pf::launch_bs<32>(a, q, kc, vc, st);
+  return pf::launch_bs<16>(a, q, kc, vc, st);
+}
+
+}  // namespace pa

@@ -235,3 +235,87 @@ class DeviceScenario:
         copy = len(self.cow_pairs) * 2 * Hkv * B * d * es * 2
         return {"decode": decode, "write": write, "copy": copy, "kv": kv,
                 "total": decode + write + copy}
+
+
+class PrefillScenario(DeviceScenario):
+    """A prefill step of a synthetic workload, built on the GPU through the library.
+
+    Blocks come from the native allocator in the draw's pool order: every sequence is added
+    with its cached tokens (written beforehand with reshape_and_cache), then appends the
+    step's new tokens. The step writes the new tokens' K/V and runs paged_attn_prefill for
+    them. K/V of sequences outside ``draw_seqs`` is seeded N(0, 1) drawn on the device.
+    """
+
+    def __init__(self, draw, draw_seqs: Optional[Sequence[int]] = None, device="cuda"):
+        import torch
+        self.torch = torch
+        self.draw = draw
+        wl = self.wl = draw.wl
+        S, B, H, d = wl.num_seqs, wl.block_size, wl.num_kv_heads, wl.head_dim
+        self.device = device
+        self.draw_seqs = set(range(S)) if draw_seqs is None else set(draw_seqs)
+        self.is_shared = False
+        self.partition_size = 0
+        self.tdtype = torch.float32 if wl.in_dtype == "f32" else torch.bfloat16
+        lens, qn = draw.context_lens, draw.query_lens
+        self.max_context_len = int(lens.max()) if S else 0
+        self.max_query_len = int(qn.max()) if S else 0
+        self.max_blocks = max(1, _ceil_div(self.max_context_len, B))
+        self.cache = c = PagedKVCache(wl.num_blocks, H, d, wl.kv_dtype, B, device,
+                                      draw.pool_order)
+        pre, new = {}, {}
+        for s in range(S):
+            pre[s] = c.add_seq(s, int(lens[s] - qn[s]))
+        for s in range(S):
+            sl, pr = c.append(s, int(qn[s]))
+            assert not pr
+            new[s] = sl
+        self.cow_pairs, self.pairs = [], None
+        self.block_tables = c.block_tables(range(S), self.max_blocks).to(device)
+        self.context_lens = torch.from_numpy(lens.astype(np.int32)).to(device)
+        self.query_start = torch.from_numpy(draw.query_start.astype(np.int32)).to(device)
+        tables_host = self.block_tables.cpu().numpy()
+        step_k, step_v, step_sl = [], [], []
+        for s in range(S):
+            k, v = self._seq_kv(s)
+            if wl.kv_dtype == "fp8":
+                self._set_scales(s, k, v, tables_host[s])
+            elif wl.kv_dtype == "int8":
+                self._set_int8(s, k, v, tables_host[s])
+            cached = int(lens[s] - qn[s])
+            if cached:
+                self._write(k[:cached], v[:cached], pre[s])
+            step_k.append(k[cached:])
+            step_v.append(v[cached:])
+            step_sl.append(new[s])
+        self.step_k = torch.cat(step_k).contiguous()
+        self.step_v = torch.cat(step_v).contiguous()
+        self.step_slots = torch.from_numpy(np.concatenate(step_sl).astype(np.int64)).to(device)
+        self.q = self._host_to_dev(draw.q)
+        self.scale = float(np.float32(1.0 / math.sqrt(d)))
+        self.out = torch.empty_like(self.q)
+        self.lse = torch.empty((self.q.shape[0], wl.num_q_heads), dtype=torch.float32,
+                               device=device)
+        self.workspace = None
+        torch.cuda.synchronize()
+
+    def step(self, stream=None):
+        c = self.cache
+        c.write(self.step_k, self.step_v, self.step_slots, stream=stream)
+        c.prefill(self.q, self.block_tables, self.context_lens, self.query_start, self.scale,
+                  self.out, max_query_len=self.max_query_len,
+                  max_context_len=self.max_context_len, lse_out=self.lse, stream=stream)
+        return self.out
+
+    def launches_per_step(self) -> int:
+        return 2
+
+    def flops(self) -> int:
+        """Multiply-adds x 2 of the causal products: every new token's row of S = q K^T
+        and of P V over its visible keys (position + 1), for every query head."""
+        wl = self.wl
+        lens = self.draw.context_lens.astype(np.int64)
+        qn = self.draw.query_lens.astype(np.int64)
+        # sum over new tokens of (position + 1) = sum_{i<n} (ctx - n + i + 1)
+        keys = int(np.sum(qn * (lens - qn) + qn * (qn + 1) // 2))
+        return 4 * wl.head_dim * wl.num_q_heads * keys

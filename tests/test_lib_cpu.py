@@ -193,3 +193,27 @@ def test_binding_refuses_host_tensors(pa):
     with pytest.raises(ValueError):
         pa.paged_attn_decode(q, kc, kc, torch.zeros(4, 3, dtype=torch.int32),
                              torch.zeros(4, dtype=torch.int32), 0.125, q.clone(), max_context_len=40)
+
+
+def test_prefill_host_validation_without_device(pa):
+    lib = pa._lib
+    nul = ctypes.c_void_p(0)
+    one = ctypes.c_void_p(256)
+    d = pa.make_desc(4, 32, 8, 128, 64, 1024, 0, pa.PA_BF16, pa.PA_BF16, pa.PA_BF16)
+
+    def call(desc, tokens=100, max_q=50, max_ctx=1024, ptr=one, qs=one, scale=0.1):
+        return lib.paged_attn_prefill(ptr, ptr, ptr, ptr, ptr, qs, tokens, max_q,
+                                      ctypes.c_float(scale), ptr, ctypes.byref(desc), max_ctx,
+                                      nul, nul, nul, nul, nul, nul)
+    split = pa.make_desc(4, 32, 8, 128, 64, 1024, 512, pa.PA_BF16, pa.PA_BF16, pa.PA_BF16)
+    assert call(split) == pa.PA_ERR_INVALID                     # no split-KV for prefill
+    assert call(d, tokens=-1) == pa.PA_ERR_INVALID
+    assert call(d, max_q=2000, max_ctx=1024) == pa.PA_ERR_INVALID  # a query past its context
+    assert call(d, max_ctx=1025) == pa.PA_ERR_INVALID            # table shorter than context
+    assert call(d, scale=float("nan")) == pa.PA_ERR_INVALID
+    assert call(d, qs=nul) == pa.PA_ERR_INVALID                  # query_start is required
+    assert call(d, tokens=0, ptr=nul, qs=nul) == pa.PA_OK         # nothing to do
+    uns = pa.make_desc(4, 32, 8, 96, 64, 1024, 0, pa.PA_BF16, pa.PA_BF16, pa.PA_BF16)
+    assert call(uns) == pa.PA_ERR_UNSUPPORTED
+    fp8 = pa.make_desc(4, 32, 8, 128, 64, 1024, 0, pa.PA_BF16, pa.PA_FP8_E4M3, pa.PA_BF16)
+    assert call(fp8) == pa.PA_ERR_INVALID                        # fp8 needs its scales

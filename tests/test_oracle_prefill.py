@@ -43,7 +43,8 @@ def _scale(draw):
 
 def test_one_new_token_is_a_decode_step():
     wl = workloads.PREFILL_WORKLOADS["chunked"].scaled(num_seqs=4, new=("chunk", 1),
-                                                       lens=("fixed", [1, 17, 300, 1000]))
+                                                       lens=("fixed", [1, 17, 300, 1000]),
+                                                       num_blocks=256)
     d = workloads.draw_prefill(wl)
     st = flows.build_prefill_state(d)
     o, l = flows.ref_prefill_outputs(d, st)
@@ -71,8 +72,8 @@ def test_whole_prompts_match_library_causal_attention(B):
 
 
 def test_chunks_are_the_last_rows_of_a_whole_context_pass():
-    d = workloads.draw_prefill(workloads.PREFILL_WORKLOADS["chunked"].scaled(num_seqs=3,
-                               lens=("fixed", [600, 513, 1500])))
+    d = workloads.draw_prefill(workloads.PREFILL_WORKLOADS["chunked"].scaled(
+        num_seqs=3, lens=("fixed", [600, 513, 1500]), num_blocks=256))
     st = flows.build_prefill_state(d)
     o, l = flows.ref_prefill_outputs(d, st)
     rng = np.random.default_rng(5)
