@@ -7,19 +7,23 @@
 // tokens after it); [Ch4PA] "PagedAttention algorithm" (keys and values are gathered from
 // non-contiguous blocks through the block table).
 //
-// One CTA per (128-row query tile, kv head, sequence). A tile row is a (new token, query
-// head of the kv head's group) pair, so one key/value tile serves the whole group. Keys are
-// taken 128 at a time:
-//   warp 5 (one lane)   TMA: Q once; K and V of key tile j into stage j % 2, one box per
-//                       (block, 64-channel half) straight from the paged pool;
+// One CTA per (128-row query tile, kv head, sequence); two CTAs share an SM, so one CTA's
+// softmax overlaps the other's products. A tile row is a (new token, query head of the kv
+// head's group) pair, so one key/value tile serves the whole group. Keys are taken 64 at
+// a time:
+//   warp 5 (one lane)   TMA: Q once; K and V of key tile j into their own two-stage rings,
+//                       one box per (block, 64-channel half) straight from the paged pool;
+//                       a K stage is refilled once its S product is done, a V stage once
+//                       its P V product is done;
 //   warp 4 (one lane)   tcgen05.mma: S_j = Q K_j^T into tensor memory (two S buffers, so
-//                       S_{j+1} runs while S_j is in softmax), then O += P_j V_j;
+//                       S_{j+1} runs while S_j is in softmax), then O += P_j V_j with P_j
+//                       read from tensor memory;
 //   warps 0-3           softmax, one thread per tile row (= tensor-memory lane): causal
 //                       mask, running max (rescaling O in tensor memory only when the max
-//                       grows by more than 2^8), P_j as bf16 into shared memory; finally
-//                       O / l to `out` and the log-sum-exp to `lse_out`.
-// Operands sit in shared memory in the 128-byte-swizzled layouts the tensor core reads:
-// Q, K and P K-major (rows of 64 channels / keys, 128 B), V MN-major (rows of keys).
+//                       grows by more than 2^8), P_j as bf16 pairs written over S_j;
+//                       finally O / l to `out` and the log-sum-exp to `lse_out`.
+// Operands in shared memory use the 128-byte-swizzled layouts the tensor core reads: Q and
+// K K-major (rows of 64 channels, 128 B), V MN-major (rows of keys).
 // Every wait is bounded; a CTA that gives up flags PA_DEVERR_TIMEOUT, lets its issued
 // copies and products finish, and releases its tensor memory.
 #pragma once
@@ -37,27 +41,30 @@ using tc::mbar_wait;
 using tc::smem_u32;
 
 constexpr int kBM = 128;                  // tile rows: (new token, head) pairs
-constexpr int kBN = 128;                  // keys per key tile
+constexpr int kBN = 64;                   // keys per key tile
 constexpr int kD = 128;                   // head dimension
 constexpr int kThreads = 192;             // warps 0-3 softmax, 4 MMA, 5 TMA
 constexpr int kMmaWarp = 4, kTmaWarp = 5;
-constexpr int kSlab = 128 * 128;          // 64 channels (128 B) x 128 rows
-constexpr int kTile = 2 * kSlab;          // 128 rows x 128 bf16
+constexpr int kQSlab = kBM * 128;         // 64 channels (128 B) x 128 rows
+constexpr int kQBytes = 2 * kQSlab;
+constexpr int kKVSlab = kBN * 128;        // 64 channels x 64 keys
+constexpr int kKVBytes = 2 * kKVSlab;
+constexpr int kKSt = 2, kVSt = 2;         // ring depths
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kTile;      // 2 stages
-constexpr int kOffV = kOffK + 2 * kTile;  // 2 stages
-constexpr int kOffP = kOffV + 2 * kTile;
-constexpr int kOffBar = kOffP + kTile;
+constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffV = kOffK + kKSt * kKVBytes;
+constexpr int kOffBar = kOffV + kVSt * kKVBytes;
 constexpr int kSmem = kOffBar + 256 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t kTmemCols = 512;       // S buffers at columns 0 / 128, O at 256
-constexpr uint32_t kOCol = 256;
+constexpr uint32_t kTmemCols = 256;       // S / P buffers at columns 0 and 64, O at 128
+constexpr uint32_t kOCol = 128;
 
 // barrier indices
-enum { kBarQ = 0, kBarKF = 1, kBarVF = 3, kBarKVE = 5, kBarSF = 7, kBarP = 9, kBarO = 10,
-       kBarFin = 11, kNumBars = 12 };
+enum { kBarQ = 0, kBarKF = 1, kBarKE = 3, kBarVF = 5, kBarVE = 7, kBarSF = 9, kBarP = 11,
+       kBarO = 12, kBarFin = 13, kNumBars = 14 };
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
-// S = Q K^T: A and B K-major, N = 128 keys. O += P V: B (V) MN-major, N = 128 channels.
+// S = Q K^T: A and B K-major, N = 64 keys. O += P V: A (P) from tensor memory, B (V)
+// MN-major, N = 128 channels.
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                              ((uint32_t)(kBM >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
@@ -110,6 +117,15 @@ __device__ __forceinline__ void tc_fence_after() {
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                ::"r"(bar) : "memory");
+}
+// D (tensor memory) = A B (+ D when acc != 0), A from tensor memory (K-major: a row per
+// lane, two bf16 per column), B from a shared-memory descriptor.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
 }
 // D (tensor memory) = A B (+ D when acc != 0), A and B from shared-memory descriptors.
 __device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
@@ -196,11 +212,12 @@ __device__ __forceinline__ bool seq_rows(const PrefillArgs& a, int s, int& q0, i
 }
 
 template <int BS>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
 prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap) {
   static_assert(kBN % BS == 0 && kBN / BS <= 32, "block size");
+  constexpr int NB_T = kBN / BS;  // blocks per key tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -219,7 +236,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   const int ntiles = (kv_end + kBN - 1) / kBN;
 
   const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK);
-  const uint32_t sV = smem_u32(smem + kOffV), sP = smem_u32(smem + kOffP);
+  const uint32_t sV = smem_u32(smem + kOffV);
   const uint32_t bar0 = smem_u32(smem + kOffBar);
   auto bar = [&](int i) { return bar0 + 8u * (uint32_t)i; };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + 8 * kNumBars);
@@ -230,8 +247,9 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     mbar_init(bar(kBarQ), 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(bar(kBarKF + i), 1);
+      mbar_init(bar(kBarKE + i), 1);
       mbar_init(bar(kBarVF + i), 1);
-      mbar_init(bar(kBarKVE + i), 1);
+      mbar_init(bar(kBarVE + i), 1);
       mbar_init(bar(kBarSF + i), 1);
     }
     mbar_init(bar(kBarP), kBM);
@@ -245,56 +263,77 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
+  // any block id out of range among the keys the tile sees? (then tiles are checked one by
+  // one; otherwise no per-tile checks)
+  int bad = 0;
+  for (int b = threadIdx.x; b < (kv_end + BS - 1) / BS; b += kThreads) {
+    const int p = bt[b];
+    bad |= p < 0 || p >= a.num_blocks;
+  }
   tc_fence_before();
-  __syncthreads();
+  const bool any_bad = __syncthreads_or(bad) != 0;
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kTmaWarp) {
-    // ---------------- producer: Q once, then K / V tiles through two stages ----------------
+    // ---------------- producer: Q once, then K and V tiles through their rings ----------------
     if (lane == 0) {
-      mbar_arrive_tx(bar(kBarQ), kTile);
+      mbar_arrive_tx(bar(kBarQ), kQBytes);
       const uint64_t pol = evict_first_policy();
       for (int h = 0; h < 2; ++h)
-        tma_load_4d(sQ + h * kSlab, &qmap, 0, h, kvh * G, q0 + tok0, bar(kBarQ), pol);
-      int last[2] = {-1, -1};
+        tma_load_4d(sQ + h * kQSlab, &qmap, 0, h, kvh * G, q0 + tok0, bar(kBarQ), pol);
+      int last_k[kKSt], last_v[kVSt];
+      for (int i = 0; i < kKSt; ++i) last_k[i] = -1;
+      for (int i = 0; i < kVSt; ++i) last_v[i] = -1;
       for (int j = 0; j < ntiles && !*dead; ++j) {
-        const int st = j & 1;
-        if (j >= 2 && !mbar_wait(bar(kBarKVE + st), ((j >> 1) - 1) & 1)) {
+        const int t0 = j * kBN;
+        const int nblk = (min(kBN, kv_end - t0) + BS - 1) / BS;
+        int phys[NB_T];
+        int nvalid = 0;
+#pragma unroll
+        for (int b = 0; b < NB_T; ++b) {
+          phys[b] = b < nblk ? bt[t0 / BS + b] : -1;
+          if (b < nblk && (phys[b] < 0 || phys[b] >= a.num_blocks)) {
+            flag_error(PA_DEVERR_BLOCK_ID);
+            phys[b] = -1;
+          }
+          nvalid += phys[b] >= 0;
+        }
+        const uint32_t bytes = (uint32_t)nvalid * 2u * BS * 128u;
+        bool ok = true;
+#pragma unroll
+        for (int kv = 0; kv < 2; ++kv) {
+          const int nst = kv ? kVSt : kKSt;
+          const int st = j % nst;
+          if (j >= nst && !mbar_wait(bar((kv ? kBarVE : kBarKE) + st), ((j / nst) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar((kv ? kBarVF : kBarKF) + st);
+          const uint32_t dst = (kv ? sV : sK) + st * kKVBytes;
+          const CUtensorMap* map = kv ? &vmap : &kmap;
+          mbar_arrive_tx(fb, bytes);
+#pragma unroll
+          for (int b = 0; b < NB_T; ++b) {
+            if (phys[b] < 0) continue;
+            const int row = (phys[b] * a.num_kv_heads + kvh) * BS;
+            tma_load_3d(dst + b * BS * 128, map, 0, 0, row, fb);
+            tma_load_3d(dst + kKVSlab + b * BS * 128, map, 0, 1, row, fb);
+          }
+          (kv ? last_v : last_k)[st] = j;
+        }
+        if (!ok) {
           flag_error(PA_DEVERR_TIMEOUT);
           *dead = 1;
           break;
         }
-        const int t0 = j * kBN;
-        const int nblk = (min(kBN, kv_end - t0) + BS - 1) / BS;
-        int nvalid = 0;
-        for (int b = 0; b < nblk; ++b) {
-          const int p = bt[t0 / BS + b];
-          if (p >= 0 && p < a.num_blocks) ++nvalid;
-          else flag_error(PA_DEVERR_BLOCK_ID);
-        }
-        const uint32_t bytes = (uint32_t)nvalid * 2u * BS * 128u;
-        for (int kv = 0; kv < 2; ++kv) {
-          const uint32_t fb = bar((kv ? kBarVF : kBarKF) + st);
-          const uint32_t dst = (kv ? sV : sK) + st * kTile;
-          const CUtensorMap* map = kv ? &vmap : &kmap;
-          mbar_arrive_tx(fb, bytes);
-          for (int b = 0; b < nblk; ++b) {
-            const int p = bt[t0 / BS + b];
-            if (p < 0 || p >= a.num_blocks) continue;
-            const int row = (p * a.num_kv_heads + kvh) * BS;
-            for (int h = 0; h < 2; ++h) tma_load_3d(dst + h * kSlab + b * BS * 128, map, 0, h, row, fb);
-          }
-        }
-        last[st] = j;
       }
       if (*dead) {
         // copies still in flight complete before the CTA's shared memory is released
-        for (int st = 0; st < 2; ++st)
-          if (last[st] >= 0) {
-            mbar_wait(bar(kBarKF + st), (last[st] >> 1) & 1);
-            mbar_wait(bar(kBarVF + st), (last[st] >> 1) & 1);
-          }
+        for (int i = 0; i < kKSt; ++i)
+          if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
+        for (int i = 0; i < kVSt; ++i)
+          if (last_v[i] >= 0) mbar_wait(bar(kBarVF + i), (last_v[i] / kVSt) & 1);
         mbar_wait(bar(kBarQ), 0);
       }
     }
@@ -303,25 +342,26 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
       auto issue_s = [&](int j) {
-        const uint32_t kst = sK + (j & 1) * kTile;
+        const uint32_t kst = sK + (j % kKSt) * kKVBytes;
         const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kSlab + (kk & 3) * 32;
-          umma_bf16(d, sdesc(sQ + off, 16, 1024), sdesc(kst + off, 16, 1024), kIdescS, kk > 0);
+          const uint32_t oq = (kk >> 2) * kQSlab + (kk & 3) * 32;
+          const uint32_t ok_ = (kk >> 2) * kKVSlab + (kk & 3) * 32;
+          umma_bf16(d, sdesc(sQ + oq, 16, 1024), sdesc(kst + ok_, 16, 1024), kIdescS, kk > 0);
         }
         umma_commit(bar(kBarSF + (j & 1)));
+        umma_commit(bar(kBarKE + (j % kKSt)));  // the K stage is free once S_j is done
       };
       auto issue_pv = [&](int j) {
-        const uint32_t vst = sV + (j & 1) * kTile;
+        const uint32_t vst = sV + (j % kVSt) * kKVBytes;
+        const uint32_t pa_ = tmem + (uint32_t)((j & 1) * kBN);  // P_j over S_j
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * kSlab + (kk & 3) * 32;
-          umma_bf16(tmem + kOCol, sdesc(sP + aoff, 16, 1024),
-                    sdesc(vst + kk * 16 * 128, kSlab, 1024), kIdescPV, (j > 0 || kk > 0));
-        }
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          umma_bf16_ts(tmem + kOCol, pa_ + kk * 8, sdesc(vst + kk * 16 * 128, kKVSlab, 1024),
+                       kIdescPV, (j > 0 || kk > 0));
         umma_commit(bar(kBarO));
-        umma_commit(bar(kBarKVE + (j & 1)));
+        umma_commit(bar(kBarVE + (j % kVSt)));
       };
       bool live = mbar_wait(bar(kBarQ), 0) && mbar_wait(bar(kBarKF), 0);
       if (live) {
@@ -330,10 +370,14 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       }
       for (int j = 0; live && j < ntiles; ++j) {
         if (j + 1 < ntiles) {
-          if (!mbar_wait(bar(kBarKF + ((j + 1) & 1)), ((j + 1) >> 1) & 1)) { live = false; break; }
+          if (!mbar_wait(bar(kBarKF + ((j + 1) % kKSt)), ((j + 1) / kKSt) & 1)) {
+            live = false;
+            break;
+          }
           issue_s(j + 1);
         }
-        if (!mbar_wait(bar(kBarP), j & 1) || !mbar_wait(bar(kBarVF + (j & 1)), (j >> 1) & 1)) {
+        if (!mbar_wait(bar(kBarP), j & 1) ||
+            !mbar_wait(bar(kBarVF + (j % kVSt)), (j / kVSt) & 1)) {
           live = false;
           break;
         }
@@ -357,7 +401,8 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     const bool row_valid = tr < ntok;
     const int prow = pos_min + min(tr, ntok - 1);       // this row's position
     const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
-    float m_used = -INFINITY, l = 0.f;
+    const float sl2 = a.scale_log2;
+    float m_used = -INFINITY, l = 0.f;                  // log2-domain reference max, sum
     bool ok = true;
     // waits are made warp-uniform: the tcgen05.ld / st below are warp-collective
     auto wait_all = [&](uint32_t b, uint32_t parity) {
@@ -369,56 +414,70 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       tc_fence_after();
       const int t0 = j * kBN;
       const int vlim = min(kBN, kv_end - t0);             // keys of the tile that exist
-      // blocks of the tile with an out-of-range id: skipped by the producer, masked here
-      uint32_t badm = 0;
-      {
-        const int nblk = (vlim + BS - 1) / BS;
-        bool bad = false;
-        if (lane < nblk) {
+      uint32_t badm = 0;  // blocks of the tile with an out-of-range id (skipped, masked)
+      if (any_bad) {
+        bool b = false;
+        if (lane < (vlim + BS - 1) / BS) {
           const int p = bt[t0 / BS + lane];
-          bad = p < 0 || p >= a.num_blocks;
+          b = p < 0 || p >= a.num_blocks;
         }
-        badm = __ballot_sync(0xffffffffu, bad);
+        badm = __ballot_sync(0xffffffffu, b);
       }
-      uint32_t sv[4][32];
+      const uint32_t sbuf = lane_addr + (uint32_t)((j & 1) * kBN);
+      uint32_t sv[2][32];
+      tmem_ld32(sbuf, sv[0]);
+      tmem_ld32(sbuf + 32, sv[1]);
+      tmem_wait_ld(sv[0]);
+      tmem_wait_ld(sv[1]);
+      // causal / existence / bad-block mask, then the row max of the raw scores
+      if (t0 + kBN - 1 > pos_min || badm != 0) {  // uniform in the CTA
+        const int lim = prow - t0;                   // visible: key <= lim
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_addr + (uint32_t)((j & 1) * kBN + c * 32), sv[c]);
+        for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
-      const bool need_mask = t0 + kBN - 1 > pos_min || badm != 0;  // uniform in the CTA
-      const int lim = prow - t0;                                  // visible: key <= lim
-      float mx = -INFINITY;
+          for (int e = 0; e < 32; ++e) {
+            const int col = c * 32 + e;
+            if (col > lim || ((badm >> (col / BS)) & 1u)) sv[c][e] = 0xff800000u;  // -inf
+          }
+      }
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int col = c * 32 + e;
-          float x = __uint_as_float(sv[c][e]) * a.scale_log2;
-          if (need_mask && (col > lim || ((badm >> (col / BS)) & 1u))) x = -INFINITY;
-          sv[c][e] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
-        }
+      for (int c = 0; c < 2; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sv[c][e]));
+#pragma unroll
+      for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
+      const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * sl2;
       const float m_new = fmaxf(m_used, mx);
       float alpha = 1.f;
       if (m_new > m_used + 8.f) {  // lazy rescale: P stays below 2^8 otherwise
         alpha = fast_exp2(m_used - m_new);
         m_used = m_new;
       }
-      const float mref = m_used == -INFINITY ? 0.f : m_used;
-      float rs = 0.f;
-      uint32_t pk[64];
+      const float mneg = m_used == -INFINITY ? 0.f : -m_used;
+      float rs8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = fast_exp2(__uint_as_float(sv[c][e]) - mref);
-          const float p1 = fast_exp2(__uint_as_float(sv[c][e + 1]) - mref);
-          rs += p0 + p1;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][e]), sl2, mneg));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][e + 1]), sl2, mneg));
+          rs8[e & 7] += p0;
+          rs8[(e + 1) & 7] += p1;
           pk[(c * 32 + e) >> 1] = pack_bf16x2(p0, p1);
         }
-      l = l * alpha + rs;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rs8[k] += rs8[k + 4];
+      l = l * alpha + ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3]));
+      tmem_st32(sbuf, pk);  // P_j over the first 32 columns of S_j
+      tmem_wait_st();
       if (j > 0) {
-        // P_{j-1} and O are free once the previous product has completed
+        // O holds P_{j-1} V_{j-1} once the previous product is done; rescale it if needed
         if (!wait_all(bar(kBarO), (j - 1) & 1)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
@@ -434,29 +493,20 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
           tmem_wait_st();
         }
       }
-      // P_j, K-major with the 128-byte swizzle: keys 64h.. in slab h, row r
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        const uint32_t addr = sP + (k >> 3) * kSlab + r * 128 + (((k & 7) ^ (r & 7)) << 4);
-        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                     ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]), "r"(pk[4 * k + 2]),
-                       "r"(pk[4 * k + 3]) : "memory");
-      }
       // rows of V past the keys that exist or in a skipped block may hold anything (NaN):
       // zero them before the product reads them
       if (vlim < kBN || badm != 0) {
-        if (!wait_all(bar(kBarVF + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
-        if (r >= vlim || ((badm >> (r / BS)) & 1u)) {
-          const uint32_t vrow = sV + (j & 1) * kTile + r * 128;
+        if (!wait_all(bar(kBarVF + (j % kVSt)), (j / kVSt) & 1)) { ok = false; break; }
+        const int vr = r >> 1, h = r & 1;  // 128 threads: 64 rows x 2 channel halves
+        if (vr >= vlim || ((badm >> (vr / BS)) & 1u)) {
+          const uint32_t vrow = sV + (j % kVSt) * kKVBytes + h * kKVSlab + vr * 128;
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};"
-                           ::"r"(vrow + h * kSlab + k * 16), "r"(0) : "memory");
+          for (int k = 0; k < 8; ++k)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + k * 16), "r"(0)
+                         : "memory");
         }
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       tc_fence_before();
       mbar_arrive(bar(kBarP));
     }
