@@ -35,6 +35,7 @@ METRIC = "paged decode attention KV GB/s (% of HBM peak) and decode tokens/s at 
 UNIT = "GB/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 DTYPE = {"f32": "f32", "bf16": "bf16-kv/f32-acc", "fp8": "fp8e4m3-kv/f32-acc",
          "int8": "int8-kv/f32-acc"}
 DESCR = {
@@ -354,6 +355,55 @@ def _last_block_waste(lens, block_size):
     return (alloc - int(lens.sum())) / alloc if alloc else 0.0
 
 
+def _bf16_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def _prefill_workloads(torch, flush):
+    """Prefill steps (write the new tokens' K/V, then causal attention over the paged cache)
+    on the prefill workloads: TFLOP/s of the attention call against the bf16 tensor peak."""
+    from paged_kv_cache_465_b200.scenario import PrefillScenario
+    peak, kind = _bf16_peak()
+    out = {}
+    for name in ("prefill", "chunked"):
+        draw = workloads.draw_prefill(name)
+        sc = PrefillScenario(draw, draw_seqs=[])
+        for _ in range(3):
+            flush()
+            sc.step()
+        steps = 30
+        st = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        for i in range(steps):
+            flush()
+            e0, e1, e2 = ev[i]
+            e0.record(st)
+            sc.cache.write(sc.step_k, sc.step_v, sc.step_slots)
+            e1.record(st)
+            sc.cache.prefill(sc.q, sc.block_tables, sc.context_lens, sc.query_start, sc.scale,
+                             sc.out, max_query_len=sc.max_query_len,
+                             max_context_len=sc.max_context_len, lse_out=sc.lse)
+            e2.record(st)
+        torch.cuda.synchronize()
+        total = sum(a.elapsed_time(c) for a, b, c in ev) / 1e3 / steps
+        attn = sum(b.elapsed_time(c) for a, b, c in ev) / 1e3 / steps
+        tflops = sc.flops() / attn / 1e12
+        out[name] = {"value": round(tflops, 1), "unit": "TFLOP/s",
+                     "pct_bf16_peak": round(100 * tflops / peak, 2), "peak_kind": kind,
+                     "ms_per_step": round(total * 1e3, 5), "attention_ms": round(attn * 1e3, 5),
+                     "new_tokens_per_s": round(draw.num_tokens / total, 1),
+                     "flops_per_step": sc.flops(), "steps": steps,
+                     "kernel": "tcgen05 prefill (S and O in tensor memory)"}
+        del sc
+        torch.cuda.empty_cache()
+    return out
+
+
 def _extra_workloads(torch, pa, args, flush):
     from paged_kv_cache_465_b200.scenario import DeviceScenario
     peak, _ = _peaks()
@@ -387,6 +437,7 @@ def _extra_workloads(torch, pa, args, flush):
                      "steps": steps}
         del sc
         torch.cuda.empty_cache()
+    out.update(_prefill_workloads(torch, flush))
     return out
 
 

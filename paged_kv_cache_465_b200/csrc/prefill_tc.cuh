@@ -58,9 +58,11 @@ constexpr int kSmem = kOffBar + 256 + 1024;  // + barriers, + alignment slack
 constexpr uint32_t kTmemCols = 256;       // S / P buffers at columns 0 and 64, O at 128
 constexpr uint32_t kOCol = 128;
 
-// barrier indices
+// barrier indices; the P V products complete on a ring of four barriers, so the softmax
+// waits for one only when it rescales O (no phase of a barrier is ever two ahead of it)
+constexpr int kORing = 4;
 enum { kBarQ = 0, kBarKF = 1, kBarKE = 3, kBarVF = 5, kBarVE = 7, kBarSF = 9, kBarP = 11,
-       kBarO = 12, kBarFin = 13, kNumBars = 14 };
+       kBarO = 12, kBarFin = 12 + kORing, kNumBars = 13 + kORing };
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
 // S = Q K^T: A and B K-major, N = 64 keys. O += P V: A (P) from tensor memory, B (V)
@@ -253,7 +255,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       mbar_init(bar(kBarSF + i), 1);
     }
     mbar_init(bar(kBarP), kBM);
-    mbar_init(bar(kBarO), 1);
+    for (int i = 0; i < kORing; ++i) mbar_init(bar(kBarO + i), 1);
     mbar_init(bar(kBarFin), 1);
     *dead = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -360,7 +362,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
         for (int kk = 0; kk < kBN / 16; ++kk)
           umma_bf16_ts(tmem + kOCol, pa_ + kk * 8, sdesc(vst + kk * 16 * 128, kKVSlab, 1024),
                        kIdescPV, (j > 0 || kk > 0));
-        umma_commit(bar(kBarO));
+        umma_commit(bar(kBarO + j % kORing));
         umma_commit(bar(kBarVE + (j % kVSt)));
       };
       bool live = mbar_wait(bar(kBarQ), 0) && mbar_wait(bar(kBarKF), 0);
@@ -476,11 +478,14 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       l = l * alpha + ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3]));
       tmem_st32(sbuf, pk);  // P_j over the first 32 columns of S_j
       tmem_wait_st();
-      if (j > 0) {
-        // O holds P_{j-1} V_{j-1} once the previous product is done; rescale it if needed
-        if (!wait_all(bar(kBarO), (j - 1) & 1)) { ok = false; break; }
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O holds P_{j-1} V_{j-1} once the previous product is done: rescale it
+        if (!wait_all(bar(kBarO + (j - 1) % kORing), ((j - 1) / kORing) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        {
 #pragma unroll 1
           for (int c = 0; c < 4; ++c) {
             uint32_t o[32];
@@ -510,7 +515,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       tc_fence_before();
       mbar_arrive(bar(kBarP));
     }
-    if (ok) ok = wait_all(bar(kBarO), (ntiles - 1) & 1);
+    if (ok) ok = wait_all(bar(kBarO + (ntiles - 1) % kORing), ((ntiles - 1) / kORing) & 1);
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
