@@ -11,10 +11,11 @@
 // softmax overlaps the other's products. A tile row is a (new token, query head of the kv
 // head's group) pair, so one key/value tile serves the whole group. Keys are taken 64 at
 // a time:
-//   warp 5 (one lane)   TMA: Q once; K and V of key tile j into their own two-stage rings,
-//                       one box per (block, 64-channel half) straight from the paged pool;
-//                       a K stage is refilled once its S product is done, a V stage once
-//                       its P V product is done;
+//   warp 5              TMA: Q once; K and V of key tile j into their own two-stage rings,
+//                       one box per (block, 64-channel half) straight from the paged pool,
+//                       issued by one lane each; block ids are read one tile ahead; a K stage
+//                       is refilled once its S product is done, a V stage once its P V
+//                       product is done;
 //   warp 4 (one lane)   tcgen05.mma: S_j = Q K_j^T into tensor memory (two S buffers, so
 //                       S_{j+1} runs while S_j is in softmax), then O += P_j V_j with P_j
 //                       read from tensor memory;
@@ -278,66 +279,76 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kTmaWarp) {
-    // ---------------- producer: Q once, then K and V tiles through their rings ----------------
+    // ---------------- producer (whole warp): Q once, then K and V tiles through their rings.
+    // Lane b < NB_T holds the physical block b of a key tile, read one tile ahead so the
+    // table load hides behind the ring waits; each lane issues one (block, half) box, so a
+    // tile's K (or V) copies leave in one warp instruction.
     if (lane == 0) {
       mbar_arrive_tx(bar(kBarQ), kQBytes);
       const uint64_t pol = evict_first_policy();
       for (int h = 0; h < 2; ++h)
         tma_load_4d(sQ + h * kQSlab, &qmap, 0, h, kvh * G, q0 + tok0, bar(kBarQ), pol);
-      int last_k[kKSt], last_v[kVSt];
-      for (int i = 0; i < kKSt; ++i) last_k[i] = -1;
-      for (int i = 0; i < kVSt; ++i) last_v[i] = -1;
-      for (int j = 0; j < ntiles && !*dead; ++j) {
-        const int t0 = j * kBN;
-        const int nblk = (min(kBN, kv_end - t0) + BS - 1) / BS;
-        int phys[NB_T];
-        int nvalid = 0;
-#pragma unroll
-        for (int b = 0; b < NB_T; ++b) {
-          phys[b] = b < nblk ? bt[t0 / BS + b] : -1;
-          if (b < nblk && (phys[b] < 0 || phys[b] >= a.num_blocks)) {
-            flag_error(PA_DEVERR_BLOCK_ID);
-            phys[b] = -1;
-          }
-          nvalid += phys[b] >= 0;
+    }
+    auto fetch = [&](int j) {
+      int p = -1;
+      if (j < ntiles && lane < NB_T && j * kBN + lane * BS < kv_end) {
+        p = bt[j * (kBN / BS) + lane];
+        if (p < 0 || p >= a.num_blocks) {
+          flag_error(PA_DEVERR_BLOCK_ID);
+          p = -1;
         }
-        const uint32_t bytes = (uint32_t)nvalid * 2u * BS * 128u;
-        bool ok = true;
+      }
+      return p;
+    };
+    int last_k[kKSt], last_v[kVSt];
+    for (int i = 0; i < kKSt; ++i) last_k[i] = -1;
+    for (int i = 0; i < kVSt; ++i) last_v[i] = -1;
+    int p_cur = fetch(0);
+    bool ok = true;
+    for (int j = 0; j < ntiles; ++j) {
+      if (__shfl_sync(0xffffffffu, *dead ? 1 : 0, 0)) break;
+      const int p_next = fetch(j + 1);
+      const uint32_t bytes =
+          (uint32_t)__popc(__ballot_sync(0xffffffffu, p_cur >= 0)) * 2u * BS * 128u;
+      const int pb = __shfl_sync(0xffffffffu, p_cur, (lane >> 1) & 31);  // lane's block
 #pragma unroll
-        for (int kv = 0; kv < 2; ++kv) {
-          const int nst = kv ? kVSt : kKSt;
-          const int st = j % nst;
-          if (j >= nst && !mbar_wait(bar((kv ? kBarVE : kBarKE) + st), ((j / nst) - 1) & 1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = bar((kv ? kBarVF : kBarKF) + st);
-          const uint32_t dst = (kv ? sV : sK) + st * kKVBytes;
-          const CUtensorMap* map = kv ? &vmap : &kmap;
-          mbar_arrive_tx(fb, bytes);
-#pragma unroll
-          for (int b = 0; b < NB_T; ++b) {
-            if (phys[b] < 0) continue;
-            const int row = (phys[b] * a.num_kv_heads + kvh) * BS;
-            tma_load_3d(dst + b * BS * 128, map, 0, 0, row, fb);
-            tma_load_3d(dst + kKVSlab + b * BS * 128, map, 0, 1, row, fb);
-          }
-          (kv ? last_v : last_k)[st] = j;
-        }
-        if (!ok) {
-          flag_error(PA_DEVERR_TIMEOUT);
-          *dead = 1;
+      for (int kv = 0; kv < 2; ++kv) {
+        const int nst = kv ? kVSt : kKSt;
+        const int st = j % nst;
+        bool w = true;
+        if (lane == 0 && j >= nst)
+          w = mbar_wait(bar((kv ? kBarVE : kBarKE) + st), ((j / nst) - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
           break;
         }
+        const uint32_t fb = bar((kv ? kBarVF : kBarKF) + st);
+        if (lane == 0) mbar_arrive_tx(fb, bytes);
+        __syncwarp();
+        if (lane < 2 * NB_T && pb >= 0) {
+          const int b = lane >> 1, h = lane & 1;
+          const uint32_t dst = (kv ? sV : sK) + st * kKVBytes + h * kKVSlab + b * BS * 128;
+          tma_load_3d(dst, kv ? &vmap : &kmap, 0, h, (pb * a.num_kv_heads + kvh) * BS, fb);
+        }
+        if (kv) last_v[st] = j;
+        else last_k[st] = j;
       }
-      if (*dead) {
-        // copies still in flight complete before the CTA's shared memory is released
-        for (int i = 0; i < kKSt; ++i)
-          if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
-        for (int i = 0; i < kVSt; ++i)
-          if (last_v[i] >= 0) mbar_wait(bar(kBarVF + i), (last_v[i] / kVSt) & 1);
-        mbar_wait(bar(kBarQ), 0);
+      if (!ok) {
+        if (lane == 0) {
+          flag_error(PA_DEVERR_TIMEOUT);
+          *dead = 1;
+        }
+        break;
       }
+      p_cur = p_next;
+    }
+    if (lane == 0 && *dead) {
+      // copies still in flight complete before the CTA's shared memory is released
+      for (int i = 0; i < kKSt; ++i)
+        if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
+      for (int i = 0; i < kVSt; ++i)
+        if (last_v[i] >= 0) mbar_wait(bar(kBarVF + i), (last_v[i] / kVSt) & 1);
+      mbar_wait(bar(kBarQ), 0);
     }
     __syncwarp();
   } else if (warp == kMmaWarp) {
