@@ -7,22 +7,24 @@
 // tokens after it); [Ch4PA] "PagedAttention algorithm" (keys and values are gathered from
 // non-contiguous blocks through the block table).
 //
-// One CTA per (128-row query tile, kv head, sequence); two CTAs share an SM, so one CTA's
-// softmax overlaps the other's products. A tile row is a (new token, query head of the kv
-// head's group) pair, so one key/value tile serves the whole group. Keys are taken 64 at
-// a time:
-//   warp 5              TMA: Q once; K and V of key tile j into their own two-stage rings,
-//                       one box per (block, 64-channel half) straight from the paged pool,
-//                       issued by one lane each; block ids are read one tile ahead; a K stage
-//                       is refilled once its S product is done, a V stage once its P V
-//                       product is done;
-//   warp 4 (one lane)   tcgen05.mma: S_j = Q K_j^T into tensor memory (two S buffers, so
-//                       S_{j+1} runs while S_j is in softmax), then O += P_j V_j with P_j
-//                       read from tensor memory;
-//   warps 0-3           softmax, one thread per tile row (= tensor-memory lane): causal
-//                       mask, running max (rescaling O in tensor memory only when the max
-//                       grows by more than 2^8), P_j as bf16 pairs written over S_j;
-//                       finally O / l to `out` and the log-sum-exp to `lse_out`.
+// One CTA per (pair of 128-row query tiles, kv head, sequence), one CTA per SM. A tile row
+// is a (new token, query head of the kv head's group) pair, so one key/value tile serves
+// the whole group, and both query tiles of the CTA share it: each K/V tile crosses L2 once
+// per 256 rows. Keys are taken 128 at a time:
+//   warp 9              TMA: both Q tiles once; K and V of key tile j into their own rings,
+//                       one (block, 64-channel half) box per lane straight from the paged
+//                       pool, block ids read one tile ahead; a K stage is refilled once its
+//                       S products are done, a V stage once its P V products are done;
+//   warp 8 (one lane)   tcgen05.mma, ping-pong over the two query tiles: O_0 += P_0(j) V_j,
+//                       S_0(j+1) = Q_0 K_{j+1}^T, then the same for tile 1. Each query tile
+//                       has one S buffer in tensor memory; P_x(j) is written over S_x(j) and
+//                       read by the P V product before S_x(j+1) overwrites it (products run
+//                       in issue order). While one tile is in softmax, the tensor core runs
+//                       the other tile's products;
+//   warps 0-3 / 4-7     softmax of query tile 0 / 1, one thread per row (= tensor-memory
+//                       lane): causal mask, running max (rescaling O in tensor memory only
+//                       when the max grows by more than 2^8), P as bf16 pairs written over
+//                       S; finally O / l to `out` and the log-sum-exp to `lse_out`.
 // Operands in shared memory use the 128-byte-swizzled layouts the tensor core reads: Q and
 // K K-major (rows of 64 channels, 128 B), V MN-major (rows of keys).
 // Every wait is bounded; a CTA that gives up flags PA_DEVERR_TIMEOUT, lets its issued
@@ -41,32 +43,50 @@ using tc::mbar_init;
 using tc::mbar_wait;
 using tc::smem_u32;
 
-constexpr int kBM = 128;                  // tile rows: (new token, head) pairs
-constexpr int kBN = 64;                   // keys per key tile
+constexpr int kBM = 128;                  // rows of a query tile: (new token, head) pairs
+constexpr int kQT = 2;                    // query tiles per CTA, sharing every key tile
+constexpr int kBN = 128;                  // keys per key tile
 constexpr int kD = 128;                   // head dimension
-constexpr int kThreads = 192;             // warps 0-3 softmax, 4 MMA, 5 TMA
-constexpr int kMmaWarp = 4, kTmaWarp = 5;
+constexpr int kThreads = 320;             // warps 0-7 softmax (two warpgroups), 8 MMA, 9 TMA
+constexpr int kMmaWarp = 8, kTmaWarp = 9;
 constexpr int kQSlab = kBM * 128;         // 64 channels (128 B) x 128 rows
-constexpr int kQBytes = 2 * kQSlab;
-constexpr int kKVSlab = kBN * 128;        // 64 channels x 64 keys
+constexpr int kQBytes = 2 * kQSlab;       // one query tile
+constexpr int kKVSlab = kBN * 128;        // 64 channels x 128 keys
 constexpr int kKVBytes = 2 * kKVSlab;
-constexpr int kKSt = 2, kVSt = 2;         // ring depths
+#ifndef PA_PF_KSTAGES
+#define PA_PF_KSTAGES 2
+#endif
+#ifndef PA_PF_VSTAGES
+#define PA_PF_VSTAGES 2
+#endif
+constexpr int kKSt = PA_PF_KSTAGES, kVSt = PA_PF_VSTAGES;  // ring depths
 constexpr int kOffQ = 0;
-constexpr int kOffK = kOffQ + kQBytes;
+constexpr int kOffK = kOffQ + kQT * kQBytes;
 constexpr int kOffV = kOffK + kKSt * kKVBytes;
 constexpr int kOffBar = kOffV + kVSt * kKVBytes;
 constexpr int kSmem = kOffBar + 256 + 1024;  // + barriers, + alignment slack
-constexpr uint32_t kTmemCols = 256;       // S / P buffers at columns 0 and 64, O at 128
-constexpr uint32_t kOCol = 128;
+constexpr uint32_t kTileCols = 256;       // tensor memory of a query tile: S (P over its
+constexpr uint32_t kOCol = 128;           // first 64 columns) at column 0, O at 128
+constexpr uint32_t kTmemCols = kQT * kTileCols;
 
-// barrier indices; the P V products complete on a ring of four barriers, so the softmax
-// waits for one only when it rescales O (no phase of a barrier is ever two ahead of it)
+// barrier indices; the P V products of a query tile complete on a ring of four barriers,
+// so its softmax waits for one only when it rescales O (no phase of a barrier is ever two
+// ahead of its waiter)
 constexpr int kORing = 4;
-enum { kBarQ = 0, kBarKF = 1, kBarKE = 3, kBarVF = 5, kBarVE = 7, kBarSF = 9, kBarP = 11,
-       kBarO = 12, kBarFin = 12 + kORing, kNumBars = 13 + kORing };
+constexpr int kBarQ = 0;
+constexpr int kBarKF = 1;
+constexpr int kBarKE = kBarKF + kKSt;
+constexpr int kBarVF = kBarKE + kKSt;
+constexpr int kBarVE = kBarVF + kVSt;
+constexpr int kBarSF = kBarVE + kVSt;      // [query tile]
+constexpr int kBarP = kBarSF + kQT;        // [query tile], kBM arrivals
+constexpr int kBarO = kBarP + kQT;         // [query tile][ring]
+constexpr int kBarFin = kBarO + kQT * kORing;
+constexpr int kNumBars = kBarFin + 1;
+static_assert(kNumBars * 8 + 8 <= 256, "barrier area");
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
-// S = Q K^T: A and B K-major, N = 64 keys. O += P V: A (P) from tensor memory, B (V)
+// S = Q K^T: A and B K-major, N = 128 keys. O += P V: A (P) from tensor memory, B (V)
 // MN-major, N = 128 channels.
 constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
                              ((uint32_t)(kBM >> 4) << 24);
@@ -171,6 +191,17 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
                  "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
                : "memory");
 }
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {"
+               "%1, %2, %3, %4, %5, %6, %7, %8,"
+               "%9, %10, %11, %12, %13, %14, %15, %16};"
+               :: "r"(taddr),
+                 "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]),
+                 "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+                 "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]),
+                 "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+               : "memory");
+}
 // tcgen05.wait::ld that also "rewrites" the loaded registers, so no use of them can be
 // scheduled before the wait.
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
@@ -215,7 +246,7 @@ __device__ __forceinline__ bool seq_rows(const PrefillArgs& a, int s, int& q0, i
 }
 
 template <int BS>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap) {
@@ -225,18 +256,24 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int G = a.group, TM = kBM / G;  // new tokens per tile
+  const int G = a.group, TM = kBM / G;  // new tokens per query tile
   const int s = blockIdx.z, kvh = blockIdx.y;
-  const int qt = (int)gridDim.x - 1 - (int)blockIdx.x;  // longest tiles (most keys) first
+  const int qp = (int)gridDim.x - 1 - (int)blockIdx.x;  // longest pairs (most keys) first
 
   int q0, n, ctx;
-  if (!seq_rows(a, s, q0, n, ctx) || qt * TM >= n) return;  // before any set-up
+  if (!seq_rows(a, s, q0, n, ctx) || 2 * qp * TM >= n) return;  // before any set-up
   const int pos0 = ctx - n;                     // position of the sequence's first new token
-  const int tok0 = qt * TM;                     // first new token of the tile
-  const int ntok = min(TM, n - tok0);           // new tokens in the tile
-  const int pos_min = pos0 + tok0;              // smallest position of a tile row
-  const int kv_end = pos_min + ntok;            // keys 0 .. kv_end-1 are seen by some row
-  const int ntiles = (kv_end + kBN - 1) / kBN;
+  // query tiles 2qp and 2qp+1 of the sequence's new tokens; the second may be empty
+  int tok0[kQT], ntok[kQT], pos_min[kQT], ntl[kQT];
+#pragma unroll
+  for (int x = 0; x < kQT; ++x) {
+    tok0[x] = (2 * qp + x) * TM;
+    ntok[x] = max(0, min(TM, n - tok0[x]));
+    pos_min[x] = pos0 + tok0[x];
+    ntl[x] = ntok[x] > 0 ? (pos_min[x] + ntok[x] + kBN - 1) / kBN : 0;  // key tiles it needs
+  }
+  const int kv_end = ntok[1] > 0 ? pos_min[1] + ntok[1] : pos_min[0] + ntok[0];
+  const int ntiles = max(ntl[0], ntl[1]);
 
   const uint32_t sQ = smem_u32(smem + kOffQ), sK = smem_u32(smem + kOffK);
   const uint32_t sV = smem_u32(smem + kOffV);
@@ -247,17 +284,8 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(kBarQ), 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(bar(kBarKF + i), 1);
-      mbar_init(bar(kBarKE + i), 1);
-      mbar_init(bar(kBarVF + i), 1);
-      mbar_init(bar(kBarVE + i), 1);
-      mbar_init(bar(kBarSF + i), 1);
-    }
-    mbar_init(bar(kBarP), kBM);
-    for (int i = 0; i < kORing; ++i) mbar_init(bar(kBarO + i), 1);
-    mbar_init(bar(kBarFin), 1);
+    for (int i = 0; i < kNumBars; ++i)
+      mbar_init(bar(i), i >= kBarP && i < kBarP + kQT ? kBM : 1);
     *dead = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -266,7 +294,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
-  // any block id out of range among the keys the tile sees? (then tiles are checked one by
+  // any block id out of range among the keys the CTA sees? (then tiles are checked one by
   // one; otherwise no per-tile checks)
   int bad = 0;
   for (int b = threadIdx.x; b < (kv_end + BS - 1) / BS; b += kThreads) {
@@ -279,20 +307,23 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   const uint32_t tmem = *tmem_slot;
 
   if (warp == kTmaWarp) {
-    // ---------------- producer (whole warp): Q once, then K and V tiles through their rings.
-    // Lane b < NB_T holds the physical block b of a key tile, read one tile ahead so the
-    // table load hides behind the ring waits; each lane issues one (block, half) box, so a
-    // tile's K (or V) copies leave in one warp instruction.
+    // ---------------- producer (whole warp): both Q tiles once, then K and V tiles through
+    // their rings; lane b < NB_T holds block b of a key tile (read one tile ahead), each
+    // lane issues one (block, half) box.
     if (lane == 0) {
-      mbar_arrive_tx(bar(kBarQ), kQBytes);
+      mbar_arrive_tx(bar(kBarQ), kQT * kQBytes);
       const uint64_t pol = evict_first_policy();
-      for (int h = 0; h < 2; ++h)
-        tma_load_4d(sQ + h * kQSlab, &qmap, 0, h, kvh * G, q0 + tok0, bar(kBarQ), pol);
+#pragma unroll
+      for (int x = 0; x < kQT; ++x)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          tma_load_4d(sQ + x * kQBytes + h * kQSlab, &qmap, 0, h, kvh * G, q0 + tok0[x],
+                      bar(kBarQ), pol);
     }
     auto fetch = [&](int j) {
       int p = -1;
       if (j < ntiles && lane < NB_T && j * kBN + lane * BS < kv_end) {
-        p = bt[j * (kBN / BS) + lane];
+        p = bt[j * NB_T + lane];
         if (p < 0 || p >= a.num_blocks) {
           flag_error(PA_DEVERR_BLOCK_ID);
           p = -1;
@@ -310,7 +341,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       const int p_next = fetch(j + 1);
       const uint32_t bytes =
           (uint32_t)__popc(__ballot_sync(0xffffffffu, p_cur >= 0)) * 2u * BS * 128u;
-      const int pb = __shfl_sync(0xffffffffu, p_cur, (lane >> 1) & 31);  // lane's block
+      const int pb = __shfl_sync(0xffffffffu, p_cur, (lane >> 1) & 31);
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int nst = kv ? kVSt : kKSt;
@@ -343,7 +374,6 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       p_cur = p_next;
     }
     if (lane == 0 && *dead) {
-      // copies still in flight complete before the CTA's shared memory is released
       for (int i = 0; i < kKSt; ++i)
         if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
       for (int i = 0; i < kVSt; ++i)
@@ -354,48 +384,63 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   } else if (warp == kMmaWarp) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      auto issue_s = [&](int j) {
+      // S_x(j) = Q_x K_j^T into S buffer j % 2 of query tile x
+      auto issue_s = [&](int x, int j) {
         const uint32_t kst = sK + (j % kKSt) * kKVBytes;
-        const uint32_t d = tmem + (uint32_t)((j & 1) * kBN);
+        const uint32_t qx = sQ + x * kQBytes;
+        const uint32_t d = tmem + x * kTileCols;  // one S buffer per query tile
 #pragma unroll
         for (int kk = 0; kk < kD / 16; ++kk) {
           const uint32_t oq = (kk >> 2) * kQSlab + (kk & 3) * 32;
           const uint32_t ok_ = (kk >> 2) * kKVSlab + (kk & 3) * 32;
-          umma_bf16(d, sdesc(sQ + oq, 16, 1024), sdesc(kst + ok_, 16, 1024), kIdescS, kk > 0);
+          umma_bf16(d, sdesc(qx + oq, 16, 1024), sdesc(kst + ok_, 16, 1024), kIdescS, kk > 0);
         }
-        umma_commit(bar(kBarSF + (j & 1)));
-        umma_commit(bar(kBarKE + (j % kKSt)));  // the K stage is free once S_j is done
+        umma_commit(bar(kBarSF + x));
       };
-      auto issue_pv = [&](int j) {
+      // O_x += P_x(j) V_j, P_x(j) over S_x(j) in tensor memory
+      auto issue_pv = [&](int x, int j) {
         const uint32_t vst = sV + (j % kVSt) * kKVBytes;
-        const uint32_t pa_ = tmem + (uint32_t)((j & 1) * kBN);  // P_j over S_j
+        const uint32_t px = tmem + x * kTileCols;  // P_x(j) over S_x(j)
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          umma_bf16_ts(tmem + kOCol, pa_ + kk * 8, sdesc(vst + kk * 16 * 128, kKVSlab, 1024),
-                       kIdescPV, (j > 0 || kk > 0));
-        umma_commit(bar(kBarO + j % kORing));
-        umma_commit(bar(kBarVE + (j % kVSt)));
+          umma_bf16_ts(tmem + x * kTileCols + kOCol, px + kk * 8,
+                       sdesc(vst + kk * 16 * 128, kKVSlab, 1024), kIdescPV, (j > 0 || kk > 0));
+        umma_commit(bar(kBarO + x * kORing + j % kORing));
       };
       bool live = mbar_wait(bar(kBarQ), 0) && mbar_wait(bar(kBarKF), 0);
       if (live) {
         tc_fence_after();
-        issue_s(0);
+        for (int x = 0; x < kQT; ++x)
+          if (ntl[x] > 0) issue_s(x, 0);
+        umma_commit(bar(kBarKE));  // the K stage is free once the S products are done
       }
+      // per key tile: P V of query tile 0, then its next S (the S buffer holds P until the
+      // P V product has read it: products run in issue order), then the same for tile 1
       for (int j = 0; live && j < ntiles; ++j) {
-        if (j + 1 < ntiles) {
-          if (!mbar_wait(bar(kBarKF + ((j + 1) % kKSt)), ((j + 1) / kKSt) & 1)) {
-            live = false;
-            break;
-          }
-          issue_s(j + 1);
-        }
-        if (!mbar_wait(bar(kBarP), j & 1) ||
-            !mbar_wait(bar(kBarVF + (j % kVSt)), (j / kVSt) & 1)) {
+        if (!mbar_wait(bar(kBarVF + (j % kVSt)), (j / kVSt) & 1)) {
           live = false;
           break;
         }
-        tc_fence_after();
-        issue_pv(j);
+        bool kready = false;
+        for (int x = 0; x < kQT && live; ++x) {
+          if (j >= ntl[x]) continue;
+          if (!mbar_wait(bar(kBarP + x), j & 1)) {
+            live = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(x, j);
+          if (j + 1 < ntl[x]) {
+            if (!kready && !mbar_wait(bar(kBarKF + ((j + 1) % kKSt)), ((j + 1) / kKSt) & 1)) {
+              live = false;
+              break;
+            }
+            kready = true;
+            issue_s(x, j + 1);
+          }
+        }
+        if (kready) umma_commit(bar(kBarKE + ((j + 1) % kKSt)));
+        umma_commit(bar(kBarVE + (j % kVSt)));
         if (*dead) live = false;
       }
       if (!live) {
@@ -408,12 +453,16 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     }
     __syncwarp();
   } else {
-    // ---------------- softmax: thread r owns tile row r (tensor-memory lane r) ----------------
-    const int r = threadIdx.x;
+    // ------- softmax: warpgroup x owns query tile x, thread r its row r (tensor-memory lane r) -------
+    const int x = warp >> 2;
+    const int r = threadIdx.x & (kBM - 1);
     const int tr = r / G, g = r - tr * G;
-    const bool row_valid = tr < ntok;
-    const int prow = pos_min + min(tr, ntok - 1);       // this row's position
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int nt = ntl[x];
+    const int pmin = pos_min[x];
+    const bool row_valid = tr < ntok[x];
+    const int prow = pmin + min(tr, max(ntok[x], 1) - 1);   // this row's position
+    const int vend = pmin + ntok[x];                          // keys this tile sees
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + x * kTileCols;
     const float sl2 = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;                  // log2-domain reference max, sum
     bool ok = true;
@@ -422,11 +471,11 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       const bool w = !*dead && mbar_wait(b, parity);
       return __all_sync(0xffffffffu, w);
     };
-    for (int j = 0; j < ntiles; ++j) {
-      if (!wait_all(bar(kBarSF + (j & 1)), (j >> 1) & 1)) { ok = false; break; }
+    for (int j = 0; j < nt; ++j) {
+      if (!wait_all(bar(kBarSF + x), j & 1)) { ok = false; break; }
       tc_fence_after();
       const int t0 = j * kBN;
-      const int vlim = min(kBN, kv_end - t0);             // keys of the tile that exist
+      const int vlim = min(kBN, kv_end - t0);             // keys of the tile that were loaded
       uint32_t badm = 0;  // blocks of the tile with an out-of-range id (skipped, masked)
       if (any_bad) {
         bool b = false;
@@ -436,17 +485,18 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
         }
         badm = __ballot_sync(0xffffffffu, b);
       }
-      const uint32_t sbuf = lane_addr + (uint32_t)((j & 1) * kBN);
-      uint32_t sv[2][32];
-      tmem_ld32(sbuf, sv[0]);
-      tmem_ld32(sbuf + 32, sv[1]);
-      tmem_wait_ld(sv[0]);
-      tmem_wait_ld(sv[1]);
+      const uint32_t sbuf = lane_addr;  // the query tile's S buffer
+      uint32_t sv[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + c * 32, sv[c]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
       // causal / existence / bad-block mask, then the row max of the raw scores
-      if (t0 + kBN - 1 > pos_min || badm != 0) {  // uniform in the CTA
+      const bool masked = t0 + kBN - 1 > pmin || badm != 0;  // uniform in the warpgroup
+      if (masked) {
         const int lim = prow - t0;                   // visible: key <= lim
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int col = c * 32 + e;
@@ -457,7 +507,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
 #pragma unroll
       for (int k = 0; k < 8; ++k) mx8[k] = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sv[c][e]));
 #pragma unroll
@@ -473,64 +523,66 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       float rs8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
-      uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 2; ++c)
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][e]), sl2, mneg));
           const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][e + 1]), sl2, mneg));
           rs8[e & 7] += p0;
           rs8[(e + 1) & 7] += p1;
-          pk[(c * 32 + e) >> 1] = pack_bf16x2(p0, p1);
+          pk[e >> 1] = pack_bf16x2(p0, p1);
         }
+        tmem_st16(sbuf + c * 16, pk);  // P over the first 64 columns of S
+      }
 #pragma unroll
       for (int k = 0; k < 4; ++k) rs8[k] += rs8[k + 4];
       l = l * alpha + ((rs8[0] + rs8[1]) + (rs8[2] + rs8[3]));
-      tmem_st32(sbuf, pk);  // P_j over the first 32 columns of S_j
       tmem_wait_st();
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O holds P_{j-1} V_{j-1} once the previous product is done: rescale it
-        if (!wait_all(bar(kBarO + (j - 1) % kORing), ((j - 1) / kORing) & 1)) {
+        // O holds P(j-1) V(j-1) once the previous product is done: rescale it
+        if (!wait_all(bar(kBarO + x * kORing + (j - 1) % kORing), ((j - 1) / kORing) & 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        {
 #pragma unroll 1
-          for (int c = 0; c < 4; ++c) {
-            uint32_t o[32];
-            tmem_ld32(lane_addr + kOCol + c * 32, o);
-            tmem_wait_ld(o);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t o[32];
+          tmem_ld32(lane_addr + kOCol + c * 32, o);
+          tmem_wait_ld(o);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(lane_addr + kOCol + c * 32, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(lane_addr + kOCol + c * 32, o);
         }
+        tmem_wait_st();
       }
       // rows of V past the keys that exist or in a skipped block may hold anything (NaN):
-      // zero them before the product reads them
+      // zero them before the products read them (both warpgroups zero the same rows)
       if (vlim < kBN || badm != 0) {
         if (!wait_all(bar(kBarVF + (j % kVSt)), (j / kVSt) & 1)) { ok = false; break; }
-        const int vr = r >> 1, h = r & 1;  // 128 threads: 64 rows x 2 channel halves
-        if (vr >= vlim || ((badm >> (vr / BS)) & 1u)) {
-          const uint32_t vrow = sV + (j % kVSt) * kKVBytes + h * kKVSlab + vr * 128;
+        if (r >= vlim || ((badm >> (r / BS)) & 1u)) {
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + k * 16), "r"(0)
-                         : "memory");
+          for (int h = 0; h < 2; ++h) {
+            const uint32_t vrow = sV + (j % kVSt) * kKVBytes + h * kKVSlab + r * 128;
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+              asm volatile("st.shared.v4.b32 [%0], {%1, %1, %1, %1};" ::"r"(vrow + k * 16), "r"(0)
+                           : "memory");
+          }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       }
       tc_fence_before();
-      mbar_arrive(bar(kBarP));
+      mbar_arrive(bar(kBarP + x));
     }
-    if (ok) ok = wait_all(bar(kBarO + (ntiles - 1) % kORing), ((ntiles - 1) / kORing) & 1);
-    if (ok) {
+    if (ok && nt > 0)
+      ok = wait_all(bar(kBarO + x * kORing + (nt - 1) % kORing), ((nt - 1) / kORing) & 1);
+    if (ok && nt > 0) {
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t orow = (int64_t)(q0 + tok0 + tr) * a.num_q_heads + kvh * G + g;
+      const int64_t orow = (int64_t)(q0 + tok0[x] + tr) * a.num_q_heads + kvh * G + g;
       uint16_t* op = static_cast<uint16_t*>(a.out) + orow * kD;
 #pragma unroll 1
       for (int c = 0; c < 4; ++c) {
@@ -551,7 +603,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       }
       if (row_valid && a.lse_out != nullptr)
         a.lse_out[orow] = l > 0.f ? (m_used + __log2f(l)) * kLn2 : -INFINITY;
-    } else {
+    } else if (!ok) {
       if (lane == 0) flag_error(PA_DEVERR_TIMEOUT);
       *dead = 1;
     }
@@ -615,7 +667,7 @@ inline cudaError_t launch_bs(const PrefillArgs& a, const void* q, const void* kc
     attr = true;
   }
   const int tiles = (a.max_query_len * a.group + kBM - 1) / kBM;
-  const dim3 grid(tiles, a.num_kv_heads, a.num_seqs);
+  const dim3 grid((tiles + kQT - 1) / kQT, a.num_kv_heads, a.num_seqs);
   prefill_tc_kernel<BS><<<grid, kThreads, kSmem, st>>>(a, qm, km, vm);
   return cudaGetLastError();
 }
