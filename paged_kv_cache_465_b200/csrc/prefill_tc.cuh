@@ -461,7 +461,6 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     const int pmin = pos_min[x];
     const bool row_valid = tr < ntok[x];
     const int prow = pmin + min(tr, max(ntok[x], 1) - 1);   // this row's position
-    const int vend = pmin + ntok[x];                          // keys this tile sees
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + x * kTileCols;
     const float sl2 = a.scale_log2;
     float m_used = -INFINITY, l = 0.f;                  // log2-domain reference max, sum
