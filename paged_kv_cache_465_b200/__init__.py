@@ -186,8 +186,9 @@ def paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale: fl
                       stream=None):
     """out[s, h] = softmax(scale * q[s, h] K^T) V over the paged cache of sequence s.
 
-    q, out [S, Hq, d] (fp32 or bf16); k_cache/v_cache [NB, Hkv, 16, d] (fp32, bf16,
-    fp8-e4m3 as float8_e4m3fn/uint8, or int8); block_tables int32 [S, MB]; context_lens
+    q, out [S, Hq, d] (fp32 or bf16); k_cache/v_cache [NB, Hkv, B, d], B = 8, 16 or 32
+    tokens per block (fp32, bf16, fp8-e4m3 as float8_e4m3fn/uint8, or int8);
+    block_tables int32 [S, MB]; context_lens
     int32 [S]; k_scales/v_scales fp32 [NB, Hkv] for fp8 and int8; k_zeros/v_zeros int32
     [NB, Hkv] for int8; lse_out fp32 [S, Hq] or None; workspace a uint8 CUDA tensor of at
     least ``workspace_size(...)`` bytes when partition_size > 0.

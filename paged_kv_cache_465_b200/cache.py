@@ -1,8 +1,9 @@
 """PagedKVCache: one layer's block pool on the GPU plus its host block allocator.
 
-A convenience object over the C ABI: the pool tensors (K, V and, for fp8, the per-(block,
-kv head) scales) live in torch-allocated device memory, the allocator is the library's
-native one, and every device operation is one of the library's kernels.
+A convenience object over the C ABI: the pool tensors (K, V and, for fp8 / int8, the
+per-(block, kv head) scales and int8 zero points) live in torch-allocated device memory,
+the allocator is the library's native one (with automatic prefix caching), and every
+device operation (write, copy, decode, prefill) is one of the library's kernels.
 """
 from __future__ import annotations
 

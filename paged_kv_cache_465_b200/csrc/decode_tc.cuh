@@ -10,7 +10,7 @@
 //
 // Why tensor cores: per KV element the group needs G multiply-adds for q.K and G for P.V;
 // at B200's HBM rate that is ~(G+1) fp32 issue slots per element on the CUDA cores, more
-// than the SMs can issue for G >= 4. Here one 16-token block costs a warp 16 mma.sync
+// than the SMs can issue for G >= 4. Here one 16-token sub-tile costs a warp 16 mma.sync
 // (m16n8k16) instead: S^T = K . Q^T (M = 16 tokens, N = 8 query heads, K = 128 channels)
 // and O^T += V^T . P^T (M = 16 channels x 8 tiles, N = 8 heads, K = 16 tokens). Both
 // products are skinny (N = G <= 8), so the warp-level mma fits them; the kernel stays
@@ -277,9 +277,10 @@ __device__ __forceinline__ float load_q_frags(const uint16_t* qp, int G, int lan
   return q_frags<FP8>(raw, scale_log2, qf);
 }
 
-// One 16-token block: S^T = K Q^T on the tensor cores, online softmax, O^T += V^T P^T.
-// kt / vt: shared addresses of the block's swizzled K and V tiles; nvalid: tokens of the
-// block inside the work item; zs: log2-domain score scale (x fp8 K scale); vs: fp8 V scale.
+// One 16-token sub-tile: S^T = K Q^T on the tensor cores, online softmax, O^T += V^T P^T.
+// kt / vt: shared addresses of the sub-tile's swizzled K and V tiles; nvalid: its tokens
+// inside the work item; hp: per-half score scale (log2 domain x K scale), V scale and int8
+// zero-point constants.
 // The K products run as two independent accumulation chains and the V fragments are read
 // before the softmax, so a warp has independent work in flight at every step.
 // Per-half dequantisation parameters of a 16-token sub-tile: tokens 0-7 come from one

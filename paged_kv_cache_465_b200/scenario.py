@@ -82,7 +82,7 @@ class DeviceScenario:
         self.context_lens = torch.from_numpy(lens.astype(np.int32)).to(device)
         tables_host = self.block_tables.cpu().numpy()
 
-        # ---- K/V values and fp8 scales (setup) ----
+        # ---- K/V values and fp8 / int8 quantisation parameters (setup) ----
         step_k, step_v, step_sl = [], [], []
         for s in range(S):
             k, v = self._seq_kv(s)
