@@ -1264,15 +1264,18 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dt
   return r == CUDA_SUCCESS;
 }
 
+constexpr int kMaxDevices = 64;  // per-device caches of the launch set-up
+
 inline int sm_count() {
-  static int dev_cached = -1, sms = 0;
+  static int cache[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
-  if (dev != dev_cached) {
-    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) sms = 0;
-    dev_cached = dev;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+      cache[dev] = n;
   }
-  return sms;
+  return cache[dev];
 }
 
 // Tensor-core kernel families: grid of one CTA per item, persistent CTAs sharing an item,
@@ -1288,6 +1291,26 @@ inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
   return e;
 }
 
+// Launch set-up of one kernel on the current device: its dynamic shared-memory limit is
+// raised and its resident CTAs per SM measured once per device the process uses (`slots`
+// is the kernel's per-device cache; concurrent first calls write the same values).
+template <typename K>
+inline cudaError_t resident_per_sm(K kernel, int threads, int smem, int (&slots)[kMaxDevices],
+                                   int* per_sm) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (slots[dev] == 0) {
+    int n = 0;
+    e = occupancy(kernel, threads, smem, &n);
+    if (e != cudaSuccess) return e;
+    slots[dev] = n;
+  }
+  *per_sm = slots[dev];
+  return cudaSuccess;
+}
+
 template <pa_dtype KV, int BS>
 inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,
                                 const PlanView* pl, TcKind kind, cudaStream_t st) {
@@ -1297,11 +1320,10 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   if (!make_map(&km, a.k_cache, rows, KV, BS) || !make_map(&vm, a.v_cache, rows, KV, BS))
     return cudaErrorInvalidValue;
   if (kind == kTcGrid) {
-    static int per_sm = 0;
-    if (per_sm == 0) {
-      cudaError_t e = occupancy(decode_tc_kernel<KV, BS>, kNW * 32, C::kSmem, &per_sm);
-      if (e != cudaSuccess) { per_sm = 0; return e; }
-    }
+    static int slots[kMaxDevices] = {};
+    int per_sm = 0;
+    cudaError_t e = resident_per_sm(decode_tc_kernel<KV, BS>, kNW * 32, C::kSmem, slots, &per_sm);
+    if (e != cudaSuccess) return e;
     decode_tc_kernel<KV, BS><<<grid, kNW * 32, C::kSmem, st>>>(a, km, vm);
     return cudaGetLastError();
   }
@@ -1311,20 +1333,18 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   if (e != cudaSuccess) return e;
   if (kind == kTcCta) {
     if constexpr (BS != kSub) return cudaErrorInvalidValue;
-    static int per_sm = 0;
-    if (per_sm == 0) {
-      e = occupancy(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, &per_sm);
-      if (e != cudaSuccess) { per_sm = 0; return e; }
-    }
+    static int slots[kMaxDevices] = {};
+    int per_sm = 0;
+    e = resident_per_sm(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, slots, &per_sm);
+    if (e != cudaSuccess) return e;
     e = launch_pdl(decode_tc_persistent<KV>, dim3(sms * per_sm), dim3(kNW * 32), C::kPSmem, st,
                    a, *pl, km, vm);
     if (e != cudaSuccess) return e;
   } else {
-    static int per_sm = 0;
-    if (per_sm == 0) {
-      e = occupancy(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, &per_sm);
-      if (e != cudaSuccess) { per_sm = 0; return e; }
-    }
+    static int slots[kMaxDevices] = {};
+    int per_sm = 0;
+    e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, slots, &per_sm);
+    if (e != cudaSuccess) return e;
     e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32),
                    TcwCfg<KV>::kSmem, st, a, *pl, km, vm);
     if (e != cudaSuccess) return e;

@@ -658,13 +658,10 @@ inline cudaError_t launch_bs(const PrefillArgs& a, const void* q, const void* kc
   if (!make_q_map(&qm, q, a.num_tokens, a.num_q_heads, a.group) ||
       !make_kv_map(&km, kc, rows, BS) || !make_kv_map(&vm, vc, rows, BS))
     return cudaErrorInvalidValue;
-  static bool attr = false;
-  if (!attr) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel<BS>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    attr = true;
-  }
+  static int slots[tc::kMaxDevices] = {};
+  int per_sm = 0;
+  const cudaError_t e = tc::resident_per_sm(prefill_tc_kernel<BS>, kThreads, kSmem, slots, &per_sm);
+  if (e != cudaSuccess) return e;
   const int tiles = (a.max_query_len * a.group + kBM - 1) / kBM;
   const dim3 grid((tiles + kQT - 1) / kQT, a.num_kv_heads, a.num_seqs);
   prefill_tc_kernel<BS><<<grid, kThreads, kSmem, st>>>(a, qm, km, vm);
