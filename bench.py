@@ -369,7 +369,7 @@ def _prefill_workloads(torch, flush):
     from paged_kv_cache_465_b200.scenario import PrefillScenario
     peak, kind = _bf16_peak()
     out = {}
-    for name in ("prefill", "chunked"):
+    for name in ("prefill", "chunked", "chunked_fp8"):
         draw = workloads.draw_prefill(name)
         sc = PrefillScenario(draw, draw_seqs=[])
         for _ in range(3):

@@ -155,9 +155,11 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
  *                 context_lens entry and >= max_query_len
  *   block_tables, context_lens, k/v scales and zeros, lse_out: as in paged_attn_decode
  *   desc          as in paged_attn_decode with partition_size 0
- * bf16 caches with head_dim 128 and a group of 1, 2, 4, 8 or 16 run on the tensor cores
- * (tcgen05, accumulators in tensor memory); every other supported shape, or
- * pa_set_decode_impl(1), runs one CUDA-core pass per new token. No workspace.
+ * bf16 q / out with a bf16, fp8 or int8 cache, head_dim 128 and a group of 1, 2, 4, 8 or
+ * 16 run on the tensor cores (tcgen05, accumulators in tensor memory; fp8 / int8 codes are
+ * converted exactly to bf16 in shared memory and their scales applied to the scores and
+ * to P); every other supported shape, or pa_set_decode_impl(1), runs one CUDA-core pass
+ * per new token. No workspace.
  * A sequence whose query range is inconsistent (descending, past num_tokens, more new
  * tokens than context or than max_query_len) is skipped and PA_DEVERR_QUERY recorded.
  */

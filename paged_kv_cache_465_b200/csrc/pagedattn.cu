@@ -238,13 +238,14 @@ pa_status paged_attn_prefill(const void* q, const void* k_cache, const void* v_c
     pf::PrefillArgs a;
     a.block_tables = block_tables; a.context_lens = context_lens; a.query_start = query_start;
     a.out = out; a.lse_out = lse_out;
+    a.k_scales = k_scales; a.v_scales = v_scales; a.k_zeros = k_zeros; a.v_zeros = v_zeros;
     a.scale_log2 = scale * kLog2e;
     a.num_seqs = desc->num_seqs; a.num_tokens = num_tokens;
     a.num_q_heads = desc->num_q_heads; a.num_kv_heads = desc->num_kv_heads;
     a.group = desc->num_q_heads / desc->num_kv_heads;
     a.max_blocks_per_seq = desc->max_blocks_per_seq; a.num_blocks = desc->num_blocks;
     a.max_context_len = max_context_len; a.max_query_len = max_query_len;
-    e = launch_prefill_tc(a, desc->block_size, q, k_cache, v_cache, st);
+    e = launch_prefill_tc(a, desc->block_size, desc->kv_dtype, q, k_cache, v_cache, st);
   } else {
     // CUDA-core path: every new token is one work row of the single-pass decode kernel
     DecodeArgs a;

@@ -47,8 +47,9 @@ constexpr int kBM = 128;                  // rows of a query tile: (new token, h
 constexpr int kQT = 2;                    // query tiles per CTA, sharing every key tile
 constexpr int kBN = 128;                  // keys per key tile
 constexpr int kD = 128;                   // head dimension
-constexpr int kThreads = 320;             // warps 0-7 softmax (two warpgroups), 8 MMA, 9 TMA
-constexpr int kMmaWarp = 8, kTmaWarp = 9;
+constexpr int kMmaWarp = 8, kTmaWarp = 9;  // warps 0-7 softmax (two warpgroups)
+constexpr int kConvWarp0 = 10;            // fp8 / int8 caches: warps 10-11 dequantise
+constexpr int kConvThreads = 64;
 constexpr int kQSlab = kBM * 128;         // 64 channels (128 B) x 128 rows
 constexpr int kQBytes = 2 * kQSlab;       // one query tile
 constexpr int kKVSlab = kBN * 128;        // 64 channels x 128 keys
@@ -63,8 +64,20 @@ constexpr int kKSt = PA_PF_KSTAGES, kVSt = PA_PF_VSTAGES;  // ring depths
 constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQT * kQBytes;
 constexpr int kOffV = kOffK + kKSt * kKVBytes;
-constexpr int kOffBar = kOffV + kVSt * kKVBytes;
-constexpr int kSmem = kOffBar + 256 + 1024;  // + barriers, + alignment slack
+// Shared-memory map per cache type: a quantised cache adds a staging buffer for the codes
+// of one K tile and one V tile (TMA lands them there, the converter warps write the bf16
+// stages from them) and the tile's per-block scales and zero points.
+template <bool QUANT>
+struct PfLayout {
+  static constexpr int kThreads = QUANT ? 384 : 320;
+  static constexpr int kStage8 = QUANT ? kBN * 128 : 0;         // 128 keys x 128 one-byte codes
+  static constexpr int kOffK8 = kOffV + kVSt * kKVBytes;
+  static constexpr int kOffV8 = kOffK8 + kStage8;
+  static constexpr int kOffScale = kOffV8 + kStage8;            // float [2][32], int [2][32]
+  static constexpr int kOffSide = kOffScale + (QUANT ? 512 : 0);  // float [4][2][32]
+  static constexpr int kOffBar = kOffSide + (QUANT ? 1024 : 0);
+  static constexpr int kSmem = kOffBar + 256 + 1024;            // + barriers, + alignment slack
+};
 constexpr uint32_t kTileCols = 256;       // tensor memory of a query tile: S (P over its
 constexpr uint32_t kOCol = 128;           // first 64 columns) at column 0, O at 128
 constexpr uint32_t kTmemCols = kQT * kTileCols;
@@ -82,7 +95,13 @@ constexpr int kBarSF = kBarVE + kVSt;      // [query tile]
 constexpr int kBarP = kBarSF + kQT;        // [query tile], kBM arrivals
 constexpr int kBarO = kBarP + kQT;         // [query tile][ring]
 constexpr int kBarFin = kBarO + kQT * kORing;
-constexpr int kNumBars = kBarFin + 1;
+constexpr int kBarK8F = kBarFin + 1;       // quantised: codes of the tile staged (TMA)
+constexpr int kBarK8E = kBarK8F + 1;       // quantised: staging read by the converters
+constexpr int kBarV8F = kBarK8E + 1;
+constexpr int kBarV8E = kBarV8F + 1;
+constexpr int kBarSC = kBarV8E + 1;        // quantised: [4] a tile's K / V scales for the softmax
+constexpr int kSideRing = 4;
+constexpr int kNumBars = kBarSC + kSideRing;
 static_assert(kNumBars * 8 + 8 <= 256, "barrier area");
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
@@ -106,6 +125,20 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%2, %3, %4}], [%5];"
       ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+// Two f16 (low half first) -> f32.
+__device__ __forceinline__ void f16x2_to_f32(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\tcvt.f32.f16 %0, a;\n\t"
+      "cvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi) : "r"(h));
+}
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, int x, int y,
@@ -226,6 +259,10 @@ struct PrefillArgs {
   const int32_t* query_start;   // [S + 1]
   void* out;                    // [T][Hq][128] bf16
   float* lse_out;               // [T][Hq] or null
+  const float* k_scales;        // fp8 / int8: [num_blocks][Hkv]
+  const float* v_scales;
+  const int32_t* k_zeros;       // int8: [num_blocks][Hkv]
+  const int32_t* v_zeros;
   float scale_log2;             // scale * log2(e)
   int num_seqs, num_tokens, num_q_heads, num_kv_heads, group;
   int max_blocks_per_seq, num_blocks, max_context_len, max_query_len;
@@ -245,12 +282,15 @@ __device__ __forceinline__ bool seq_rows(const PrefillArgs& a, int s, int& q0, i
   return ok;
 }
 
-template <int BS>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BS, pa_dtype KV>
+__global__ void __launch_bounds__(PfLayout<KV != PA_BF16>::kThreads, 1)
 prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
                   const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap) {
   static_assert(kBN % BS == 0 && kBN / BS <= 32, "block size");
+  constexpr bool QUANT = KV != PA_BF16;  // fp8 / int8 codes, dequantised to bf16 in smem
+  using L = PfLayout<QUANT>;
+  constexpr int kThreads = L::kThreads, kOffBar = L::kOffBar;
   constexpr int NB_T = kBN / BS;  // blocks per key tile
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -284,8 +324,15 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kNumBars; ++i)
-      mbar_init(bar(i), i >= kBarP && i < kBarP + kQT ? kBM : 1);
+    for (int i = 0; i < kNumBars; ++i) {
+      uint32_t count = 1;
+      if (i >= kBarP && i < kBarP + kQT) count = kBM;
+      // quantised: the bf16 stages are filled, and the staging read, by the converters
+      if (QUANT && ((i >= kBarKF && i < kBarKF + kKSt) || (i >= kBarVF && i < kBarVF + kVSt) ||
+                    i == kBarK8E || i == kBarV8E || (i >= kBarSC && i < kBarSC + kSideRing)))
+        count = kConvThreads;
+      mbar_init(bar(i), count);
+    }
     *dead = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -343,7 +390,34 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
           (uint32_t)__popc(__ballot_sync(0xffffffffu, p_cur >= 0)) * 2u * BS * 128u;
       const int pb = __shfl_sync(0xffffffffu, p_cur, (lane >> 1) & 31);
 #pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
+      for (int kv = 0; kv < 2 && QUANT; ++kv) {
+        // quantised: the tile's codes go to the staging buffer once the converters have
+        // read the previous tile, with the blocks' scales (and zero points) beside them
+        bool w = true;
+        if (lane == 0 && j >= 1) w = mbar_wait(bar(kv ? kBarV8E : kBarK8E), (j - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
+        }
+        if (lane < NB_T) {
+          float* sc = reinterpret_cast<float*>(smem + L::kOffScale) + kv * 32;
+          int* zp = reinterpret_cast<int*>(smem + L::kOffScale + 256) + kv * 32;
+          const int64_t bh = (int64_t)(p_cur >= 0 ? p_cur : 0) * a.num_kv_heads + kvh;
+          sc[lane] = p_cur >= 0 ? (kv ? a.v_scales : a.k_scales)[bh] : 1.f;  // absent: masked
+          zp[lane] = (KV == PA_INT8 && p_cur >= 0) ? (kv ? a.v_zeros : a.k_zeros)[bh] : 0;
+        }
+        __syncwarp();
+        const uint32_t fb = bar(kv ? kBarV8F : kBarK8F);
+        if (lane == 0) mbar_arrive_tx(fb, bytes / 2);  // one byte per element
+        __syncwarp();
+        if (lane < NB_T && p_cur >= 0)
+          tma_load_2d(smem_u32(smem + (kv ? L::kOffV8 : L::kOffK8)) + lane * BS * 128,
+                      kv ? &vmap : &kmap, 0, (p_cur * a.num_kv_heads + kvh) * BS, fb);
+        if (kv) last_v[0] = j;
+        else last_k[0] = j;
+      }
+#pragma unroll
+      for (int kv = 0; kv < 2 && !QUANT; ++kv) {
         const int nst = kv ? kVSt : kKSt;
         const int st = j % nst;
         bool w = true;
@@ -374,10 +448,16 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       p_cur = p_next;
     }
     if (lane == 0 && *dead) {
-      for (int i = 0; i < kKSt; ++i)
-        if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
-      for (int i = 0; i < kVSt; ++i)
-        if (last_v[i] >= 0) mbar_wait(bar(kBarVF + i), (last_v[i] / kVSt) & 1);
+      // copies still in flight complete before the CTA's shared memory is released
+      if (QUANT) {
+        if (last_k[0] >= 0) mbar_wait(bar(kBarK8F), last_k[0] & 1);
+        if (last_v[0] >= 0) mbar_wait(bar(kBarV8F), last_v[0] & 1);
+      } else {
+        for (int i = 0; i < kKSt; ++i)
+          if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
+        for (int i = 0; i < kVSt; ++i)
+          if (last_v[i] >= 0) mbar_wait(bar(kBarVF + i), (last_v[i] / kVSt) & 1);
+      }
       mbar_wait(bar(kBarQ), 0);
     }
     __syncwarp();
@@ -452,6 +532,78 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       mbar_wait(bar(kBarFin), 0);
     }
     __syncwarp();
+  } else if (QUANT && warp >= kConvWarp0) {
+    // ---------------- converters (quantised caches): staged codes -> bf16 stages ----------------
+    // Thread ct takes 16 chunks of 16 codes: chunk = ct + 64 it, key row t = chunk / 8,
+    // channels 16 (chunk % 8) ..; value = the E4M3 code's value (fp8) or code - zero (int8)
+    // of the key's block, exact in bf16, stored in the 128-byte-swizzled K-major (K) /
+    // MN-major (V) layout the products read, exactly where TMA would put bf16. The blocks'
+    // scales go to the softmax through a ring of four slots (K scale on the scores, V
+    // scale on P), so the dequantisation adds no rounding.
+    const int ct = threadIdx.x - kConvWarp0 * 32;
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+#pragma unroll 1
+      for (int kv = 0; kv < 2; ++kv) {
+        const int nst = kv ? kVSt : kKSt;
+        const int st = j % nst;
+        bool w = !*dead && mbar_wait(bar(kv ? kBarV8F : kBarK8F), j & 1);
+        if (w && j >= nst) w = mbar_wait(bar((kv ? kBarVE : kBarKE) + st), ((j / nst) - 1) & 1);
+        if (!w) {
+          ok = false;
+          break;
+        }
+        const uint8_t* src = smem + (kv ? L::kOffV8 : L::kOffK8);
+        const float* sc = reinterpret_cast<const float*>(smem + L::kOffScale) + kv * 32;
+        const int* zp = reinterpret_cast<const int*>(smem + L::kOffScale + 256) + kv * 32;
+        const uint32_t dst = (kv ? sV : sK) + st * kKVBytes;
+#pragma unroll 4
+        for (int it = 0; it < kBN * 8 / kConvThreads; ++it) {
+          const int chunk = ct + kConvThreads * it;
+          const int t = chunk >> 3, q8 = chunk & 7;
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + t * 128 + q8 * 16);
+          const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float f[4];
+            if constexpr (KV == PA_INT8) {
+              const float z = (float)zp[t / BS];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) f[e] = (float)(int8_t)(wd[k] >> (8 * e)) - z;
+            } else {  // E4M3 -> f16 -> f32, both exact
+              f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] & 0xffffu)), f[0], f[1]);
+              f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] >> 16)), f[2], f[3]);
+            }
+            o[2 * k] = pack_bf16x2(f[0], f[1]);
+            o[2 * k + 1] = pack_bf16x2(f[2], f[3]);
+          }
+          // channels 16 q8 .. 16 q8 + 15: half q8 / 4 of the channels, 16-byte chunks
+          // 2 (q8 % 4) and 2 (q8 % 4) + 1 of the key's 128-byte row, swizzled by row % 8
+          const uint32_t row = dst + (q8 >> 2) * kKVSlab + t * 128;
+          const int c0 = 2 * (q8 & 3);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(row + ((c0 ^ (t & 7)) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                         "r"(o[3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(row + (((c0 + 1) ^ (t & 7)) << 4)), "r"(o[4]), "r"(o[5]), "r"(o[6]),
+                         "r"(o[7]) : "memory");
+        }
+        // the tile's block scales for the softmax (slot j % 4 is free: the softmax of tile
+        // j - 4 finished before the S products of tile j - 2, which freed this stage)
+        if (ct < NB_T)
+          reinterpret_cast<float*>(smem + L::kOffSide)[((j % kSideRing) * 2 + kv) * 32 + ct] =
+              sc[ct];
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(bar(kv ? kBarV8E : kBarK8E));           // staging read
+        mbar_arrive(bar((kv ? kBarVF : kBarKF) + st));       // bf16 stage written
+      }
+      if (ok) mbar_arrive(bar(kBarSC + j % kSideRing));     // K and V scales of tile j
+    }
+    if (!ok) {
+      flag_error(PA_DEVERR_TIMEOUT);
+      *dead = 1;
+    }
   } else {
     // ------- softmax: warpgroup x owns query tile x, thread r its row r (tensor-memory lane r) -------
     const int x = warp >> 2;
@@ -472,6 +624,10 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     };
     for (int j = 0; j < nt; ++j) {
       if (!wait_all(bar(kBarSF + x), j & 1)) { ok = false; break; }
+      if (QUANT && !wait_all(bar(kBarSC + j % kSideRing), (j / kSideRing) & 1)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const int t0 = j * kBN;
       const int vlim = min(kBN, kv_end - t0);             // keys of the tile that were loaded
@@ -490,6 +646,22 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       for (int c = 0; c < 4; ++c) tmem_ld32(sbuf + c * 32, sv[c]);
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_wait_ld(sv[c]);
+      // quantised caches: the scores of key block b carry its K scale (the products ran on
+      // the codes' exact values); scale them into the log2 domain before the mask, so that
+      // masked keys are -inf whatever their block's scale
+      const float* side = reinterpret_cast<const float*>(smem + L::kOffSide) +
+                          (j % kSideRing) * 2 * 32;  // [K scales][V scales] of tile j
+      if constexpr (QUANT) {
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+#pragma unroll
+          for (int b = 0; b < 32 / BS; ++b) {
+            const float ks = side[(c * 32) / BS + b] * sl2;
+#pragma unroll
+            for (int e = b * BS; e < (b + 1) * BS; ++e)
+              sv[c][e] = __float_as_uint(__uint_as_float(sv[c][e]) * ks);
+          }
+      }
       // causal / existence / bad-block mask, then the row max of the raw scores
       const bool masked = t0 + kBN - 1 > pmin || badm != 0;  // uniform in the warpgroup
       if (masked) {
@@ -511,7 +683,8 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
         for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sv[c][e]));
 #pragma unroll
       for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
-      const float mx = fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * sl2;
+      const float mx =
+          fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])) * (QUANT ? 1.f : sl2);
       const float m_new = fmaxf(m_used, mx);
       float alpha = 1.f;
       if (m_new > m_used + 8.f) {  // lazy rescale: P stays below 2^8 otherwise
@@ -522,16 +695,22 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       float rs8[8];
 #pragma unroll
       for (int k = 0; k < 8; ++k) rs8[k] = 0.f;
+      const float xs = QUANT ? 1.f : sl2;  // quantised: scores already scaled above
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][e]), sl2, mneg));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][e + 1]), sl2, mneg));
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][e]), xs, mneg));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][e + 1]), xs, mneg));
           rs8[e & 7] += p0;
           rs8[(e + 1) & 7] += p1;
-          pk[e >> 1] = pack_bf16x2(p0, p1);
+          if constexpr (QUANT) {  // P carries the V scale of its key's block
+            const float vs = side[32 + (c * 32 + e) / BS];
+            pk[e >> 1] = pack_bf16x2(p0 * vs, p1 * vs);
+          } else {
+            pk[e >> 1] = pack_bf16x2(p0, p1);
+          }
         }
         tmem_st16(sbuf + c * 16, pk);  // P over the first 64 columns of S
       }
@@ -650,42 +829,70 @@ inline bool make_kv_map(CUtensorMap* m, const void* pool, int64_t token_rows, in
          CUDA_SUCCESS;
 }
 
-template <int BS>
+// A one-byte-code pool (fp8 / int8) [NB][Hkv][BS][128] as rows of 128 bytes; a box is one
+// block's tokens, landing unswizzled in the staging buffer.
+inline bool make_kv8_map(CUtensorMap* m, const void* pool, int64_t token_rows, int bs) {
+  auto enc = tc::encoder();
+  if (enc == nullptr) return false;
+  cuuint64_t dims[2] = {128, (cuuint64_t)token_rows};
+  cuuint64_t strides[1] = {128};
+  cuuint32_t box[2] = {128, (cuuint32_t)bs};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(pool), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+template <int BS, pa_dtype KV>
 inline cudaError_t launch_bs(const PrefillArgs& a, const void* q, const void* kc, const void* vc,
                              cudaStream_t st) {
+  using L = PfLayout<KV != PA_BF16>;
   CUtensorMap qm, km, vm;
   const int64_t rows = (int64_t)a.num_blocks * a.num_kv_heads * BS;
-  if (!make_q_map(&qm, q, a.num_tokens, a.num_q_heads, a.group) ||
-      !make_kv_map(&km, kc, rows, BS) || !make_kv_map(&vm, vc, rows, BS))
+  const bool maps = KV == PA_BF16
+                        ? make_kv_map(&km, kc, rows, BS) && make_kv_map(&vm, vc, rows, BS)
+                        : make_kv8_map(&km, kc, rows, BS) && make_kv8_map(&vm, vc, rows, BS);
+  if (!maps || !make_q_map(&qm, q, a.num_tokens, a.num_q_heads, a.group))
     return cudaErrorInvalidValue;
   static int slots[tc::kMaxDevices] = {};
   int per_sm = 0;
-  const cudaError_t e = tc::resident_per_sm(prefill_tc_kernel<BS>, kThreads, kSmem, slots, &per_sm);
+  const cudaError_t e =
+      tc::resident_per_sm(prefill_tc_kernel<BS, KV>, L::kThreads, L::kSmem, slots, &per_sm);
   if (e != cudaSuccess) return e;
   const int tiles = (a.max_query_len * a.group + kBM - 1) / kBM;
   const dim3 grid((tiles + kQT - 1) / kQT, a.num_kv_heads, a.num_seqs);
-  prefill_tc_kernel<BS><<<grid, kThreads, kSmem, st>>>(a, qm, km, vm);
+  prefill_tc_kernel<BS, KV><<<grid, L::kThreads, L::kSmem, st>>>(a, qm, km, vm);
   return cudaGetLastError();
 }
 
 }  // namespace pf
 
-// Shapes the tensor-core prefill kernel takes: bf16 everywhere, head_dim 128, a group that
-// divides the 128 tile rows, blocks of 8, 16 or 32 tokens.
+// Shapes the tensor-core prefill kernel takes: bf16 q / out, a bf16, fp8 or int8 cache,
+// head_dim 128, a group that divides the 128 tile rows, blocks of 8, 16 or 32 tokens.
 inline bool prefill_tc_supported(const pa_decode_desc* d) {
   const int G = d->num_q_heads / d->num_kv_heads;
-  if (d->kv_dtype != PA_BF16 || d->q_dtype != PA_BF16 || d->out_dtype != PA_BF16) return false;
+  if (d->q_dtype != PA_BF16 || d->out_dtype != PA_BF16) return false;
+  if (d->kv_dtype != PA_BF16 && d->kv_dtype != PA_FP8_E4M3 && d->kv_dtype != PA_INT8)
+    return false;
   if (d->head_dim != pf::kD) return false;
   if (G != 1 && G != 2 && G != 4 && G != 8 && G != 16) return false;
   if (d->block_size != 8 && d->block_size != 16 && d->block_size != 32) return false;
   return (int64_t)d->num_blocks * d->num_kv_heads * d->block_size < ((int64_t)1 << 31);
 }
 
-inline cudaError_t launch_prefill_tc(const pf::PrefillArgs& a, int block_size, const void* q,
-                                     const void* kc, const void* vc, cudaStream_t st) {
-  if (block_size == 8) return pf::launch_bs<8>(a, q, kc, vc, st);
-  if (block_size == 32) return pf::launch_bs<32>(a, q, kc, vc, st);
-  return pf::launch_bs<16>(a, q, kc, vc, st);
+inline cudaError_t launch_prefill_tc(const pf::PrefillArgs& a, int block_size, pa_dtype kv,
+                                     const void* q, const void* kc, const void* vc,
+                                     cudaStream_t st) {
+  auto by_bs = [&](auto kvc) -> cudaError_t {
+    constexpr pa_dtype KV = decltype(kvc)::value;
+    if (block_size == 8) return pf::launch_bs<8, KV>(a, q, kc, vc, st);
+    if (block_size == 32) return pf::launch_bs<32, KV>(a, q, kc, vc, st);
+    return pf::launch_bs<16, KV>(a, q, kc, vc, st);
+  };
+  if (kv == PA_FP8_E4M3) return by_bs(std::integral_constant<pa_dtype, PA_FP8_E4M3>{});
+  if (kv == PA_INT8) return by_bs(std::integral_constant<pa_dtype, PA_INT8>{});
+  return by_bs(std::integral_constant<pa_dtype, PA_BF16>{});
 }
 
 }  // namespace pa

@@ -94,8 +94,20 @@ def test_group_sizes(pa, scen, hq, hkv):
     _run(pa, scen, workloads.draw_prefill(wl))
 
 
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("kv", ["fp8", "int8"])
+@pytest.mark.parametrize("B", [8, 16, 32])
+def test_quantised_caches(pa, scen, impl, kv, B):
+    """fp8 / int8 caches: the tensor-core kernel dequantises staged codes to bf16 in shared
+    memory (per-block scale and zero point); the CUDA-core kernel reads them directly."""
+    wl = workloads.PREFILL_WORKLOADS["chunked"].scaled(
+        num_seqs=4, kv_dtype=kv, block_size=B, num_blocks=16384 // B,
+        lens=("fixed", [1, 200, 777, 1500]), new=("chunk", 300))
+    _run(pa, scen, workloads.draw_prefill(wl), impl)
+
+
 @pytest.mark.parametrize("kv,dim", [("fp8", 128), ("int8", 128), ("bf16", 64), ("bf16", 256)])
-def test_cuda_core_dtypes_and_head_dims(pa, scen, kv, dim):
+def test_other_dtypes_and_head_dims(pa, scen, kv, dim):
     wl = workloads.PREFILL_WORKLOADS["chunked"].scaled(
         num_seqs=3, head_dim=dim, kv_dtype=kv, lens=("fixed", [40, 300, 700]),
         new=("chunk", 100), num_blocks=512)

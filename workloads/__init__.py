@@ -293,6 +293,9 @@ PREFILL_WORKLOADS: Dict[str, PrefillWorkload] = {
     # 16 sequences, 512-token chunks after cached contexts of U{512..3584}: 32q/8kv, bf16.
     "chunked": PrefillWorkload("chunked", 12, 16, 32, 8, 128, 16, 8192, "bf16", "bf16",
                                ("uniform", 1024, 4096), ("chunk", 512)),
+    # the chunked recipe over an fp8-e4m3 cache (per-(block, kv head) scales)
+    "chunked_fp8": PrefillWorkload("chunked_fp8", 12, 16, 32, 8, 128, 16, 8192, "fp8", "bf16",
+                                   ("uniform", 1024, 4096), ("chunk", 512)),
 }
 
 
