@@ -2,13 +2,15 @@
 
 Against: textbook attention written as Python loops over contiguous per-token arrays
 (never through a block table), closed forms (one token; zero query; identical keys),
-SciPy's logsumexp, invariance under the physical placement of blocks, and shared-prefix
-sequences matching private unshared copies.
+SciPy's logsumexp, invariance under the physical placement of blocks, shared-prefix
+sequences matching private unshared copies, and one-byte caches against float attention on
+values decoded independently (torch's E4M3 decoder; code minus zero point).
 """
 import math
 
 import numpy as np
 import pytest
+import torch
 from scipy.special import logsumexp
 
 import workloads
@@ -152,3 +154,50 @@ def test_fp8_dequant_is_code_times_scale(B):
         # subnormal step 2^-9 * scale
         assert np.all(err <= np.maximum(np.abs(kf[:, 2]) * 2 ** -4, 2 ** -10 * sc) + 1e-12)
     assert np.all(np.isfinite(out)) and np.all(np.isfinite(lse))
+
+
+@pytest.mark.parametrize("kv", ["fp8", "int8"])
+def test_quantised_attention_on_dequantised_values(kv):
+    """One-byte caches: the attention equals float attention over values decoded on their
+    own: fp8 codes through torch's float8_e4m3fn, int8 as (code - zero point); each times
+    its block's scale, K and V with separate scales (and zero points), gathered token by
+    token in a Python loop."""
+    rng = np.random.default_rng(21)
+    NB, H, B, dd, G = 24, 2, 16, 32, 3
+    if kv == "fp8":
+        codes = rng.integers(0, 256, (2, NB, H, B, dd)).astype(np.uint8)
+        codes[(codes & 0x7F) == 0x7F] = 0x38                   # no NaN patterns
+        kc, vc = codes
+        zk = zv = None
+        dec = torch.from_numpy(codes.copy()).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    else:
+        kc, vc = rng.integers(-128, 128, (2, NB, H, B, dd)).astype(np.int8)
+        zk = rng.integers(-30, 31, (NB, H)).astype(np.int32)
+        zv = rng.integers(-30, 31, (NB, H)).astype(np.int32)
+        dec = np.stack([kc.astype(np.int64) - zk[:, :, None, None],
+                        vc.astype(np.int64) - zv[:, :, None, None]]).astype(np.float64)
+    ks = rng.uniform(0.002, 0.02, (NB, H)).astype(np.float32)
+    vs = rng.uniform(0.5, 3.0, (NB, H)).astype(np.float32)
+    lens = np.array([1, 16, 17, 90], np.int32)
+    perm = rng.permutation(NB)
+    bt = np.full((4, 6), -1, np.int32)
+    used = 0
+    for s, n in enumerate(lens):
+        nb = -(-int(n) // B)
+        bt[s, :nb] = perm[used:used + nb]
+        used += nb
+    q = rng.standard_normal((4, H * G, dd)).astype(np.float32)
+    sc = 0.7
+    out, lse = attention.ref_decode(q, kc, vc, bt, lens, sc, H, "f32", kv, ks, vs,
+                                    k_zeros=zk, v_zeros=zv)
+    for s, n in enumerate(lens):
+        for h in range(H * G):
+            kvh = h // G
+            K = np.array([dec[0, bt[s, t // B], kvh, t % B] * float(ks[bt[s, t // B], kvh])
+                          for t in range(n)])
+            V = np.array([dec[1, bt[s, t // B], kvh, t % B] * float(vs[bt[s, t // B], kvh])
+                          for t in range(n)])
+            z = sc * (K @ q[s, h].astype(np.float64))
+            w = np.exp(z - logsumexp(z))
+            assert lse[s, h] == pytest.approx(logsumexp(z), abs=1e-12)
+            assert np.allclose(out[s, h], w @ V, rtol=0, atol=1e-12 * np.abs(V).max())

@@ -109,6 +109,15 @@ def test_e4m3_encode_matches_torch_in_range():
     assert np.array_equal(codecs.e4m3_encode(y), ref)
 
 
+def test_e4m3_nan_encodes_to_a_nan_pattern():
+    """The format has no infinities and its only NaN patterns are S.1111.111: NaN must encode
+    to one of them (torch agrees on the positive one), never to a finite code."""
+    y = np.array([np.nan], np.float32)
+    c = codecs.e4m3_encode(y)
+    assert np.isnan(codecs.e4m3_decode(c))[0] and (int(c[0]) & 0x7F) == 0x7F
+    assert int(c[0]) == int(torch.from_numpy(y).to(torch.float8_e4m3fn).view(torch.uint8)[0])
+
+
 def test_e4m3_roundtrip_all_finite_codes():
     codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
     vals = codecs.e4m3_decode(codes).astype(np.float32)

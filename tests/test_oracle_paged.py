@@ -173,48 +173,64 @@ def test_cow_append_keeps_shared_content_semantics():
             assert np.array_equal(kc[row[t // B], :, t % B], full[t])
 
 
+def _nearest_code(y, cache_dt, zero=0):
+    """Brute force: the codes whose decoded value is nearest to y (all of them on a tie)."""
+    if cache_dt == "fp8":
+        vals = codecs.E4M3_TABLE
+        cand = [c for c in range(256) if np.isfinite(vals[c]) and bool(c & 0x80) == bool(np.signbit(y))]
+        dist = [abs(float(y) - vals[c]) for c in cand]
+    else:
+        cand = list(range(-128, 128))
+        dist = [abs(float(y) - (c - zero)) for c in cand]
+    best = min(dist)
+    return [c for c, dd in zip(cand, dist) if dd == best]
+
+
 @pytest.mark.parametrize("in_dt,cache_dt", [("f32", "f32"), ("f32", "bf16"), ("bf16", "bf16"),
-                                            ("bf16", "fp8"), ("f32", "fp8")])
+                                            ("bf16", "fp8"), ("f32", "fp8"), ("f32", "int8"),
+                                            ("bf16", "int8")])
 def test_reshape_and_cache_readback(in_dt, cache_dt):
+    """K and V get different inputs, scales and zero points; every written element is read
+    back against the format's definition (fp8 / int8: a nearest code to x / scale, the int8
+    code offset by the block's zero point and clipped to the byte's range)."""
     rng = np.random.default_rng(11)
     NB, H, B, d, T = 10, 3, 16, 16, 37
-    xf = rng.standard_normal((T, H, d)).astype(np.float32)
-    x = xf if in_dt == "f32" else codecs.bf16_encode(xf)
-    xv = xf if in_dt == "f32" else codecs.bf16_decode(x).astype(np.float32)
+    quant = cache_dt in ("fp8", "int8")
+    big = 40.0 if cache_dt == "int8" else 1.0       # int8: values span many codes and clip
+    raw = {n: (rng.standard_normal((T, H, d)) * big).astype(np.float32) for n in "kv"}
+    x = {n: raw[n] if in_dt == "f32" else codecs.bf16_encode(raw[n]) for n in "kv"}
+    xv = {n: raw[n] if in_dt == "f32" else codecs.bf16_decode(x[n]).astype(np.float32) for n in "kv"}
     slots = rng.permutation(NB * B)[:T].astype(np.int64)
     slots[3] = -1
-    sc = (rng.uniform(0.5, 2.0, (NB, H))).astype(np.float32)
-    kc = paged.new_cache(NB, H, B, d, cache_dt)
-    vc = paged.new_cache(NB, H, B, d, cache_dt)
-    paged.ref_reshape_and_cache(x, x, kc, vc, slots, in_dt, cache_dt, sc, sc)
+    sc = {n: rng.uniform(0.5, 2.0, (NB, H)).astype(np.float32) for n in "kv"}
+    zp = {n: rng.integers(-40, 41, (NB, H)).astype(np.int32) for n in "kv"}
+    cache = {n: paged.new_cache(NB, H, B, d, cache_dt) for n in "kv"}
+    paged.ref_reshape_and_cache(x["k"], x["v"], cache["k"], cache["v"], slots, in_dt, cache_dt,
+                                sc["k"] if quant else None, sc["v"] if quant else None,
+                                zp["k"] if cache_dt == "int8" else None,
+                                zp["v"] if cache_dt == "int8" else None)
     written = np.zeros((NB, B), bool)
     for t, sl in enumerate(slots):
         if sl < 0:
             continue
         blk, off = sl // B, sl % B
         written[blk, off] = True
-        got = kc[blk, :, off, :]
-        if cache_dt == "f32":
-            assert np.array_equal(got, xv[t])
-        elif cache_dt == "bf16":
-            ref = torch.from_numpy(xv[t].copy()).to(torch.bfloat16).view(torch.int16).numpy()
-            assert np.array_equal(got, ref.view(np.uint16))
-        else:
-            # nearest E4M3 value to x/scale (ties even), brute force per element
-            y = (xv[t] / sc[blk][:, None]).astype(np.float32)
-            vals = codecs.E4M3_TABLE
-            for h in range(H):
-                for j in range(d):
-                    cand = [c for c in range(256) if np.isfinite(vals[c])
-                            and bool(c & 0x80) == bool(np.signbit(y[h, j]))]
-                    dist = [abs(float(y[h, j]) - vals[c]) for c in cand]
-                    best = min(dist)
-                    ok = [c for c, dd in zip(cand, dist) if dd == best]
-                    assert got[h, j] in ok
-        assert np.array_equal(vc[blk, :, off, :], kc[blk, :, off, :])
+        for n in "kv":
+            got = cache[n][blk, :, off, :]
+            if cache_dt == "f32":
+                assert np.array_equal(got, xv[n][t])
+            elif cache_dt == "bf16":
+                ref = torch.from_numpy(xv[n][t].copy()).to(torch.bfloat16).view(torch.int16).numpy()
+                assert np.array_equal(got, ref.view(np.uint16))
+            else:
+                y = (xv[n][t] / sc[n][blk][:, None]).astype(np.float32)
+                for h in range(H):
+                    z = int(zp[n][blk, h]) if cache_dt == "int8" else 0
+                    for j in range(d):
+                        assert int(got[h, j]) in _nearest_code(y[h, j], cache_dt, z)
     # unwritten slots stay zero
-    mask = np.broadcast_to(~written[:, None, :, None], kc.shape)
-    assert np.all(kc[mask] == 0)
+    mask = np.broadcast_to(~written[:, None, :, None], cache["k"].shape)
+    assert np.all(cache["k"][mask] == 0) and np.all(cache["v"][mask] == 0)
 
 
 def test_copy_blocks_copies_tiles_and_scales():

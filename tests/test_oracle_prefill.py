@@ -41,16 +41,18 @@ def _scale(draw):
     return float(np.float32(1.0 / math.sqrt(draw.wl.head_dim)))
 
 
-def test_one_new_token_is_a_decode_step():
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8"])
+def test_one_new_token_is_a_decode_step(kv):
     wl = workloads.PREFILL_WORKLOADS["chunked"].scaled(num_seqs=4, new=("chunk", 1),
                                                        lens=("fixed", [1, 17, 300, 1000]),
-                                                       num_blocks=256)
+                                                       num_blocks=256, kv_dtype=kv)
     d = workloads.draw_prefill(wl)
     st = flows.build_prefill_state(d)
     o, l = flows.ref_prefill_outputs(d, st)
     od, ld = attention.ref_decode(d.q, st.k_cache, st.v_cache, st.block_tables,
                                   st.context_lens, _scale(d), wl.num_kv_heads, wl.in_dtype,
-                                  wl.kv_dtype)
+                                  wl.kv_dtype, st.k_scales, st.v_scales, k_zeros=st.k_zeros,
+                                  v_zeros=st.v_zeros)
     assert np.allclose(o, od, rtol=0, atol=1e-12) and np.allclose(l, ld, rtol=0, atol=1e-12)
 
 
