@@ -1,0 +1,80 @@
+"""The bench's host-side contract, on CPU: the reference arm's JSON line (the oracle timed on
+host cores), rank handling under a multi-rank launch, the warm-up floor, the clock summary
+taken during the timed region, and the whole-job throughput arithmetic."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _run(args, env_extra=None):
+    env = dict(os.environ)
+    env.update(env_extra or {})
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT,
+                          env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_reference_arm_prints_one_contract_line():
+    p = _run(["--impl", "reference", "--workload", "tiny", "--steps", "4", "--warmup", "3"])
+    assert p.returncode == 0, p.stderr
+    lines = [l for l in p.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    j = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "impl", "cpu_baseline", "e2e"):
+        assert key in j, key
+    assert j["impl"] == "reference" and j["metric"] == bench.METRIC and j["unit"] == "GB/s"
+    assert j["value"] > 0 and j["steps"] == 4 and j["warmup"] == 3 and j["n_gpus"] == 1
+    assert j["higher_is_better"] is True and j["dtype"] == "f64"
+    assert j["config"]["workload"] == bench.DESCR["tiny"]
+    cb = j["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"] and cb["sample"]
+    assert j["e2e"] == {"value": j["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    p = _run(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "3"],
+             {"WORLD_SIZE": "2", "RANK": "1"})
+    assert p.returncode == 0 and p.stdout.strip() == ""
+
+
+def test_warmup_floor():
+    p = _run(["--impl", "reference", "--workload", "tiny", "--steps", "3", "--warmup", "2"])
+    assert p.returncode != 0 and "--warmup must be >= 3" in p.stderr
+
+
+def test_clock_summary():
+    cs = bench.ClockSampler(0)
+    # timestamp, clocks.sm, clocks.max.sm, power.draw, clocks_event_reasons.active
+    cs.samples = [(0.5, "t, 1100, 1965, 300.0, 0x0000000000000001"),
+                  (1.0, "t, 1965, 1965, 900.5, 0x0000000000000000"),
+                  (1.2, "t, 1900, 1965, 1000.0, 0x0000000000000004"),
+                  (1.4, "t, 1950, 1965, 990.0, 0x0000000000000000"),
+                  (1.6, "garbled"),
+                  (9.0, "t, 300, 1965, 100.0, 0x0000000000000048")]
+    s = cs.summary(0.9, 1.5)
+    assert s["samples"] == 3 and s["sm_mhz"] == 1950.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["note"] == "inside timed region"
+    # a timed region shorter than the sampling period takes the nearest samples
+    s = cs.summary(8.9, 8.95)
+    assert s["note"].startswith("nearest") and "hw_slowdown" in s["reasons"] \
+        and "hw_thermal_slowdown" in s["reasons"]
+    # idle is never reported as a reason
+    assert "gpu_idle" not in cs.summary(0.0, 0.6)["reasons"]
+    empty = bench.ClockSampler(0)
+    assert empty.summary(0.0, 1.0)["sm_mhz"] is None
+
+
+def test_job_throughput_and_slowest_rank():
+    # 2 ranks, 1 GB per rank-step, 10 steps, slowest rank 4 s -> 5 GB/s for the job
+    assert bench.job_throughput(10 ** 9, 10, 2, 4.0) == pytest.approx(5.0)
+    assert bench.slowest_rank_seconds(1.25) == 1.25
