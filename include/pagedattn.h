@@ -15,9 +15,10 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Pointers named *_cache, q, out, k, v, block_tables, context_lens, slot_mapping, pairs,
- *   *_scales, lse_out and workspace are DEVICE pointers; the caller owns them. The library
- *   allocates no device memory.
+ * - Pointers named *_cache, q, out, k, v, block_tables, context_lens, query_start,
+ *   slot_mapping, pairs, *_scales, *_zeros, lse_out and workspace are DEVICE pointers; the
+ *   caller owns them. The library allocates no device memory (paged_attn_decode_noalloc's
+ *   fixed array is compiled into the library, below).
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device
  *   work is enqueued asynchronously on it; a PA_OK return means "enqueued".
  * - Every call validates its host-side arguments first and returns an error without
