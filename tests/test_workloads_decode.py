@@ -87,3 +87,41 @@ def test_int8_params_put_the_block_range_on_the_byte_range(s):
             assert c.min() <= -127 and c.max() >= 126
             back = (c.astype(np.float64) - kz[b, h]) * ks[b, h]
             assert np.max(np.abs(back - blk[:, h])) <= ks[b, h] * 1.0 + 1e-6
+
+
+@pytest.mark.parametrize("name", ["tiny", "b32", "shared"])
+def test_decode_state_layout(name):
+    """The oracle's state builder against the draw, token by token: every cached token's K
+    and V sit at slot table[t // B] * B + t % B with the draw's values (bf16 / f32 bits
+    unchanged), the step token is the last position, tables use ceil(ctx / B) blocks, and
+    sequences share physical blocks only on the shared-prefix workload."""
+    from oracle import flows
+    wl = workloads.WORKLOADS[name]
+    if name == "b32":
+        wl = wl.scaled(num_seqs=6, num_blocks=1024)
+    d = workloads.draw(wl)
+    st = flows.build_state(d)
+    B = wl.block_size
+    owners = {}
+    for s in range(wl.num_seqs):
+        n = int(d.context_lens[s])
+        row = st.block_tables[s]
+        nblk = -(-n // B)
+        assert np.all(row[:nblk] >= 0) and np.all(row[nblk:] == -1)
+        for b in row[:nblk]:
+            owners.setdefault(int(b), set()).add(s)
+        k, v = d.kv(s)
+        t = np.arange(n)
+        blk, off = row[t // B], t % B
+        assert np.array_equal(st.k_cache[blk, :, off, :], k)
+        assert np.array_equal(st.v_cache[blk, :, off, :], v)
+        last = n - 1
+        assert st.step_slots[s].tolist()[-1] == int(row[last // B]) * B + last % B
+    shared = [b for b, o in owners.items() if len(o) > 1]
+    if name == "shared":
+        # the 12 full blocks of the 200-token prefix are shared by all 100 sequences; the
+        # partial 13th was copied on write by 99 of them
+        assert len(shared) == 12 and all(len(owners[b]) == 100 for b in shared)
+        assert len(st.cow_pairs) == 99
+    else:
+        assert not shared and not st.cow_pairs
