@@ -60,6 +60,14 @@ MUTANTS = {
                                     "state.v_zeros, state.k_zeros, seqs=seqs)"),
     "state_tokens_shifted": ("flows.py", "ref_reshape_and_cache(k[:-1], v[:-1], kc, vc, pre[s],",
                              "ref_reshape_and_cache(k[1:], v[1:], kc, vc, pre[s],"),
+    "decode_scale_one_over_d": ("flows.py", "1.0 / np.sqrt(wl.head_dim) if scale is None else "
+                                "scale))\n    return ref_decode(",
+                                "1.0 / wl.head_dim if scale is None else "
+                                "scale))\n    return ref_decode("),
+    "prefill_scale_one_over_d": ("flows.py", "1.0 / np.sqrt(wl.head_dim) if scale is None else "
+                                 "scale))\n    return ref_prefill(",
+                                 "1.0 / wl.head_dim if scale is None else "
+                                 "scale))\n    return ref_prefill("),
     # codecs
     "e4m3_bias_8": ("codecs.py", "2.0 ** (e - 7)", "2.0 ** (e - 8)"),
     "e4m3_subnormal_exponent": ("codecs.py", "2.0 ** (1 - 7)", "2.0 ** (0 - 7)"),
