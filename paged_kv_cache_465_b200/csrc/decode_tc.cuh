@@ -730,14 +730,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
 }
 
 // =======================================================================================
-// Split path: plan kernel + persistent kernels; lse_reduce_kernel merges the partitions.
+// Split path: plan kernel + persistent kernels; the partitions are merged by the warp
+// workers themselves (rows of up to 32 partitions) or by lse_reduce_kernel afterwards.
 // =======================================================================================
 // Workspace of the split path (offsets in bytes, each region 256-aligned):
 //   [0]     uint32 fetch counter, uint32 total items
 //   list    int2 (seq, partition) per partition item, largest items first
 //   m, l    float [S][Hq][P];  acc float [S][Hq][P][kD]   (partials, as the CUDA-core path)
-// Sequences with a single partition are written to `out` directly; the others are merged
-// by lse_reduce_kernel afterwards (spread over every (seq, q head)).
+//   arrive  uint32 [S][Hkv]: partials stored so far (warp workers merging in place)
+// Sequences with a single partition are written to `out` directly. The others are merged
+// by the warp that stores their last partial (warp workers, P <= 32), else by
+// lse_reduce_kernel afterwards (spread over every (seq, q head)).
 struct PlanView {
   uint32_t* counters;  // [0] fetch, [1] total
   int2* list;
@@ -745,7 +748,8 @@ struct PlanView {
 
 // One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
 // largest first (full partitions, then partial ones by size), writes the list, zeroes the
-// fetch counter, and writes out = 0 / lse = -inf for empty sequences.
+// fetch counter (and the arrival counters of the merging warp workers), and writes
+// out = 0 / lse = -inf for empty sequences.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
   __shared__ int cnt[130], off[130];
   pdl_wait();
@@ -753,6 +757,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   const int P = a.part_tokens;
   const int nbk = P / kSub;  // sub-tiles of a full partition (<= 128)
   for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
+  if (a.fused_merge)
+    for (int64_t i = threadIdx.x; i < (int64_t)a.num_seqs * a.num_kv_heads; i += blockDim.x)
+      a.arrive[i] = 0u;
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int ctx = checked_ctx(a, s);
@@ -787,6 +794,49 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
     }
     if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
+  }
+}
+
+// Merge of the partitions of the G query rows row0 .. row0+G-1 (one (sequence, kv head)),
+// run by the warp that stored the last of their partials; np <= 32. Lane p holds
+// partition p's running max and sum, lane k owns channel quad k (4 k .. 4 k + 3):
+// M = max_p m_p, L = sum_p 2^(m_p - M) l_p, out = sum_p 2^(m_p - M) acc_p / L. The
+// arithmetic and its order are those of lse_reduce_kernel, so the result does not depend
+// on which warp merges. Partials are read through L2 (ld.global.cg): other SMs wrote them
+// during this launch.
+__device__ __forceinline__ void merge_rows(const DecodeArgs& a, int64_t row0, int G, int np,
+                                           int lane) {
+  static_assert(kD == 128, "one channel quad per lane");
+  for (int g = 0; g < G; ++g) {
+    const int64_t row = row0 + g;
+    const float* pm = a.part_m + row * a.max_parts;
+    const float* pl = a.part_l + row * a.max_parts;
+    const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * kD);
+    const float mp = lane < np ? __ldcg(pm + lane) : -INFINITY;
+    float M = mp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (lane < np && M != -INFINITY) ? fast_exp2(mp - M) : 0.f;
+    float lsum = 0.f;
+    if (lane < np) lsum = fmaf(w, __ldcg(pl + lane), lsum);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < np; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float4 v = __ldcg(pacc + (int64_t)k * (kD / 4) + lane);
+      acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
+      acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const int64_t o = row * kD + 4 * lane;
+    store_out(a.out, a.out_dtype, o, acc.x * inv);
+    store_out(a.out, a.out_dtype, o + 1, acc.y * inv);
+    store_out(a.out, a.out_dtype, o + 2, acc.z * inv);
+    store_out(a.out, a.out_dtype, o + 3, acc.w * inv);
+    if (lane == 0 && a.lse_out != nullptr)
+      a.lse_out[row] = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
   }
 }
 
@@ -1208,6 +1258,22 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
           a.part_m[pr] = ms[h];
           a.part_l[pr] = ls[h];
         }
+      }
+    }
+    // ---- the last partial of a (sequence, kv head) to be stored merges them all ----
+    if (cur.np > 1 && a.fused_merge) {
+      __threadfence();  // this lane's partial stores, before the arrival below
+      __syncwarp();
+      uint32_t prev = 0;
+      if (lane == 0) {
+        __threadfence();
+        prev = atomicAdd(a.arrive + (int64_t)cur.s * Hkv + cur.kvh, 1u);
+      }
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev == (uint32_t)cur.np - 1) {
+        __threadfence();  // the other partials, stored before their arrivals, are visible
+        __syncwarp();
+        merge_rows(a, row0, G, cur.np, lane);
       }
     }
     // ---- advance ----
