@@ -184,6 +184,44 @@ def _e2e(torch, sc, steps: int, flush):
     return total, h2d, d2h
 
 
+def _host_bookkeeping(pa, steps: int = 100):
+    """Host side of the step, through the Python binding: the allocator's bookkeeping for
+    one new token per sequence of the batch-256 workload (its context lengths, 16-token
+    blocks), as one append_batch call per step and, for comparison, one append call per
+    sequence; and the prefix cache on the shared-system-prompt example (100 requests of one
+    200-token prompt plus 50 private tokens each), one add_seq_tokens call per request."""
+    wl = workloads.WORKLOADS["b256"]
+    lens = [int(x) - 1 for x in workloads.draw(wl).context_lens]
+    ids = np.arange(len(lens), dtype=np.int32)  # the running batch, as a serving loop holds it
+    out = {"unit": "us", "threads": 1, "num_seqs": len(lens)}
+    for how in ("append_batch", "append"):
+        a = pa.BlockAllocator(wl.num_blocks, 16)
+        for s, n in zip(ids.tolist(), lens):
+            a.add_seq(s, n)
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            if how == "append_batch":
+                a.append_batch(ids, 1)
+            else:
+                for s in ids.tolist():
+                    a.append(s, 1)
+        dt = (time.perf_counter() - t0) / steps
+        out[f"{how}_us_per_step"] = round(dt * 1e6, 2)
+    rng = np.random.default_rng(2)
+    prompt = rng.integers(0, 32000, 200).tolist()
+    reqs = [prompt + rng.integers(0, 32000, 50).tolist() for _ in range(100)]
+    a = pa.BlockAllocator(512, 16)
+    t0 = time.perf_counter()
+    cached = sum(a.add_seq_tokens(r, toks)[1] for r, toks in enumerate(reqs))
+    dt = (time.perf_counter() - t0) / len(reqs)
+    out["add_seq_tokens_us_per_request"] = round(dt * 1e6, 2)
+    out["prefix_cached_tokens"] = int(cached)
+    out["steps"] = steps
+    out["note"] = ("host time per decode step next to the device step; one call per step "
+                   "(append_batch) against one call per sequence (append)")
+    return out
+
+
 def _cpu_baseline(draw, seconds: float = 12.0):
     """The oracle, as it stands, on the host cores: this step's cache write plus decode for a
     bounded sample of the workload's sequences (cycled until ~`seconds` elapse)."""
@@ -325,6 +363,8 @@ def run_ours(args):
         result["roofline"]["traffic"] = traffic
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = _cpu_baseline(draw, args.cpu_seconds)
+    if rank == 0:
+        result["host"] = _host_bookkeeping(pa)
     if rank == 0 and args.extra and world == 1:
         result["workloads"] = _extra_workloads(torch, pa, args, flush)
     if dist is not None:

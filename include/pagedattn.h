@@ -15,9 +15,10 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Pointers named *_cache, q, out, k, v, block_tables, context_lens, slot_mapping, pairs,
- *   *_scales, lse_out and workspace are DEVICE pointers; the caller owns them. The library
- *   allocates no device memory.
+ * - Pointers named *_cache, q, out, k, v, block_tables, context_lens, query_start,
+ *   slot_mapping, pairs, *_scales, *_zeros, lse_out and workspace are DEVICE pointers; the
+ *   caller owns them. The library allocates no device memory (paged_attn_decode_noalloc's
+ *   fixed array is compiled into the library, below).
  * - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream). Device
  *   work is enqueued asynchronously on it; a PA_OK return means "enqueued".
  * - Every call validates its host-side arguments first and returns an error without
@@ -301,6 +302,24 @@ pa_status pa_alloc_fork(pa_allocator* a, int parent_id, int child_id);
  * copy-on-write copy and *num_cow_out is 0 or 1. */
 pa_status pa_alloc_append(pa_allocator* a, int seq_id, int num_tokens, int64_t* slots_out,
                           int32_t* cow_pairs_out, int* num_cow_out);
+/*
+ * One decode step's appends in one call: num_tokens[i] tokens to sequence seq_ids[i] for
+ * i = 0 .. n-1, in that order, with the same results as n pa_alloc_append calls, except
+ * that the batch is all-or-nothing: when the free queue cannot serve the whole batch (the
+ * copies included), PA_ERR_NO_BLOCKS is returned and nothing changes. Sequence ids must be
+ * distinct and known (else PA_ERR_INVALID, nothing changed).
+ *   seq_ids, num_tokens  host int32 [n]
+ *   slots_out            host int64 [sum of num_tokens] or NULL: sequence i's slots follow
+ *                        sequence i-1's
+ *   cow_pairs_out        host int32 [n][2], NULL only if no copy can occur: the (src, dst)
+ *                        copy-on-write pairs in batch order; *num_cow_out (may be NULL)
+ *                        receives their number
+ * One call per step instead of one per sequence keeps the host's share of a decode step
+ * small for large batches.
+ */
+pa_status pa_alloc_append_batch(pa_allocator* a, int n, const int32_t* seq_ids,
+                                const int32_t* num_tokens, int64_t* slots_out,
+                                int32_t* cow_pairs_out, int* num_cow_out);
 pa_status pa_alloc_free_seq(pa_allocator* a, int seq_id);
 /* Copies at most `cap` entries of the sequence's block table into out (host int32) and
  * returns the table's length, or -1 for an unknown sequence. */

@@ -19,6 +19,7 @@ shared block is copied only when a writer modifies it.
 """
 from __future__ import annotations
 
+import copy
 import hashlib
 from collections import deque
 from typing import Dict, List, Optional, Sequence, Tuple
@@ -195,6 +196,29 @@ class RefAllocator:
             row.append(self._pop())
         self.lens[seq] = L + num_tokens
         return self._slots(seq, L, num_tokens), pairs
+
+    def append_batch(self, seqs: Sequence[int], counts: Sequence[int]
+                     ) -> Tuple[np.ndarray, List[Tuple[int, int]]]:
+        """append(seqs[i], counts[i]) for every i, in order, as one all-or-nothing call: the
+        policy's "a failed call changes nothing" read for a batch. Ids must be distinct and
+        known. Returns the slots of all tokens (sequence after sequence) and the copy pairs
+        in batch order."""
+        seqs, counts = [int(x) for x in seqs], [int(x) for x in counts]
+        if len(seqs) != len(counts) or len(set(seqs)) != len(seqs) or \
+                any(s not in self.tables for s in seqs) or any(c < 0 for c in counts):
+            raise InvalidCall("append_batch")
+        saved = copy.deepcopy(self.__dict__)
+        slots, pairs = [], []
+        try:
+            for s, c in zip(seqs, counts):
+                sl, pr = self.append(s, c)
+                slots.append(sl)
+                pairs.extend(pr)
+        except NoBlocks:
+            self.__dict__.clear()
+            self.__dict__.update(saved)
+            raise
+        return (np.concatenate(slots) if slots else np.zeros(0, np.int64)), pairs
 
     def free_seq(self, seq: int) -> None:
         if seq not in self.tables:

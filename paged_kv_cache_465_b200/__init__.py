@@ -80,6 +80,7 @@ _SIGS = {
     "pa_alloc_add_seq": (_i, [_vp, _i, _i, _vp]),
     "pa_alloc_fork": (_i, [_vp, _i, _i]),
     "pa_alloc_append": (_i, [_vp, _i, _i, _vp, _vp, _P(_i)]),
+    "pa_alloc_append_batch": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _P(_i)]),
     "pa_alloc_free_seq": (_i, [_vp, _i]),
     "pa_alloc_block_table": (_i, [_vp, _i, _vp, _i]),
     "pa_alloc_seq_len": (_i, [_vp, _i]),
@@ -425,6 +426,25 @@ class BlockAllocator:
                                     pair.ctypes.data_as(ctypes.c_void_p), ctypes.byref(n)),
                "pa_alloc_append")
         return slots, ([(int(pair[0]), int(pair[1]))] if n.value else [])
+
+    def append_batch(self, seqs, num_tokens) -> Tuple[np.ndarray, np.ndarray]:
+        """Appends num_tokens[i] tokens to seqs[i] for every i in one library call, in order,
+        all or nothing (``NoBlocks`` and no change when the whole batch does not fit).
+        ``num_tokens`` may be one int for every sequence. Returns (slots of all the tokens,
+        sequence after sequence; int32 [k, 2] copy-on-write pairs in batch order)."""
+        ids = np.ascontiguousarray(seqs, dtype=np.int32).ravel()
+        cnt = np.ascontiguousarray(np.broadcast_to(np.asarray(num_tokens, dtype=np.int32),
+                                                   ids.shape), dtype=np.int32)
+        slots = np.empty(int(cnt.sum()) if cnt.size else 0, dtype=np.int64)
+        pairs = np.empty((max(ids.size, 1), 2), dtype=np.int32)
+        n = ctypes.c_int(0)
+        _check(_lib.pa_alloc_append_batch(self._h, int(ids.size),
+                                          ids.ctypes.data_as(ctypes.c_void_p),
+                                          cnt.ctypes.data_as(ctypes.c_void_p),
+                                          slots.ctypes.data_as(ctypes.c_void_p),
+                                          pairs.ctypes.data_as(ctypes.c_void_p),
+                                          ctypes.byref(n)), "pa_alloc_append_batch")
+        return slots, pairs[:n.value].copy()
 
     def free_seq(self, seq: int) -> None:
         _check(_lib.pa_alloc_free_seq(self._h, int(seq)), "pa_alloc_free_seq")

@@ -50,6 +50,11 @@ class PagedKVCache:
     def append(self, seq: int, num_tokens: int) -> Tuple[np.ndarray, List[Tuple[int, int]]]:
         return self.alloc.append(seq, num_tokens)
 
+    def append_batch(self, seqs, num_tokens=1) -> Tuple[np.ndarray, np.ndarray]:
+        """A decode step's bookkeeping in one library call (all or nothing): the new tokens'
+        slots, sequence after sequence, and the copy-on-write pairs to copy first."""
+        return self.alloc.append_batch(seqs, num_tokens)
+
     def free_seq(self, seq: int) -> None:
         self.alloc.free_seq(seq)
 

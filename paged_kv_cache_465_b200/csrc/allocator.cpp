@@ -25,6 +25,7 @@
 // queue (so the queue order is the LRU order) and loses it when the queue hands it out.
 // The free queue is an intrusive doubly linked list, so a hit can take a waiting block out
 // of the middle in O(1).
+#include <algorithm>
 #include <array>
 #include <climits>
 #include <cstdint>
@@ -187,13 +188,38 @@ struct pa_allocator {
     refs[b] -= 1;
     if (refs[b] == 0) push_back(b);
   }
-  void slots(int seq, int start, int n, int64_t* out) const {
+  // Appends n tokens to an existing sequence whose preconditions were checked (enough free
+  // blocks; a pair buffer when a copy can occur): copies the last block first when it is
+  // partially filled and shared, then pops one block per block boundary crossed. Writes
+  // the tokens' slots and the copy pair; returns the number of pairs (0 or 1).
+  // `row` and `len` are the sequence's block table and length.
+  int append_checked(std::vector<int32_t>& row, int& len, int n, int64_t* slots_out,
+                     int32_t* pair_out) {
+    const int L = len;
+    const bool cow = n > 0 && L % block_size != 0 && refs[row.back()] > 1;
+    if (cow) {
+      const int32_t old_b = row.back();
+      const int32_t new_b = pop();
+      refs[old_b] -= 1;
+      row.back() = new_b;
+      pair_out[0] = old_b;
+      pair_out[1] = new_b;
+    }
+    const int64_t grow = ceil_div((int64_t)L + n, block_size) - ceil_div(L, block_size);
+    for (int64_t i = 0; i < grow; ++i) row.push_back(pop());
+    len = L + n;
+    row_slots(row, L, n, slots_out);
+    return cow ? 1 : 0;
+  }
+  void row_slots(const std::vector<int32_t>& row, int start, int n, int64_t* out) const {
     if (out == nullptr) return;
-    const std::vector<int32_t>& row = tables.at(seq);
     for (int i = 0; i < n; ++i) {
       const int p = start + i;
       out[i] = (int64_t)row[p / block_size] * block_size + p % block_size;
     }
+  }
+  void slots(int seq, int start, int n, int64_t* out) const {
+    row_slots(tables.at(seq), start, n, out);
   }
 };
 
@@ -319,28 +345,70 @@ pa_status pa_alloc_append(pa_allocator* a, int seq_id, int num_tokens, int64_t* 
   if (a == nullptr || num_tokens < 0) return PA_ERR_INVALID;
   auto it = a->tables.find(seq_id);
   if (it == a->tables.end()) return PA_ERR_INVALID;
-  std::vector<int32_t>& row = it->second;
+  const std::vector<int32_t>& row = it->second;
   const int B = a->block_size;
-  const int L = a->lens[seq_id];
+  const int L = a->lens.at(seq_id);
   if ((int64_t)L + num_tokens > INT32_MAX) return PA_ERR_INVALID;
   const bool cow = num_tokens > 0 && L % B != 0 && a->refs[row.back()] > 1;
   if (cow && cow_pairs_out == nullptr) return PA_ERR_INVALID;
   const int64_t grow = ceil_div((int64_t)L + num_tokens, B) - ceil_div(L, B);
   if ((cow ? 1 : 0) + grow > (int64_t)a->nfree) return PA_ERR_NO_BLOCKS;
-  int ncow = 0;
-  if (cow) {
-    const int32_t old_b = row.back();
-    const int32_t new_b = a->pop();
-    a->refs[old_b] -= 1;
-    row.back() = new_b;
-    cow_pairs_out[0] = old_b;
-    cow_pairs_out[1] = new_b;
-    ncow = 1;
-  }
-  for (int64_t i = 0; i < grow; ++i) row.push_back(a->pop());
-  a->lens[seq_id] = L + num_tokens;
+  const int ncow = a->append_checked(it->second, a->lens[seq_id], num_tokens, slots_out,
+                                     cow_pairs_out);
   if (num_cow_out) *num_cow_out = ncow;
-  a->slots(seq_id, L, num_tokens, slots_out);
+  return PA_OK;
+}
+
+pa_status pa_alloc_append_batch(pa_allocator* a, int n, const int32_t* seq_ids,
+                                const int32_t* num_tokens, int64_t* slots_out,
+                                int32_t* cow_pairs_out, int* num_cow_out) {
+  if (a == nullptr || n < 0) return PA_ERR_INVALID;
+  if (n > 0 && (seq_ids == nullptr || num_tokens == nullptr)) return PA_ERR_INVALID;
+  const int B = a->block_size;
+  std::vector<int32_t> ids(seq_ids, seq_ids + n);  // distinct ids
+  std::sort(ids.begin(), ids.end());
+  if (std::adjacent_find(ids.begin(), ids.end()) != ids.end()) return PA_ERR_INVALID;
+  // checks, and the blocks the whole batch pops: the appends run in batch order, and a
+  // copy-on-write drops the old block's ref_count, which later sequences of the batch see
+  struct Item {
+    std::vector<int32_t>* row;
+    int* len;
+  };
+  std::vector<Item> items((size_t)n);
+  std::unordered_map<int32_t, int> ref_delta;
+  int64_t need = 0;
+  bool any_cow = false;
+  for (int i = 0; i < n; ++i) {
+    const int s = seq_ids[i], k = num_tokens[i];
+    if (k < 0) return PA_ERR_INVALID;
+    auto it = a->tables.find(s);
+    if (it == a->tables.end()) return PA_ERR_INVALID;
+    int& L = a->lens.find(s)->second;
+    if ((int64_t)L + k > INT32_MAX) return PA_ERR_INVALID;
+    items[i] = Item{&it->second, &L};
+    if (k > 0 && L % B != 0) {
+      const int32_t last = it->second.back();
+      auto d = ref_delta.find(last);
+      const int refs = a->refs[last] + (d == ref_delta.end() ? 0 : d->second);
+      if (refs > 1) {
+        ref_delta[last] -= 1;
+        need += 1;
+        any_cow = true;
+      }
+    }
+    need += ceil_div((int64_t)L + k, B) - ceil_div(L, B);
+  }
+  if (any_cow && cow_pairs_out == nullptr) return PA_ERR_INVALID;
+  if (need > (int64_t)a->nfree) return PA_ERR_NO_BLOCKS;
+  int64_t off = 0;
+  int ncow = 0;
+  for (int i = 0; i < n; ++i) {
+    ncow += a->append_checked(*items[i].row, *items[i].len, num_tokens[i],
+                              slots_out ? slots_out + off : nullptr,
+                              cow_pairs_out ? cow_pairs_out + 2 * ncow : nullptr);
+    off += num_tokens[i];
+  }
+  if (num_cow_out) *num_cow_out = ncow;
   return PA_OK;
 }
 

@@ -1,6 +1,7 @@
 """The bench's host-side contract, on CPU: the reference arm's JSON line (the oracle timed on
 host cores), rank handling under a multi-rank launch, the warm-up floor, the clock summary
-taken during the timed region, and the whole-job throughput arithmetic."""
+taken during the timed region, the whole-job throughput arithmetic, and the host
+bookkeeping timing (allocator and prefix cache through the binding)."""
 import json
 import os
 import subprocess
@@ -78,3 +79,18 @@ def test_job_throughput_and_slowest_rank():
     # 2 ranks, 1 GB per rank-step, 10 steps, slowest rank 4 s -> 5 GB/s for the job
     assert bench.job_throughput(10 ** 9, 10, 2, 4.0) == pytest.approx(5.0)
     assert bench.slowest_rank_seconds(1.25) == 1.25
+
+
+def test_host_bookkeeping_timing():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(
+        "_pa_build", os.path.join(ROOT, "paged_kv_cache_465_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import paged_kv_cache_465_b200 as pa
+    h = bench._host_bookkeeping(pa, steps=3)
+    assert h["num_seqs"] == 256 and h["unit"] == "us"
+    assert h["append_batch_us_per_step"] > 0 and h["append_us_per_step"] > 0
+    assert h["add_seq_tokens_us_per_request"] > 0
+    assert h["prefix_cached_tokens"] == 99 * 192     # 12 full blocks reused per later request

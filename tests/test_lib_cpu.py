@@ -51,7 +51,7 @@ def _state(a):
 def test_allocator_matches_oracle_random_traces(pa):
     from oracle.paged import RefAllocator, NoBlocks as RefNoBlocks, InvalidCall
     rng = np.random.default_rng(123)
-    for trial in range(25):
+    for trial in range(30):
         nb = int(rng.integers(4, 300))
         order = rng.permutation(nb) if trial % 2 else None
         ref = RefAllocator(nb, 16, order=order)
@@ -64,8 +64,16 @@ def test_allocator_matches_oracle_random_traces(pa):
                 args = ("add_seq", nxt, int(rng.integers(0, 120)))
             elif op == 1:
                 args = ("fork", live[int(rng.integers(len(live)))], nxt)
-            elif op in (2, 3):
+            elif op == 2:
                 args = ("append", live[int(rng.integers(len(live)))], int(rng.integers(0, 50)))
+            elif op == 3:
+                # a batch over a random subset (forks share last blocks); now and then a
+                # duplicate or unknown id, which both sides must refuse
+                k = int(rng.integers(1, len(live) + 1))
+                ids = [live[i] for i in rng.choice(len(live), size=k, replace=False)]
+                if rng.random() < 0.1:
+                    ids.append(ids[0] if rng.random() < 0.5 else nxt + 1000)
+                args = ("append_batch", ids, rng.integers(0, 20, len(ids)).tolist())
             else:
                 args = ("free_seq", live[int(rng.integers(len(live)))])
             r_exc = n_exc = None
@@ -90,10 +98,40 @@ def test_allocator_matches_oracle_random_traces(pa):
                     assert np.array_equal(r_res, n_res)
                 if args[0] == "append":
                     assert np.array_equal(r_res[0], n_res[0]) and list(r_res[1]) == n_res[1]
+                if args[0] == "append_batch":
+                    assert np.array_equal(r_res[0], n_res[0])
+                    assert [tuple(p) for p in n_res[1].tolist()] == list(r_res[1])
             assert _state(nat) == (list(ref.free), ref.refs)
             for s in live:
                 assert nat.block_table(s) == ref.block_table(s)
                 assert nat.seq_len(s) == ref.seq_len(s)
+
+
+def test_append_batch_equals_single_appends_and_is_atomic(pa):
+    """A decode step of 100 forks that share a partial last block: one batch call gives the
+    slots, pairs and state of 100 single calls; a batch one block short changes nothing."""
+    one, bat = pa.BlockAllocator(256, 16), pa.BlockAllocator(256, 16)
+    for a in (one, bat):
+        a.add_seq(0, 200)
+        for c in range(1, 100):
+            a.fork(0, c)
+    ids = list(range(99, -1, -1))
+    s1, p1 = [], []
+    for s in ids:
+        sl, pr = one.append(s, 1)
+        s1.append(sl)
+        p1 += pr
+    s2, p2 = bat.append_batch(ids, 1)
+    assert np.array_equal(np.concatenate(s1), s2) and p1 == [tuple(p) for p in p2.tolist()]
+    assert len(p1) == 99 and _state(one) == _state(bat)
+    assert all(one.block_table(s) == bat.block_table(s) for s in ids)
+    before = (_state(bat), [bat.block_table(s) for s in ids], [bat.seq_len(s) for s in ids])
+    assert bat.num_free() == 256 - 13 - 99
+    with pytest.raises(pa.NoBlocks):          # 201 -> 233 tokens: 2 new blocks each, 200 > 144
+        bat.append_batch(ids, 32)
+    assert before == (_state(bat), [bat.block_table(s) for s in ids], [bat.seq_len(s) for s in ids])
+    with pytest.raises(pa.PagedAttnError):
+        bat.append_batch([1, 1], 1)
 
 
 def test_allocator_shared_prefix_example(pa):

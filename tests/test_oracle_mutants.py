@@ -107,6 +107,7 @@ MUTANTS = {
                              "        v_cache[src] = v_cache[dst]\n"),
     "copy_blocks_without_scales": ("paged.py", "                arr[dst] = arr[src]\n",
                                    "                pass\n"),
+    "batch_not_atomic": ("paged.py", "            self.__dict__.update(saved)\n", ""),
     "hash_not_chained": ("paged.py", "            m.update(parent)\n", "            pass\n"),
     "hash_big_endian": ("paged.py", 'dtype="<i4"', 'dtype=">i4"'),
     # closed forms

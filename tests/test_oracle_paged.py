@@ -248,3 +248,32 @@ def test_copy_blocks_copies_tiles_and_scales():
         assert ks[t] == pytest.approx(ks0[s]) and np.array_equal(vs[t], vs0[s])
     untouched = [b for b in range(NB) if b not in (7, 9, 11)]
     assert np.array_equal(kc[untouched], k0[untouched]) and np.array_equal(ks[untouched], ks0[untouched])
+
+
+def test_append_batch_hand_worked_and_all_or_nothing():
+    """Three forks share a partially filled last block (ref_count 3). Appending one token to
+    each in one batch copies it for the first two (ref 3 -> 2 -> 1); the third then owns it
+    and writes in place. A batch one block short changes nothing."""
+    B = 16
+    a = RefAllocator(8, B)
+    a.add_seq(0, 20)                            # blocks 0, 1 (block 1 holds 4 tokens)
+    a.fork(0, 1)
+    a.fork(0, 2)
+    slots, pairs = a.append_batch([1, 2, 0], [1, 1, 1])
+    assert pairs == [(1, 2), (1, 3)]            # seq 1 copies into 2, seq 2 into 3
+    assert a.block_table(1) == [0, 2] and a.block_table(2) == [0, 3] and a.block_table(0) == [0, 1]
+    assert list(slots) == [2 * B + 4, 3 * B + 4, 1 * B + 4]
+    assert a.refs[:4] == [3, 1, 1, 1] and list(a.free) == [4, 5, 6, 7]
+    # 4 free blocks; seq 0 needs 1 more (to 40 tokens), seqs 1 and 2 two each (to 49): 5 > 4
+    snap = (list(a.free), list(a.refs), {s: list(r) for s, r in a.tables.items()}, dict(a.lens))
+    with pytest.raises(NoBlocks):
+        a.append_batch([0, 1, 2], [19, 28, 28])
+    assert snap == (list(a.free), list(a.refs), {s: list(r) for s, r in a.tables.items()},
+                    dict(a.lens))
+    # without its last member the batch fits (1 + 2 = 3 blocks of 4)
+    slots, pairs = a.append_batch([0, 1], [19, 28])
+    assert pairs == [] and len(slots) == 47 and a.num_free() == 1
+    with pytest.raises(InvalidCall):
+        a.append_batch([0, 0], [1, 1])          # duplicate id
+    with pytest.raises(InvalidCall):
+        a.append_batch([0, 9], [1, 1])          # unknown id
