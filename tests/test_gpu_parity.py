@@ -145,6 +145,43 @@ def test_fp8_write_rounding_midpoints(pa):
         _same_codes(got, ref)
 
 
+def test_int8_write_ties_and_clipping(pa):
+    """int8 cache write at every half-integer x / scale in [-200, 200] (ties to even before
+    the zero point is added), one float32 step either side, and values past the byte's
+    range, with several zero points and scales (1 and 0.5 keep x / scale exact)."""
+    B, d = 16, 128
+    base = np.arange(-200, 200, dtype=np.float64) + 0.5
+    vals = np.concatenate([base, np.nextafter(base.astype(np.float32), np.float32(-1e9)),
+                           np.nextafter(base.astype(np.float32), np.float32(1e9)),
+                           np.array([0.0, -0.0, 1e9, -1e9, 127.5, -128.5, 127.49998], np.float32)])
+    vals = vals.astype(np.float32)
+    per = B * d
+    NB = -(-vals.size // per) * 4
+    x = np.zeros((NB * per,), np.float32)
+    reps = NB // (-(-vals.size // per))
+    for r in range(reps):
+        x[r * (NB // reps) * per: r * (NB // reps) * per + vals.size] = vals
+    zeros = np.array([[0], [7], [-30], [100]] * (NB // 4), np.int32)[:NB]
+    for sc in (1.0, 0.5):
+        scales = np.full((NB, 1), sc, np.float32)
+        xs = (x * np.float32(sc)).astype(np.float32).reshape(-1, 1, d)
+        T = xs.shape[0]
+        slots = np.arange(T, dtype=np.int64)
+        kref = opaged.new_cache(NB, 1, B, d, "int8")
+        vref = opaged.new_cache(NB, 1, B, d, "int8")
+        opaged.ref_reshape_and_cache(xs, xs, kref, vref, slots, "f32", "int8", scales, scales,
+                                     zeros, zeros)
+        k = torch.from_numpy(xs).cuda()
+        kc = torch.zeros((NB, 1, B, d), dtype=torch.int8, device="cuda")
+        vc = torch.zeros_like(kc)
+        s_d = torch.from_numpy(scales).cuda()
+        z_d = torch.from_numpy(zeros).cuda()
+        pa.reshape_and_cache(k, k, kc, vc, torch.from_numpy(slots).cuda(), k_scales=s_d,
+                             v_scales=s_d, k_zeros=z_d, v_zeros=z_d)
+        assert pa.device_error() == 0
+        assert np.array_equal(cache_codes(kc), kref)
+
+
 @pytest.mark.parametrize("cache_dt", ["f32", "bf16", "fp8", "int8"])
 def test_copy_blocks_bitexact(pa, cache_dt):
     rng = np.random.default_rng(5)
