@@ -32,7 +32,6 @@
 #pragma once
 
 #include "decode_tc.cuh"
-#include "exp2_fma.cuh"
 
 namespace pa {
 namespace pf {
@@ -681,10 +680,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if ((e & 8) == 0)  // columns e and e + 8 share a running max: one 3-input max
-            mx8[e & 7] = max3f(mx8[e & 7], __uint_as_float(sv[c][e]),
-                               __uint_as_float(sv[c][e + 8]));
+        for (int e = 0; e < 32; ++e) mx8[e & 7] = fmaxf(mx8[e & 7], __uint_as_float(sv[c][e]));
 #pragma unroll
       for (int k = 0; k < 4; ++k) mx8[k] = fmaxf(mx8[k], mx8[k + 4]);
       const float mx =
@@ -705,21 +701,8 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
-          // the two arguments in one packed fused multiply-add (same rounding as two)
-          float p0, p1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(sv[c][e]), __uint_as_float(sv[c][e + 1])),
-                           f2_pack(xs, xs), f2_pack(mneg, mneg)), p0, p1);
-          // bf16 caches: 5 of every 16 pairs on the FMA pipe (exp2_fma), the rest on the
-          // special-function unit, about the split at which both take the same time. The
-          // quantised kernels keep every exponential on the special-function unit: the
-          // polynomial's registers would make them spill.
-          if (!QUANT && (e >> 1) % 3 == 1) {
-            p0 = exp2_fma(p0);
-            p1 = exp2_fma(p1);
-          } else {
-            p0 = fast_exp2(p0);
-            p1 = fast_exp2(p1);
-          }
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sv[c][e]), xs, mneg));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sv[c][e + 1]), xs, mneg));
           rs8[e & 7] += p0;
           rs8[(e + 1) & 7] += p1;
           if constexpr (QUANT) {  // P carries the V scale of its key's block
