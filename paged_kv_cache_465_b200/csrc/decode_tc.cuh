@@ -509,11 +509,23 @@ struct SubWin {
   uint32_t z0, z1;     // int8: packed (K, V) zero points
 };
 
+// Sub-tile c's window entry in two steps, so that a caller can issue the block-table reads
+// and use them later: load_sub_ids reads the raw block ids, load_sub_params checks them and
+// reads the blocks' scales (and zero points). Both steps together are load_sub.
+template <int BS>
+__device__ __forceinline__ void load_sub_ids(const int32_t* btrow, int c, int t1, SubWin& w) {
+  if constexpr (BS == 8) {
+    w.p0 = btrow[2 * c];
+    w.p1 = c * kSub + 8 < t1 ? btrow[2 * c + 1] : -3;  // -3: second half absent
+  } else {
+    w.p0 = btrow[c * kSub / BS];
+  }
+}
+
 template <pa_dtype KV, int BS>
-__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
-                                         int t1, int kvh, SubWin& w) {
-  auto one = [&](int blk, int& p, float& ks, float& vs, uint32_t& z) {
-    p = btrow[blk];
+__device__ __forceinline__ void load_sub_params(const DecodeArgs& a, int c, int t1, int kvh,
+                                                SubWin& w) {
+  auto one = [&](int& p, float& ks, float& vs, uint32_t& z) {
     ks = 1.f;
     vs = 1.f;
     z = 0;
@@ -530,16 +542,23 @@ __device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btr
     }
   };
   if constexpr (BS == 8) {
-    one(2 * c, w.p0, w.ks0, w.vs0, w.z0);
+    one(w.p0, w.ks0, w.vs0, w.z0);
     if (c * kSub + 8 < t1) {
-      one(2 * c + 1, w.p1, w.ks1, w.vs1, w.z1);
+      one(w.p1, w.ks1, w.vs1, w.z1);
     } else {
       w.p1 = -3; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
     }
   } else {
-    one(c * kSub / BS, w.p0, w.ks0, w.vs0, w.z0);
+    one(w.p0, w.ks0, w.vs0, w.z0);
     w.p1 = w.p0; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
   }
+}
+
+template <pa_dtype KV, int BS>
+__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
+                                         int t1, int kvh, SubWin& w) {
+  load_sub_ids<BS>(btrow, c, t1, w);
+  load_sub_params<KV, BS>(a, c, t1, kvh, w);
 }
 
 __device__ __forceinline__ void empty_sub(SubWin& w) {
@@ -1159,10 +1178,65 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   int pslot = 0, pk = 0;
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
+  // From the second item on, the item after the current one is fetched in kFetchDone
+  // steps, one per consumed sub-tile. Each step uses only values that a global read issued
+  // one step earlier returns (work ticket, list entry, context length, block ids), so the
+  // reads overlap the current item's tiles instead of stalling the warp between items.
+  // An item shorter than that finishes the fetch at its end.
+  constexpr int kFetchDone = 5;
+  // int8 caches with 8-token blocks keep the fetch in one piece at the item boundary: the
+  // staged form would make that variant spill
+  constexpr bool kStaged = !(KV == PA_INT8 && BS == 8);
+  int nstage = kFetchDone;  // nxt and nxt_w are resolved
+  bool nxt_q = false;       // nxt's q copy is issued
+  uint32_t tk = 0;          // work ticket (lane 0 until broadcast)
+  int2 sp = make_int2(0, 0);
+  int sp_ctx = 0;
+  auto fetch_step = [&]() {
+    if (nstage == 0) {
+      if (lane == 0) tk = atomicAdd(&pl.counters[0], 1u);
+    } else if (nstage == 1) {
+      tk = __shfl_sync(0xffffffffu, tk, 0);
+      if (tk < total) sp = pl.list[tk / Hkv];
+    } else if (nstage == 2) {
+      if (tk < total) sp_ctx = a.context_lens[sp.x];
+    } else if (nstage == 3) {
+      nxt = Item{0, 0, 0, 0, 0, 0, 0, 0};
+      if (tk < total) {
+        int ctx = sp_ctx;  // clamped and flagged as checked_ctx does
+        if (ctx < 0 || ctx > a.max_context_len) {
+          if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
+          ctx = ctx < 0 ? 0 : a.max_context_len;
+        }
+        const int t0 = sp.y * P;
+        nxt.valid = 1;
+        nxt.s = sp.x;
+        nxt.kvh = (int)(tk % Hkv);
+        nxt.part = sp.y;
+        nxt.t1 = min(ctx, t0 + P);
+        nxt.c_begin = t0 / kSub;
+        nxt.nsub = (nxt.t1 + kSub - 1) / kSub - nxt.c_begin;
+        nxt.np = (ctx + P - 1) / P;
+      }
+      if (nxt.valid && lane < nxt.nsub)
+        load_sub_ids<BS>(a.block_tables + (int64_t)nxt.s * a.max_blocks_per_seq,
+                         nxt.c_begin + lane, nxt.t1, nxt_w);
+      else
+        empty_sub(nxt_w);
+    } else if (nstage == 4) {
+      if (nxt.valid && lane < nxt.nsub)
+        load_sub_params<KV, BS>(a, nxt.c_begin + lane, nxt.t1, nxt.kvh, nxt_w);
+      if (!dead) {  // the q buffer is free: the current item's fragments are in registers
+        copy_q(nxt);
+        nxt_q = true;
+      }
+    }
+    ++nstage;
+  };
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
-      if (pslot == 1 && (!nxt.valid || pk >= nxt.nsub)) break;
+      if (pslot == 1 && (nstage < kFetchDone || !nxt.valid || pk >= nxt.nsub)) break;
       const Item& v = pslot == 0 ? cur : nxt;
       const SubWin sw = shfl_sub<BS>(pslot == 0 ? cur_w : nxt_w, pk);
       const int stage = g_iss % NST;
@@ -1190,7 +1264,12 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf), G, lane,
                                            a.scale_log2, qf);
     __syncwarp();
-    if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
+    // the buffer is free once every lane holds its fragments (first item: nxt is resolved
+    // already; later ones issue it in the last fetch step)
+    if (!dead && nstage == kFetchDone && !nxt_q) {
+      copy_q(nxt);
+      nxt_q = true;
+    }
     w.reset();
     for (int i = 0; i < cur.nsub; ++i) {
       const SubWin sw = shfl_sub<BS>(cur_w, i);
@@ -1207,6 +1286,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       __syncwarp();
       ++g_cons;
       produce();
+      if (kStaged && nstage < kFetchDone) fetch_step();
     }
     // ---- item done: its output (single partition) or its partial ----
 #pragma unroll
@@ -1277,10 +1357,19 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       }
     }
     // ---- advance ----
-    cur = nxt;
-    cur_w = nxt_w;
-    nxt = fetch();
-    load_window(nxt, nxt_w);
+    if constexpr (kStaged) {
+      while (nstage < kFetchDone) fetch_step();  // a short item: finish the fetch here
+      cur = nxt;
+      cur_w = nxt_w;
+      nstage = 0;
+      fetch_step();  // the work ticket of the item after it
+    } else {
+      cur = nxt;
+      cur_w = nxt_w;
+      nxt = fetch();
+      load_window(nxt, nxt_w);
+    }
+    nxt_q = false;
     pslot = 0;
     produce();
   }
