@@ -18,7 +18,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 PIN_FILES = ["test_oracle_codecs.py", "test_oracle_facts.py", "test_oracle_paged.py",
              "test_oracle_attention.py", "test_oracle_prefill.py",
-             "test_oracle_hashes.py", "test_workloads_prefill.py"]
+             "test_oracle_hashes.py", "test_workloads_prefill.py", "test_workloads_decode.py"]
 
 # id -> (file under oracle/, text, replacement). The text must occur exactly once.
 MUTANTS = {
@@ -58,6 +58,8 @@ MUTANTS = {
                               "k_scales, v_scales, v_zeros, k_zeros)\n            for g in"),
     "prefill_state_zeros_swapped": ("flows.py", "state.k_zeros, state.v_zeros, seqs=seqs)",
                                     "state.v_zeros, state.k_zeros, seqs=seqs)"),
+    "state_tokens_shifted": ("flows.py", "ref_reshape_and_cache(k[:-1], v[:-1], kc, vc, pre[s],",
+                             "ref_reshape_and_cache(k[1:], v[1:], kc, vc, pre[s],"),
     # codecs
     "e4m3_bias_8": ("codecs.py", "2.0 ** (e - 7)", "2.0 ** (e - 8)"),
     "e4m3_subnormal_exponent": ("codecs.py", "2.0 ** (1 - 7)", "2.0 ** (0 - 7)"),
@@ -144,7 +146,8 @@ def _plant(dst, case):
 
 # the pins closest to each oracle file run first, so that a caught mistake stops early
 FIRST = {"attention.py": ["test_oracle_attention.py", "test_oracle_prefill.py"],
-         "flows.py": ["test_oracle_prefill.py", "test_oracle_attention.py"],
+         "flows.py": ["test_workloads_decode.py", "test_oracle_prefill.py",
+                      "test_oracle_attention.py"],
          "codecs.py": ["test_oracle_codecs.py"],
          "paged.py": ["test_oracle_paged.py", "test_oracle_hashes.py"],
          "facts.py": ["test_oracle_facts.py"]}
