@@ -123,6 +123,11 @@ struct DecodeArgs {
   int max_context_len;
   int final_pass;    // 1: one item covers the whole context, write out directly
   int skip_single;   // split path: single-partition sequences were written directly
+  // split path, warp workers: the warp that stores the last partial of a (sequence, kv
+  // head) merges its partitions itself (no reduce launch). arrive[s * Hkv + kvh] counts
+  // the partials stored so far; the plan kernel zeroes it.
+  int fused_merge;
+  uint32_t* arrive;  // [S][Hkv]
   pa_dtype q_dtype, out_dtype;
   // prefill rows (CUDA-core kernel only): work row s is new token s; the tokens of
   // sequence q are rows query_start[q] .. query_start[q+1]-1, the last ones of its context

@@ -509,11 +509,23 @@ struct SubWin {
   uint32_t z0, z1;     // int8: packed (K, V) zero points
 };
 
+// Sub-tile c's window entry in two steps, so that a caller can issue the block-table reads
+// and use them later: load_sub_ids reads the raw block ids, load_sub_params checks them and
+// reads the blocks' scales (and zero points). Both steps together are load_sub.
+template <int BS>
+__device__ __forceinline__ void load_sub_ids(const int32_t* btrow, int c, int t1, SubWin& w) {
+  if constexpr (BS == 8) {
+    w.p0 = btrow[2 * c];
+    w.p1 = c * kSub + 8 < t1 ? btrow[2 * c + 1] : -3;  // -3: second half absent
+  } else {
+    w.p0 = btrow[c * kSub / BS];
+  }
+}
+
 template <pa_dtype KV, int BS>
-__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
-                                         int t1, int kvh, SubWin& w) {
-  auto one = [&](int blk, int& p, float& ks, float& vs, uint32_t& z) {
-    p = btrow[blk];
+__device__ __forceinline__ void load_sub_params(const DecodeArgs& a, int c, int t1, int kvh,
+                                                SubWin& w) {
+  auto one = [&](int& p, float& ks, float& vs, uint32_t& z) {
     ks = 1.f;
     vs = 1.f;
     z = 0;
@@ -530,16 +542,23 @@ __device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btr
     }
   };
   if constexpr (BS == 8) {
-    one(2 * c, w.p0, w.ks0, w.vs0, w.z0);
+    one(w.p0, w.ks0, w.vs0, w.z0);
     if (c * kSub + 8 < t1) {
-      one(2 * c + 1, w.p1, w.ks1, w.vs1, w.z1);
+      one(w.p1, w.ks1, w.vs1, w.z1);
     } else {
       w.p1 = -3; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
     }
   } else {
-    one(c * kSub / BS, w.p0, w.ks0, w.vs0, w.z0);
+    one(w.p0, w.ks0, w.vs0, w.z0);
     w.p1 = w.p0; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
   }
+}
+
+template <pa_dtype KV, int BS>
+__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
+                                         int t1, int kvh, SubWin& w) {
+  load_sub_ids<BS>(btrow, c, t1, w);
+  load_sub_params<KV, BS>(a, c, t1, kvh, w);
 }
 
 __device__ __forceinline__ void empty_sub(SubWin& w) {
@@ -730,14 +749,17 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
 }
 
 // =======================================================================================
-// Split path: plan kernel + persistent kernels; lse_reduce_kernel merges the partitions.
+// Split path: plan kernel + persistent kernels; the partitions are merged by the warp
+// workers themselves (rows of up to 32 partitions) or by lse_reduce_kernel afterwards.
 // =======================================================================================
 // Workspace of the split path (offsets in bytes, each region 256-aligned):
 //   [0]     uint32 fetch counter, uint32 total items
 //   list    int2 (seq, partition) per partition item, largest items first
 //   m, l    float [S][Hq][P];  acc float [S][Hq][P][kD]   (partials, as the CUDA-core path)
-// Sequences with a single partition are written to `out` directly; the others are merged
-// by lse_reduce_kernel afterwards (spread over every (seq, q head)).
+//   arrive  uint32 [S][Hkv]: partials stored so far (warp workers merging in place)
+// Sequences with a single partition are written to `out` directly. The others are merged
+// by the warp that stores their last partial (warp workers, P <= 32), else by
+// lse_reduce_kernel afterwards (spread over every (seq, q head)).
 struct PlanView {
   uint32_t* counters;  // [0] fetch, [1] total
   int2* list;
@@ -745,7 +767,8 @@ struct PlanView {
 
 // One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
 // largest first (full partitions, then partial ones by size), writes the list, zeroes the
-// fetch counter, and writes out = 0 / lse = -inf for empty sequences.
+// fetch counter (and the arrival counters of the merging warp workers), and writes
+// out = 0 / lse = -inf for empty sequences.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
   __shared__ int cnt[130], off[130];
   pdl_wait();
@@ -753,6 +776,9 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   const int P = a.part_tokens;
   const int nbk = P / kSub;  // sub-tiles of a full partition (<= 128)
   for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
+  if (a.fused_merge)
+    for (int64_t i = threadIdx.x; i < (int64_t)a.num_seqs * a.num_kv_heads; i += blockDim.x)
+      a.arrive[i] = 0u;
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int ctx = checked_ctx(a, s);
@@ -787,6 +813,49 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
     }
     if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
+  }
+}
+
+// Merge of the partitions of the G query rows row0 .. row0+G-1 (one (sequence, kv head)),
+// run by the warp that stored the last of their partials; np <= 32. Lane p holds
+// partition p's running max and sum, lane k owns channel quad k (4 k .. 4 k + 3):
+// M = max_p m_p, L = sum_p 2^(m_p - M) l_p, out = sum_p 2^(m_p - M) acc_p / L. The
+// arithmetic and its order are those of lse_reduce_kernel, so the result does not depend
+// on which warp merges. Partials are read through L2 (ld.global.cg): other SMs wrote them
+// during this launch.
+__device__ __forceinline__ void merge_rows(const DecodeArgs& a, int64_t row0, int G, int np,
+                                           int lane) {
+  static_assert(kD == 128, "one channel quad per lane");
+  for (int g = 0; g < G; ++g) {
+    const int64_t row = row0 + g;
+    const float* pm = a.part_m + row * a.max_parts;
+    const float* pl = a.part_l + row * a.max_parts;
+    const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * kD);
+    const float mp = lane < np ? __ldcg(pm + lane) : -INFINITY;
+    float M = mp;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    const float w = (lane < np && M != -INFINITY) ? fast_exp2(mp - M) : 0.f;
+    float lsum = 0.f;
+    if (lane < np) lsum = fmaf(w, __ldcg(pl + lane), lsum);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+    for (int k = 0; k < np; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, k);
+      const float4 v = __ldcg(pacc + (int64_t)k * (kD / 4) + lane);
+      acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
+      acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
+    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+    const int64_t o = row * kD + 4 * lane;
+    store_out(a.out, a.out_dtype, o, acc.x * inv);
+    store_out(a.out, a.out_dtype, o + 1, acc.y * inv);
+    store_out(a.out, a.out_dtype, o + 2, acc.z * inv);
+    store_out(a.out, a.out_dtype, o + 3, acc.w * inv);
+    if (lane == 0 && a.lse_out != nullptr)
+      a.lse_out[row] = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
   }
 }
 
@@ -1109,10 +1178,65 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   int pslot = 0, pk = 0;
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
+  // From the second item on, the item after the current one is fetched in kFetchDone
+  // steps, one per consumed sub-tile. Each step uses only values that a global read issued
+  // one step earlier returns (work ticket, list entry, context length, block ids), so the
+  // reads overlap the current item's tiles instead of stalling the warp between items.
+  // An item shorter than that finishes the fetch at its end.
+  constexpr int kFetchDone = 5;
+  // int8 caches with 8-token blocks keep the fetch in one piece at the item boundary: the
+  // staged form would make that variant spill
+  constexpr bool kStaged = !(KV == PA_INT8 && BS == 8);
+  int nstage = kFetchDone;  // nxt and nxt_w are resolved
+  bool nxt_q = false;       // nxt's q copy is issued
+  uint32_t tk = 0;          // work ticket (lane 0 until broadcast)
+  int2 sp = make_int2(0, 0);
+  int sp_ctx = 0;
+  auto fetch_step = [&]() {
+    if (nstage == 0) {
+      if (lane == 0) tk = atomicAdd(&pl.counters[0], 1u);
+    } else if (nstage == 1) {
+      tk = __shfl_sync(0xffffffffu, tk, 0);
+      if (tk < total) sp = pl.list[tk / Hkv];
+    } else if (nstage == 2) {
+      if (tk < total) sp_ctx = a.context_lens[sp.x];
+    } else if (nstage == 3) {
+      nxt = Item{0, 0, 0, 0, 0, 0, 0, 0};
+      if (tk < total) {
+        int ctx = sp_ctx;  // clamped and flagged as checked_ctx does
+        if (ctx < 0 || ctx > a.max_context_len) {
+          if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
+          ctx = ctx < 0 ? 0 : a.max_context_len;
+        }
+        const int t0 = sp.y * P;
+        nxt.valid = 1;
+        nxt.s = sp.x;
+        nxt.kvh = (int)(tk % Hkv);
+        nxt.part = sp.y;
+        nxt.t1 = min(ctx, t0 + P);
+        nxt.c_begin = t0 / kSub;
+        nxt.nsub = (nxt.t1 + kSub - 1) / kSub - nxt.c_begin;
+        nxt.np = (ctx + P - 1) / P;
+      }
+      if (nxt.valid && lane < nxt.nsub)
+        load_sub_ids<BS>(a.block_tables + (int64_t)nxt.s * a.max_blocks_per_seq,
+                         nxt.c_begin + lane, nxt.t1, nxt_w);
+      else
+        empty_sub(nxt_w);
+    } else if (nstage == 4) {
+      if (nxt.valid && lane < nxt.nsub)
+        load_sub_params<KV, BS>(a, nxt.c_begin + lane, nxt.t1, nxt.kvh, nxt_w);
+      if (!dead) {  // the q buffer is free: the current item's fragments are in registers
+        copy_q(nxt);
+        nxt_q = true;
+      }
+    }
+    ++nstage;
+  };
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
-      if (pslot == 1 && (!nxt.valid || pk >= nxt.nsub)) break;
+      if (pslot == 1 && (nstage < kFetchDone || !nxt.valid || pk >= nxt.nsub)) break;
       const Item& v = pslot == 0 ? cur : nxt;
       const SubWin sw = shfl_sub<BS>(pslot == 0 ? cur_w : nxt_w, pk);
       const int stage = g_iss % NST;
@@ -1140,7 +1264,12 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf), G, lane,
                                            a.scale_log2, qf);
     __syncwarp();
-    if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
+    // the buffer is free once every lane holds its fragments (first item: nxt is resolved
+    // already; later ones issue it in the last fetch step)
+    if (!dead && nstage == kFetchDone && !nxt_q) {
+      copy_q(nxt);
+      nxt_q = true;
+    }
     w.reset();
     for (int i = 0; i < cur.nsub; ++i) {
       const SubWin sw = shfl_sub<BS>(cur_w, i);
@@ -1157,6 +1286,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       __syncwarp();
       ++g_cons;
       produce();
+      if (kStaged && nstage < kFetchDone) fetch_step();
     }
     // ---- item done: its output (single partition) or its partial ----
 #pragma unroll
@@ -1210,11 +1340,36 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
         }
       }
     }
+    // ---- the last partial of a (sequence, kv head) to be stored merges them all ----
+    if (cur.np > 1 && a.fused_merge) {
+      __threadfence();  // this lane's partial stores, before the arrival below
+      __syncwarp();
+      uint32_t prev = 0;
+      if (lane == 0) {
+        __threadfence();
+        prev = atomicAdd(a.arrive + (int64_t)cur.s * Hkv + cur.kvh, 1u);
+      }
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev == (uint32_t)cur.np - 1) {
+        __threadfence();  // the other partials, stored before their arrivals, are visible
+        __syncwarp();
+        merge_rows(a, row0, G, cur.np, lane);
+      }
+    }
     // ---- advance ----
-    cur = nxt;
-    cur_w = nxt_w;
-    nxt = fetch();
-    load_window(nxt, nxt_w);
+    if constexpr (kStaged) {
+      while (nstage < kFetchDone) fetch_step();  // a short item: finish the fetch here
+      cur = nxt;
+      cur_w = nxt_w;
+      nstage = 0;
+      fetch_step();  // the work ticket of the item after it
+    } else {
+      cur = nxt;
+      cur_w = nxt_w;
+      nxt = fetch();
+      load_window(nxt, nxt_w);
+    }
+    nxt_q = false;
     pslot = 0;
     produce();
   }

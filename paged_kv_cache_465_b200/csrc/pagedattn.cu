@@ -21,7 +21,7 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Split-path workspace: plan area (counters, item list) followed by the partials
 // (m, l, acc) of every (seq, q head, partition).
 struct WorkspaceLayout {
-  size_t cnt_off, list_off, m_off, l_off, acc_off, total;
+  size_t cnt_off, list_off, m_off, l_off, acc_off, arr_off, total;
   int parts;
 };
 
@@ -49,7 +49,7 @@ bool desc_supported(const pa_decode_desc* d) {
 }
 
 WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
-  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0};
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0, 0};
   if (d->partition_size == 0 || max_context_len <= 0) return w;
   w.parts = (max_context_len + d->partition_size - 1) / d->partition_size;
   const size_t rows = (size_t)d->num_seqs * d->num_q_heads * w.parts;
@@ -58,7 +58,8 @@ WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
   w.m_off = w.list_off + round_up((size_t)d->num_seqs * w.parts * 8, 256);
   w.l_off = w.m_off + round_up(rows * sizeof(float), 256);
   w.acc_off = w.l_off + round_up(rows * sizeof(float), 256);
-  w.total = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
+  w.arr_off = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
+  w.total = w.arr_off + round_up((size_t)d->num_seqs * d->num_kv_heads * sizeof(uint32_t), 256);
   return w;
 }
 
@@ -121,7 +122,7 @@ using namespace pa;
 
 extern "C" {
 
-const char* pa_version(void) { return "pagedattn 0.3 sm_100a"; }
+const char* pa_version(void) { return "pagedattn 0.4 sm_100a"; }
 
 pa_status pa_set_decode_impl(int impl) {
   if (impl < 0 || impl > 5) return PA_ERR_INVALID;
@@ -195,6 +196,11 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
       pl.counters = reinterpret_cast<uint32_t*>(ws + wl.cnt_off);
       pl.list = reinterpret_cast<int2*>(ws + wl.list_off);
       a.skip_single = 1;  // single-partition sequences are written by the kernel itself
+      // warp workers merge rows of up to 32 partitions themselves (one lane per partition)
+      if (kind == tc::kTcWarps && wl.parts <= 32) {
+        a.fused_merge = 1;
+        a.arrive = reinterpret_cast<uint32_t*>(ws + wl.arr_off);
+      }
     }
     e = launch_tc(a, desc, grid, kind == tc::kTcGrid ? nullptr : &pl, kind, st);
   } else {
@@ -206,7 +212,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     }
   }
   if (e != cudaSuccess) return PA_ERR_CUDA;
-  if (split && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
+  if (split && !a.fused_merge && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 

@@ -85,6 +85,103 @@ def test_reshape_and_cache_bitexact(pa, in_dt, cache_dt, d):
     assert np.array_equal(cache_codes(vc), vref)
 
 
+def _fp8_write(pa, x, in_dt, scales, B=16, d=128):
+    """Writes x [T, 1, d] (T a multiple of B) through reshape_and_cache into an fp8 cache,
+    token t into slot t, and returns the GPU's codes and the oracle's."""
+    T = x.shape[0]
+    NB = T // B
+    slots = np.arange(T, dtype=np.int64)
+    kref = opaged.new_cache(NB, 1, B, d, "fp8")
+    vref = opaged.new_cache(NB, 1, B, d, "fp8")
+    opaged.ref_reshape_and_cache(x, x, kref, vref, slots, in_dt, "fp8", scales, scales)
+    src = torch.from_numpy(x)
+    if in_dt == "bf16":
+        src = src.view(torch.int16).view(torch.bfloat16)
+    k = src.cuda()
+    kc = torch.zeros((NB, 1, B, d), dtype=torch.uint8, device="cuda")
+    vc = torch.zeros_like(kc)
+    sc = torch.from_numpy(scales).cuda()
+    pa.reshape_and_cache(k, k, kc, vc, torch.from_numpy(slots).cuda(), k_scales=sc, v_scales=sc)
+    assert pa.device_error() == 0
+    return cache_codes(kc), kref
+
+
+def _same_codes(got, ref):
+    """Equal codes, except that a NaN may be either NaN pattern (S.1111.111)."""
+    nan = (ref & 0x7F) == 0x7F
+    assert np.array_equal(got[~nan], ref[~nan])
+    assert np.all((got[nan] & 0x7F) == 0x7F)
+
+
+def test_fp8_write_every_bf16_value(pa):
+    """All 65536 bf16 bit patterns (zeros, subnormals, normals, infinities, NaNs) through the
+    fp8 cache write, with power-of-two and other block scales."""
+    x = np.arange(65536, dtype=np.uint32).astype(np.uint16).reshape(512, 1, 128)
+    scales = np.array([[1.0], [0.5], [2.0 ** -8], [3.0], [0.37], [2.0 ** 6], [1e-3], [7.25]] * 4,
+                      np.float32)
+    got, ref = _fp8_write(pa, x, "bf16", scales)
+    _same_codes(got, ref)
+
+
+def test_fp8_write_rounding_midpoints(pa):
+    """float32 inputs at every midpoint between adjacent E4M3 magnitudes (ties to even), one
+    float32 step either side of it, past the largest finite value (saturation), and the
+    specials; block scales 1 and 2^-3 (x / scale exact), 0.3 (rounded division)."""
+    mags = codecs.E4M3_TABLE[:127]
+    mids = ((mags[1:] + mags[:-1]) / 2).astype(np.float32)
+    vals = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e9)),
+                           mags.astype(np.float32),
+                           np.array([448, 460, 464, 464.0001, 480, 1e30, np.inf, np.nan, 0.0,
+                                     1e-45, 2.0 ** -10, 3 * 2.0 ** -10], np.float32)])
+    vals = np.concatenate([vals, -vals]).astype(np.float32)
+    per = 16 * 128
+    n_blocks = -(-vals.size // per)
+    x = np.zeros(n_blocks * per, np.float32)
+    x[:vals.size] = vals
+    for sc in (1.0, 0.125, 0.3):
+        scales = np.full((n_blocks, 1), sc, np.float32)
+        got, ref = _fp8_write(pa, (x * np.float32(sc)).astype(np.float32).reshape(-1, 1, 128),
+                              "f32", scales)
+        _same_codes(got, ref)
+
+
+def test_int8_write_ties_and_clipping(pa):
+    """int8 cache write at every half-integer x / scale in [-200, 200] (ties to even before
+    the zero point is added), one float32 step either side, and values past the byte's
+    range, with several zero points and scales (1 and 0.5 keep x / scale exact)."""
+    B, d = 16, 128
+    base = np.arange(-200, 200, dtype=np.float64) + 0.5
+    vals = np.concatenate([base, np.nextafter(base.astype(np.float32), np.float32(-1e9)),
+                           np.nextafter(base.astype(np.float32), np.float32(1e9)),
+                           np.array([0.0, -0.0, 1e9, -1e9, 127.5, -128.5, 127.49998], np.float32)])
+    vals = vals.astype(np.float32)
+    per = B * d
+    NB = -(-vals.size // per) * 4
+    x = np.zeros((NB * per,), np.float32)
+    reps = NB // (-(-vals.size // per))
+    for r in range(reps):
+        x[r * (NB // reps) * per: r * (NB // reps) * per + vals.size] = vals
+    zeros = np.array([[0], [7], [-30], [100]] * (NB // 4), np.int32)[:NB]
+    for sc in (1.0, 0.5):
+        scales = np.full((NB, 1), sc, np.float32)
+        xs = (x * np.float32(sc)).astype(np.float32).reshape(-1, 1, d)
+        T = xs.shape[0]
+        slots = np.arange(T, dtype=np.int64)
+        kref = opaged.new_cache(NB, 1, B, d, "int8")
+        vref = opaged.new_cache(NB, 1, B, d, "int8")
+        opaged.ref_reshape_and_cache(xs, xs, kref, vref, slots, "f32", "int8", scales, scales,
+                                     zeros, zeros)
+        k = torch.from_numpy(xs).cuda()
+        kc = torch.zeros((NB, 1, B, d), dtype=torch.int8, device="cuda")
+        vc = torch.zeros_like(kc)
+        s_d = torch.from_numpy(scales).cuda()
+        z_d = torch.from_numpy(zeros).cuda()
+        pa.reshape_and_cache(k, k, kc, vc, torch.from_numpy(slots).cuda(), k_scales=s_d,
+                             v_scales=s_d, k_zeros=z_d, v_zeros=z_d)
+        assert pa.device_error() == 0
+        assert np.array_equal(cache_codes(kc), kref)
+
+
 @pytest.mark.parametrize("cache_dt", ["f32", "bf16", "fp8", "int8"])
 def test_copy_blocks_bitexact(pa, cache_dt):
     rng = np.random.default_rng(5)
