@@ -34,7 +34,10 @@
  *   ([KVPaged] "KV quantization: FP8 and INT8": one byte per element with a scale and a
  *   zero point) carry the same scales plus int32 zero points[num_blocks][num_kv_heads]:
  *   stored code = clamp(round_half_even(x / scale) + zero, -128, 127), value =
- *   (code - zero) * scale.
+ *   (code - zero) * scale. Zero points must lie in [-128, 127], the byte's own range
+ *   (an affine int8 code needs no other); there code - zero is exact in every kernel. A
+ *   block whose K or V zero point lies outside is treated like a bad block id: attention
+ *   skips it and the cache write skips its rows, and PA_DEVERR_ZERO is recorded.
  * - q and out: [num_seqs][num_q_heads][head_dim] row-major. Query head h reads kv head
  *   h / (num_q_heads / num_kv_heads) ([KVPaged] "GQA and MQA": query heads are grouped and
  *   each group shares one KV head).
@@ -82,6 +85,17 @@ typedef enum {
 #define PA_DEVERR_TIMEOUT 0x10   /* a bounded wait on an asynchronous copy gave up      */
 #define PA_DEVERR_QUERY 0x20     /* prefill query_start not ascending, past num_tokens, */
                                  /* or more new tokens than context (or max_query_len)  */
+#define PA_DEVERR_ZERO 0x40      /* int8 zero point outside [-128, 127]                 */
+
+/*
+ * partition_size value that lets the library choose the split for a decode call: the
+ * largest of 512, 256, 128 and 64 tokens that gives at least two work items per resident
+ * warp worker of the device (2 x SMs x 16) if every sequence were max_context_len long,
+ * else 64; one pass (0) when max_context_len <= 64. The choice depends only on num_seqs,
+ * num_kv_heads, max_context_len and the SM count, so results stay independent of where
+ * blocks sit; paged_attn_partition_size() reports it.
+ */
+#define PA_PARTITION_AUTO (-1)
 
 /* Shape and dtypes of one paged decode-attention call. */
 typedef struct {
@@ -94,7 +108,8 @@ typedef struct {
   int num_blocks;          /* physical blocks in the pool (bounds check)               */
   int partition_size;      /* split-KV partition in tokens, a multiple of block_size   */
                            /* and of 16;                                               */
-                           /* 0 = one pass over the whole context per (seq, kv head)   */
+                           /* 0 = one pass over the whole context per (seq, kv head);  */
+                           /* PA_PARTITION_AUTO = the library's choice (below)         */
   pa_dtype q_dtype, kv_dtype, out_dtype;
 } pa_decode_desc;
 
@@ -104,6 +119,22 @@ typedef struct {
  * descriptor as well; paged_attn_decode then reports the error.
  */
 size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len);
+
+/*
+ * The partition (tokens; 0 = one pass) a paged_attn_decode call with this descriptor uses:
+ * desc->partition_size itself, or the library's choice for PA_PARTITION_AUTO. -1 for an
+ * invalid descriptor.
+ */
+int paged_attn_partition_size(const pa_decode_desc* desc, int max_context_len);
+
+/*
+ * Number of kernel launches one paged_attn_decode call with this descriptor makes under
+ * the current pa_set_decode_impl choice (0 for an invalid, unsupported or empty call):
+ * the plan kernel of the persistent tensor-core kernels, the attention kernel, and the
+ * log-sum-exp reduce when the split path's partitions are not merged in place. For
+ * callers that count launches (profiling, launch budgets).
+ */
+int paged_attn_decode_launches(const pa_decode_desc* desc, int max_context_len);
 
 /*
  * Decode attention over the paged cache ([KVPaged] "Core principle: what is the KV cache":
@@ -180,18 +211,20 @@ pa_status paged_attn_prefill(const void* q, const void* k_cache, const void* v_c
 
 /*
  * paged_attn_decode for callers that cannot allocate device memory. Some callers may not
- * call cudaMalloc at all: code running while a stream is being captured, a plugin inside a
- * host runtime that owns every device allocation through its own allocator, a caller with
- * no workspace argument to forward. This entry point takes the same arguments as
- * paged_attn_decode minus the workspace and computes the same result; the split-KV scratch
- * comes from one fixed array compiled into this library (PA_NOALLOC_SCRATCH_BYTES per GPU,
- * held by every GPU that loads the library until the process exits). The pages have no
- * counterpart of this call; it exists only for such callers.
+ * call cudaMalloc at all: a plugin inside a host runtime that owns every device allocation
+ * through its own allocator, a caller with no workspace argument to forward, a latency-
+ * bound loop that must not risk cudaMalloc's implicit device synchronisation. This entry
+ * point takes the same arguments as paged_attn_decode minus the workspace and computes the
+ * same result, bit for bit; the split-KV scratch comes from one fixed array compiled into
+ * this library (PA_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU that loads the library
+ * until the process exits). The pages have no counterpart of this call; it exists only for
+ * such callers.
  * - Calls that need more scratch than PA_NOALLOC_SCRATCH_BYTES
  *   (paged_attn_workspace_size(desc, max_context_len) larger than it) return
  *   PA_ERR_WORKSPACE and enqueue nothing.
- * - The first call on a device looks the array's device address up (once per device, with
- *   that device current); make that first call before any stream capture.
+ * - The first call on a device, whatever its shape, looks the array's device address up
+ *   (once per device, with that device current); make that first call before any stream
+ *   capture.
  * - It calls no cudaMalloc, cudaFree or other allocating routine.
  * - Every call on a device shares the one array, which keeps the last call's contents. The
  *   kernels re-initialise what they read (work counter, partials) on every call, so stale

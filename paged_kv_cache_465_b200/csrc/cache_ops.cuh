@@ -76,6 +76,10 @@ __global__ void reshape_and_cache_kernel(const void* __restrict__ k, const void*
       const int64_t sh = blk * num_kv_heads + h;
       const float s = (is_v ? v_scales : k_scales)[sh];
       const int z = (is_v ? v_zeros : k_zeros)[sh];
+      if (!zero_in_range(z)) {  // the row is not written
+        flag_error(PA_DEVERR_ZERO);
+        continue;
+      }
       uint32_t w[2] = {0u, 0u};
 #pragma unroll
       for (int j = 0; j < 8; ++j) {

@@ -19,6 +19,11 @@ __device__ unsigned int g_error_word;
 
 __device__ __forceinline__ void flag_error(unsigned int bits) { atomicOr(&g_error_word, bits); }
 
+// int8 zero points must lie in the byte's range: only there is code - zero exact in every
+// kernel's arithmetic (f16 and bf16 operands of the tensor-core paths). A block whose
+// zero point is outside is skipped like a bad block id and PA_DEVERR_ZERO recorded.
+__device__ __forceinline__ bool zero_in_range(int z) { return z >= -128 && z <= 127; }
+
 // ---------------------------------------------------------------------------------------
 // Conversions. Each is one documented PTX conversion instruction.
 // ---------------------------------------------------------------------------------------

@@ -266,8 +266,14 @@ decode_simt_kernel(const DecodeArgs a) {
           vs = a.v_scales[bh];
         }
         if constexpr (KV == PA_INT8) {
-          kz = (float)a.k_zeros[bh];
-          vz = (float)a.v_zeros[bh];
+          const int kzi = a.k_zeros[bh], vzi = a.v_zeros[bh];
+          if (!zero_in_range(kzi) || !zero_in_range(vzi)) {  // the block is skipped
+            if (half == 0) flag_error(PA_DEVERR_ZERO);
+            valid = false;
+            row = -1;
+          }
+          kz = (float)kzi;
+          vz = (float)vzi;
         }
       }
     }

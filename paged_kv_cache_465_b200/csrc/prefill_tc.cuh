@@ -322,6 +322,16 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + 8 * kNumBars);
   volatile int* dead = reinterpret_cast<volatile int*>(tmem_slot + 1);
   const int32_t* bt = a.block_tables + (int64_t)s * a.max_blocks_per_seq;
+  // a block the kernel cannot use: id out of range, or (int8) a zero point outside the
+  // byte's range; such blocks are skipped (not loaded, their keys masked)
+  auto block_bad = [&](int p) {
+    if (p < 0 || p >= a.num_blocks) return true;
+    if constexpr (KV == PA_INT8) {
+      const int64_t bh = (int64_t)p * a.num_kv_heads + kvh;
+      return !zero_in_range(a.k_zeros[bh]) || !zero_in_range(a.v_zeros[bh]);
+    }
+    return false;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kNumBars; ++i) {
@@ -344,10 +354,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
   // any block id out of range among the keys the CTA sees? (then tiles are checked one by
   // one; otherwise no per-tile checks)
   int bad = 0;
-  for (int b = threadIdx.x; b < (kv_end + BS - 1) / BS; b += kThreads) {
-    const int p = bt[b];
-    bad |= p < 0 || p >= a.num_blocks;
-  }
+  for (int b = threadIdx.x; b < (kv_end + BS - 1) / BS; b += kThreads) bad |= block_bad(bt[b]);
   tc_fence_before();
   const bool any_bad = __syncthreads_or(bad) != 0;
   tc_fence_after();
@@ -373,6 +380,9 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
         p = bt[j * NB_T + lane];
         if (p < 0 || p >= a.num_blocks) {
           flag_error(PA_DEVERR_BLOCK_ID);
+          p = -1;
+        } else if (block_bad(p)) {
+          flag_error(PA_DEVERR_ZERO);
           p = -1;
         }
       }
@@ -634,10 +644,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       uint32_t badm = 0;  // blocks of the tile with an out-of-range id (skipped, masked)
       if (any_bad) {
         bool b = false;
-        if (lane < (vlim + BS - 1) / BS) {
-          const int p = bt[t0 / BS + lane];
-          b = p < 0 || p >= a.num_blocks;
-        }
+        if (lane < (vlim + BS - 1) / BS) b = block_bad(bt[t0 / BS + lane]);
         badm = __ballot_sync(0xffffffffu, b);
       }
       const uint32_t sbuf = lane_addr;  // the query tile's S buffer
@@ -855,7 +862,7 @@ inline cudaError_t launch_bs(const PrefillArgs& a, const void* q, const void* kc
                         : make_kv8_map(&km, kc, rows, BS) && make_kv8_map(&vm, vc, rows, BS);
   if (!maps || !make_q_map(&qm, q, a.num_tokens, a.num_q_heads, a.group))
     return cudaErrorInvalidValue;
-  static int slots[tc::kMaxDevices] = {};
+  static tc::DeviceCache slots;
   int per_sm = 0;
   const cudaError_t e =
       tc::resident_per_sm(prefill_tc_kernel<BS, KV>, L::kThreads, L::kSmem, slots, &per_sm);
