@@ -34,6 +34,7 @@ PA_OK, PA_ERR_INVALID, PA_ERR_UNSUPPORTED, PA_ERR_CUDA, PA_ERR_NO_BLOCKS, PA_ERR
 PA_DEVERR_BLOCK_ID, PA_DEVERR_SLOT, PA_DEVERR_PAIR, PA_DEVERR_CONTEXT, PA_DEVERR_TIMEOUT = \
     0x1, 0x2, 0x4, 0x8, 0x10
 PA_DEVERR_QUERY = 0x20
+PA_DEVERR_ZERO = 0x40
 _STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID", -2: "PA_ERR_UNSUPPORTED", -3: "PA_ERR_CUDA",
            -4: "PA_ERR_NO_BLOCKS", -5: "PA_ERR_WORKSPACE", -6: "PA_ERR_DEVICE"}
 
@@ -62,6 +63,8 @@ _P = ctypes.POINTER
 _SIGS = {
     "pa_version": (ctypes.c_char_p, []),
     "paged_attn_workspace_size": (_sz, [_P(pa_decode_desc), _i]),
+    "paged_attn_decode_launches": (_i, [_P(pa_decode_desc), _i]),
+    "paged_attn_partition_size": (_i, [_P(pa_decode_desc), _i]),
     "paged_attn_decode": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i, _vp,
                                _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "paged_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _f, _vp, _P(pa_decode_desc), _i,
@@ -169,6 +172,19 @@ def make_desc(num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
 
 def workspace_size(desc: pa_decode_desc, max_context_len: int) -> int:
     return int(_lib.paged_attn_workspace_size(ctypes.byref(desc), int(max_context_len)))
+
+
+PARTITION_AUTO = -1  # partition_size: the library chooses the split (PA_PARTITION_AUTO)
+
+
+def partition_size_for(desc: pa_decode_desc, max_context_len: int) -> int:
+    """The partition (tokens, 0 = one pass) a decode call with this descriptor uses."""
+    return int(_lib.paged_attn_partition_size(ctypes.byref(desc), int(max_context_len)))
+
+
+def decode_launches(desc: pa_decode_desc, max_context_len: int) -> int:
+    """Kernel launches of one paged_attn_decode call with this descriptor (current impl)."""
+    return int(_lib.paged_attn_decode_launches(ctypes.byref(desc), int(max_context_len)))
 
 
 def decode_desc_for(q, k_cache, block_tables, partition_size: int) -> pa_decode_desc:

@@ -37,6 +37,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
 #include <type_traits>
 
 #include "decode_simt.cuh"
@@ -45,8 +46,9 @@ namespace pa {
 
 // 0 = automatic, 1 = CUDA-core path only, 2 = tensor cores where supported (automatic
 // kernel choice), 3 / 4 / 5 = tensor cores with the grid / persistent-CTA / warp-worker
-// kernel where the shape allows it (see tc_kind).
-static int g_decode_impl = 0;
+// kernel where the shape allows it (see tc_kind). Atomic: calls on other host threads read
+// it while pa_set_decode_impl writes it.
+static std::atomic<int> g_decode_impl{0};
 
 // Stage depth of the persistent kernel's per-warp rings (blocks in flight per warp).
 #ifndef PA_TC_PSTAGE_BF16
@@ -538,7 +540,15 @@ __device__ __forceinline__ void load_sub_params(const DecodeArgs& a, int c, int 
       const int64_t bh = (int64_t)p * a.num_kv_heads + kvh;
       ks = a.k_scales[bh];
       vs = a.v_scales[bh];
-      if constexpr (KV == PA_INT8) z = pack_zeros(a.k_zeros[bh], a.v_zeros[bh]);
+      if constexpr (KV == PA_INT8) {
+        const int kz = a.k_zeros[bh], vz = a.v_zeros[bh];
+        if (!zero_in_range(kz) || !zero_in_range(vz)) {
+          flag_error(PA_DEVERR_ZERO);
+          p = -1;
+          return;
+        }
+        z = pack_zeros(kz, vz);
+      }
     }
   };
   if constexpr (BS == 8) {
@@ -949,8 +959,15 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
       } else if constexpr (FP8) {
         ks = a.k_scales[(int64_t)p * Hkv + v.kvh];
         vs = a.v_scales[(int64_t)p * Hkv + v.kvh];
-        if constexpr (KV == PA_INT8)
-          z = pack_zeros(a.k_zeros[(int64_t)p * Hkv + v.kvh], a.v_zeros[(int64_t)p * Hkv + v.kvh]);
+        if constexpr (KV == PA_INT8) {
+          const int kz = a.k_zeros[(int64_t)p * Hkv + v.kvh];
+          const int vz = a.v_zeros[(int64_t)p * Hkv + v.kvh];
+          if (!zero_in_range(kz) || !zero_in_range(vz)) {
+            flag_error(PA_DEVERR_ZERO);
+            p = -1;
+          }
+          z = pack_zeros(kz, vz);
+        }
       }
     }
   };
@@ -1084,6 +1101,9 @@ constexpr int kWW = PA_TCW_WARPS;
 #ifndef PA_TCW_MIN_WARPS
 #define PA_TCW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
 #endif
+#ifndef PA_TCW_STAGED_FETCH
+#define PA_TCW_STAGED_FETCH 1  // 1: the next item is fetched in steps behind the current one
+#endif
 
 template <pa_dtype KV>
 struct TcwCfg {
@@ -1186,7 +1206,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   constexpr int kFetchDone = 5;
   // int8 caches with 8-token blocks keep the fetch in one piece at the item boundary: the
   // staged form would make that variant spill
-  constexpr bool kStaged = !(KV == PA_INT8 && BS == 8);
+  constexpr bool kStaged = PA_TCW_STAGED_FETCH && !(KV == PA_INT8 && BS == 8);
   int nstage = kFetchDone;  // nxt and nxt_w are resolved
   bool nxt_q = false;       // nxt's q copy is issued
   uint32_t tk = 0;          // work ticket (lane 0 until broadcast)
@@ -1385,18 +1405,18 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
 // ---------------------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------------------
+// The driver's tensor-map encoder, looked up once (a function-local static is initialised
+// once even when several host threads make their first call together).
 inline PFN_cuTensorMapEncodeTiled_v12000 encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static bool tried = false;
-  if (!tried) {
-    tried = true;
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
             cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+  }();
   return fn;
 }
 
@@ -1421,16 +1441,18 @@ inline bool make_map(CUtensorMap* m, const void* base, int64_t total_rows, pa_dt
 
 constexpr int kMaxDevices = 64;  // per-device caches of the launch set-up
 
+// Per-device cache entries are atomics: first calls on several host threads may fill the
+// same entry at once (with the same value), and later calls read it without a lock.
+using DeviceCache = std::atomic<int>[kMaxDevices];
+
 inline int sm_count() {
-  static int cache[kMaxDevices] = {};
+  static DeviceCache cache;  // static storage: zero-initialised
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
-  if (cache[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
-      cache[dev] = n;
-  }
-  return cache[dev];
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0 && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess)
+    cache[dev].store(n, std::memory_order_relaxed);
+  return n;
 }
 
 // Tensor-core kernel families: grid of one CTA per item, persistent CTAs sharing an item,
@@ -1448,21 +1470,21 @@ inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
 
 // Launch set-up of one kernel on the current device: its dynamic shared-memory limit is
 // raised and its resident CTAs per SM measured once per device the process uses (`slots`
-// is the kernel's per-device cache; concurrent first calls write the same values).
+// is the kernel's per-device cache; concurrent first calls store the same values).
 template <typename K>
-inline cudaError_t resident_per_sm(K kernel, int threads, int smem, int (&slots)[kMaxDevices],
+inline cudaError_t resident_per_sm(K kernel, int threads, int smem, DeviceCache& slots,
                                    int* per_sm) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  if (slots[dev] == 0) {
-    int n = 0;
+  int n = slots[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     e = occupancy(kernel, threads, smem, &n);
     if (e != cudaSuccess) return e;
-    slots[dev] = n;
+    slots[dev].store(n, std::memory_order_relaxed);
   }
-  *per_sm = slots[dev];
+  *per_sm = n;
   return cudaSuccess;
 }
 
@@ -1475,7 +1497,7 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   if (!make_map(&km, a.k_cache, rows, KV, BS) || !make_map(&vm, a.v_cache, rows, KV, BS))
     return cudaErrorInvalidValue;
   if (kind == kTcGrid) {
-    static int slots[kMaxDevices] = {};
+    static DeviceCache slots;
     int per_sm = 0;
     cudaError_t e = resident_per_sm(decode_tc_kernel<KV, BS>, kNW * 32, C::kSmem, slots, &per_sm);
     if (e != cudaSuccess) return e;
@@ -1488,7 +1510,7 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   if (e != cudaSuccess) return e;
   if (kind == kTcCta) {
     if constexpr (BS != kSub) return cudaErrorInvalidValue;
-    static int slots[kMaxDevices] = {};
+    static DeviceCache slots;
     int per_sm = 0;
     e = resident_per_sm(decode_tc_persistent<KV>, kNW * 32, C::kPSmem, slots, &per_sm);
     if (e != cudaSuccess) return e;
@@ -1496,7 +1518,7 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
                    a, *pl, km, vm);
     if (e != cudaSuccess) return e;
   } else {
-    static int slots[kMaxDevices] = {};
+    static DeviceCache slots;
     int per_sm = 0;
     e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, slots, &per_sm);
     if (e != cudaSuccess) return e;

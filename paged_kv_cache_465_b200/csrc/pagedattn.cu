@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -31,9 +32,34 @@ bool desc_ok(const pa_decode_desc* d) {
   if (d->num_q_heads <= 0 || d->num_kv_heads <= 0 || d->num_kv_heads > 65535) return false;
   if (d->num_q_heads % d->num_kv_heads != 0) return false;
   if (d->head_dim <= 0 || d->block_size <= 0 || d->num_blocks <= 0) return false;
-  if (d->max_blocks_per_seq <= 0 || d->partition_size < 0) return false;
-  if (d->partition_size % d->block_size != 0) return false;
+  if (d->max_blocks_per_seq <= 0) return false;
+  if (d->partition_size == PA_PARTITION_AUTO) return true;
+  if (d->partition_size < 0 || d->partition_size % d->block_size != 0) return false;
   return true;
+}
+
+// The partition the library takes for PA_PARTITION_AUTO: the largest of 512, 256, 128 and
+// 64 tokens that makes at least two work items per resident warp worker if every sequence
+// were max_context_len long (num_seqs * Hkv * ceil(max_context_len / P) items), else 64;
+// contexts of at most 64 tokens get one pass (0). It depends on the shape and the SM count
+// only, never on the context lengths (device data) or on where blocks sit, so results stay
+// independent of the physical placement.
+int auto_partition(const pa_decode_desc* d, int max_context_len) {
+  if (max_context_len <= 64) return 0;
+  int sms = tc::sm_count();
+  if (sms <= 0) sms = 148;
+  const int64_t target = 2 * (int64_t)sms * PA_TCW_MIN_WARPS;
+  const int64_t units = (int64_t)d->num_seqs * d->num_kv_heads;
+  for (int p = 512; p >= 128; p /= 2)
+    if (units * ((max_context_len + p - 1) / p) >= target) return p;
+  return 64;
+}
+
+// desc with PA_PARTITION_AUTO replaced by the partition the library takes.
+pa_decode_desc resolved(const pa_decode_desc* d, int max_context_len) {
+  pa_decode_desc r = *d;
+  if (r.partition_size == PA_PARTITION_AUTO) r.partition_size = auto_partition(d, max_context_len);
+  return r;
 }
 
 bool desc_supported(const pa_decode_desc* d) {
@@ -64,6 +90,32 @@ WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
 }
 
 int pad_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
+
+#ifndef PA_TCW_FUSED_MERGE
+#define PA_TCW_FUSED_MERGE 1  // 1: warp workers merge rows of up to 32 partitions in place
+#endif
+
+// Which kernels a decode call runs: the tensor-core family (and which of its kernels) or
+// the CUDA-core path; whether the split path's partitions are merged in place by the warp
+// workers (rows of up to 32 partitions) or by a reduce launch afterwards.
+struct DecodeRoute {
+  bool split, tc, fused_merge;
+  tc::TcKind kind;
+  int launches;  // kernel launches of the call
+};
+
+DecodeRoute route_for(const pa_decode_desc* d, const WorkspaceLayout& wl, int impl) {
+  DecodeRoute r{wl.total > 0, false, false, tc::kTcGrid, 1};
+  if (impl != 1 && tc_supported(d)) {
+    r.tc = true;
+    r.kind = tc_kind(d, r.split, impl);
+    r.fused_merge = PA_TCW_FUSED_MERGE && r.kind == tc::kTcWarps && wl.parts <= 32;
+    r.launches = (r.kind != tc::kTcGrid ? 2 : 1) + (r.split && !r.fused_merge ? 1 : 0);
+  } else {
+    r.launches = r.split ? 2 : 1;
+  }
+  return r;
+}
 
 template <pa_dtype KV, int D, int GP>
 cudaError_t launch_simt(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
@@ -126,13 +178,27 @@ const char* pa_version(void) { return "pagedattn 0.4 sm_100a"; }
 
 pa_status pa_set_decode_impl(int impl) {
   if (impl < 0 || impl > 5) return PA_ERR_INVALID;
-  g_decode_impl = impl;
+  g_decode_impl.store(impl, std::memory_order_relaxed);
   return PA_OK;
 }
 
 size_t paged_attn_workspace_size(const pa_decode_desc* desc, int max_context_len) {
   if (!desc_ok(desc) || max_context_len < 0) return 0;
-  return layout_for(desc, max_context_len).total;
+  const pa_decode_desc d = resolved(desc, max_context_len);
+  return layout_for(&d, max_context_len).total;
+}
+
+int paged_attn_partition_size(const pa_decode_desc* desc, int max_context_len) {
+  if (!desc_ok(desc) || max_context_len < 0) return -1;
+  return resolved(desc, max_context_len).partition_size;
+}
+
+int paged_attn_decode_launches(const pa_decode_desc* desc, int max_context_len) {
+  if (!desc_ok(desc) || max_context_len < 0) return 0;
+  const pa_decode_desc d = resolved(desc, max_context_len);
+  if (!desc_supported(&d) || d.num_seqs == 0) return 0;
+  return route_for(&d, layout_for(&d, max_context_len),
+                   g_decode_impl.load(std::memory_order_relaxed)).launches;
 }
 
 pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -142,6 +208,8 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
                             const int32_t* k_zeros, const int32_t* v_zeros, float* lse_out,
                             void* workspace, size_t workspace_bytes, void* stream) {
   if (!desc_ok(desc) || max_context_len < 0 || !std::isfinite(scale)) return PA_ERR_INVALID;
+  const pa_decode_desc rdesc = resolved(desc, max_context_len);
+  desc = &rdesc;
   if (!desc_supported(desc)) return PA_ERR_UNSUPPORTED;
   if (desc->num_seqs == 0) return PA_OK;
   if (!q || !k_cache || !v_cache || !block_tables || !context_lens || !out) return PA_ERR_INVALID;
@@ -188,21 +256,20 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
   const int D = desc->head_dim;
   const int gp = pad_group(a.group);
   cudaError_t e;
-  if (g_decode_impl != 1 && tc_supported(desc)) {
-    const tc::TcKind kind = tc_kind(desc, split, g_decode_impl);
+  const DecodeRoute r = route_for(desc, wl, g_decode_impl.load(std::memory_order_relaxed));
+  if (r.tc) {
     tc::PlanView pl;
-    if (kind != tc::kTcGrid) {
+    if (r.kind != tc::kTcGrid) {
       char* ws = static_cast<char*>(workspace);
       pl.counters = reinterpret_cast<uint32_t*>(ws + wl.cnt_off);
       pl.list = reinterpret_cast<int2*>(ws + wl.list_off);
       a.skip_single = 1;  // single-partition sequences are written by the kernel itself
-      // warp workers merge rows of up to 32 partitions themselves (one lane per partition)
-      if (kind == tc::kTcWarps && wl.parts <= 32) {
+      if (r.fused_merge) {
         a.fused_merge = 1;
         a.arrive = reinterpret_cast<uint32_t*>(ws + wl.arr_off);
       }
     }
-    e = launch_tc(a, desc, grid, kind == tc::kTcGrid ? nullptr : &pl, kind, st);
+    e = launch_tc(a, desc, grid, r.kind == tc::kTcGrid ? nullptr : &pl, r.kind, st);
   } else {
     switch (desc->kv_dtype) {
       case PA_F32: e = launch_simt_d<PA_F32>(a, D, gp, grid, st); break;
@@ -240,7 +307,7 @@ pa_status paged_attn_prefill(const void* q, const void* k_cache, const void* v_c
   const cudaStream_t st = as_stream(stream);
   if (max_query_len == 0) return PA_OK;
   cudaError_t e;
-  if (g_decode_impl != 1 && prefill_tc_supported(desc)) {
+  if (g_decode_impl.load(std::memory_order_relaxed) != 1 && prefill_tc_supported(desc)) {
     pf::PrefillArgs a;
     a.block_tables = block_tables; a.context_lens = context_lens; a.query_start = query_start;
     a.out = out; a.lse_out = lse_out;
@@ -368,8 +435,28 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRA
 
 namespace {
 constexpr int kMaxDevices = 128;
-void* g_noalloc_ptr[kMaxDevices];
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];  // static storage: zero-initialised
 std::mutex g_noalloc_mu;
+
+// Device address of the fixed array on the current device, looked up on the first call
+// there (with that device current) and cached.
+pa_status noalloc_scratch(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    p = g_noalloc_ptr[dev].load(std::memory_order_relaxed);
+    if (p == nullptr) {
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return PA_ERR_CUDA;
+      g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *ptr = p;
+  return PA_OK;
+}
 }  // namespace
 
 pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
@@ -379,25 +466,16 @@ pa_status paged_attn_decode_noalloc(const void* q, const void* k_cache, const vo
                                     const float* v_scales, const int32_t* k_zeros,
                                     const int32_t* v_zeros, float* lse_out, void* stream) {
   if (!desc_ok(desc) || max_context_len < 0) return PA_ERR_INVALID;
-  const size_t need = paged_attn_workspace_size(desc, max_context_len);
-  if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_WORKSPACE;
+  if (paged_attn_workspace_size(desc, max_context_len) > PA_NOALLOC_SCRATCH_BYTES)
+    return PA_ERR_WORKSPACE;
+  // the look-up runs on every call, needed or not, so that the first call on a device does
+  // it whatever its shape
   void* ws = nullptr;
-  if (need > 0) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PA_ERR_CUDA;
-    if (dev < 0 || dev >= kMaxDevices) return PA_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-      void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
-        return PA_ERR_CUDA;
-      g_noalloc_ptr[dev] = p;
-    }
-    ws = g_noalloc_ptr[dev];
-  }
+  const pa_status st = noalloc_scratch(&ws);
+  if (st != PA_OK) return st;
   return paged_attn_decode(q, k_cache, v_cache, block_tables, context_lens, scale, out, desc,
                            max_context_len, k_scales, v_scales, k_zeros, v_zeros, lse_out, ws,
-                           ws ? (size_t)PA_NOALLOC_SCRATCH_BYTES : 0, stream);
+                           (size_t)PA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 pa_status pa_device_error(int* bits_out, void* stream) {

@@ -207,8 +207,19 @@ class DeviceScenario:
                  lse_out=self.lse, workspace=self.workspace, stream=stream)
         return self.out
 
+    def resolved_partition(self) -> int:
+        """The split partition the library takes for this step (0 = one pass)."""
+        from . import decode_desc_for, partition_size_for
+        return partition_size_for(decode_desc_for(self.q, self.cache.k_cache, self.block_tables,
+                                                  self.partition_size), self.max_context_len)
+
     def launches_per_step(self) -> int:
-        return (1 if self.pairs is not None else 0) + 1 + (2 if self.partition_size else 1)
+        """The library's kernel launches in one step: block copies, cache write, decode."""
+        from . import decode_desc_for, decode_launches
+        desc = decode_desc_for(self.q, self.cache.k_cache, self.block_tables,
+                               self.partition_size)
+        return (1 if self.pairs is not None else 0) + 1 + decode_launches(
+            desc, self.max_context_len)
 
     # -- algorithmic traffic of one step (bytes that must move) -----------------------------
     def kv_bytes(self) -> int:

@@ -262,7 +262,7 @@ SPLIT_IMPLS = ["simt", "tc-grid", "tc-cta", "tc-warps"]
 
 
 @pytest.mark.parametrize("impl", SPLIT_IMPLS)
-@pytest.mark.parametrize("part", [0, 512])
+@pytest.mark.parametrize("part", [0, 512, -1])   # -1: the library chooses the split
 def test_batch32_workload(pa, scen, impl, part):
     _run_and_compare(pa, scen, workloads.draw("b32"), impl, partition_size=part)
 
@@ -304,8 +304,8 @@ def test_long_context_full_size_sampled(pa, scen, impl):
 # invariances, needles, closed forms, edge cases
 # ---------------------------------------------------------------------------------------
 @pytest.mark.parametrize("impl", SPLIT_IMPLS)
-@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b256", 512),
-                                       ("b256_int8", 512)])
+@pytest.mark.parametrize("name,part", [("b32", 0), ("b32", 512), ("b32", -1), ("b256", 512),
+                                       ("b256_int8", 512), ("shared", -1)])
 def test_physical_placement_bit_identical(pa, scen, impl, name, part):
     wl = workloads.WORKLOADS[name].scaled(num_seqs=6)
     pa.set_decode_impl(impl)
@@ -328,6 +328,7 @@ def test_physical_placement_bit_identical(pa, scen, impl, name, part):
 @pytest.mark.parametrize("name,part,lens", [
     ("b32", 0, [1, 2, 15, 16, 17, 31, 33, 4096]),
     ("b32", 512, [511, 512, 513, 1024, 1025, 3000]),
+    ("b32", -1, [1, 2, 15, 16, 17, 31, 33, 64, 65, 4096]),
     ("b256", 512, [16, 17, 500, 512, 2049, 8192]),
     ("b256", 0, [1, 16, 100, 8192]),
     ("b256_int8", 512, [16, 17, 500, 513, 2049]),
@@ -436,8 +437,9 @@ def test_block_sizes_tiny_and_shared(pa, scen, B, impl):
 
 @pytest.mark.parametrize("impl", SPLIT_IMPLS)
 @pytest.mark.parametrize("B", [8, 32])
-@pytest.mark.parametrize("name,part,seqs", [("b32", 0, 32), ("b32", 512, 32), ("b256", 512, 12),
-                                            ("b256", 0, 6), ("b256_int8", 512, 12)])
+@pytest.mark.parametrize("name,part,seqs", [("b32", 0, 32), ("b32", 512, 32), ("b32", -1, 32),
+                                            ("b256", 512, 12), ("b256", 0, 6),
+                                            ("b256_int8", 512, 12)])
 def test_block_sizes_workloads(pa, scen, impl, B, name, part, seqs):
     _run_and_compare(pa, scen, workloads.draw(_bs(name, B, num_seqs=seqs)), impl,
                      partition_size=part)

@@ -255,3 +255,36 @@ def test_prefill_host_validation_without_device(pa):
     assert call(uns) == pa.PA_ERR_UNSUPPORTED
     fp8 = pa.make_desc(4, 32, 8, 128, 64, 1024, 0, pa.PA_BF16, pa.PA_FP8_E4M3, pa.PA_BF16)
     assert call(fp8) == pa.PA_ERR_INVALID                        # fp8 needs its scales
+
+
+def test_library_chosen_partition(pa):
+    """PA_PARTITION_AUTO: the largest of 512/256/128/64 tokens giving at least two items per
+    resident warp worker (2 x SMs x 16; 148 SMs when no device answers) for contexts of
+    max_context_len, else 64; one pass up to 64 tokens. The workspace and launch count
+    follow the chosen partition."""
+    target = 2 * 148 * 16
+
+    def rule(S, Hkv, L):
+        if L <= 64:
+            return 0
+        for p in (512, 256, 128):
+            if S * Hkv * -(-L // p) >= target:
+                return p
+        return 64
+
+    for S, Hkv, L, B in [(32, 8, 4096, 16), (256, 8, 8192, 16), (100, 8, 250, 16), (8, 8, 131072, 16),
+                         (1, 1, 64, 16), (1, 1, 65, 8), (3, 2, 40, 32), (4096, 8, 600, 32),
+                         (64, 8, 1000, 8)]:
+        d = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, pa.PARTITION_AUTO, pa.PA_BF16,
+                         pa.PA_BF16, pa.PA_BF16, block_size=B)
+        p = pa.partition_size_for(d, L)
+        assert p == rule(S, Hkv, L), (S, Hkv, L, p)
+        e = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, p, pa.PA_BF16, pa.PA_BF16,
+                         pa.PA_BF16, block_size=B)
+        assert pa.workspace_size(d, L) == pa.workspace_size(e, L)
+        assert pa.decode_launches(d, L) == pa.decode_launches(e, L) > 0
+    # an explicit partition is reported as given; a bad one is refused
+    d = pa.make_desc(4, 8, 2, 128, 4, 64, 48, pa.PA_BF16, pa.PA_BF16, pa.PA_BF16)
+    assert pa.partition_size_for(d, 60) == 48
+    d = pa.make_desc(4, 8, 2, 128, 4, 64, -2, pa.PA_BF16, pa.PA_BF16, pa.PA_BF16)
+    assert pa.partition_size_for(d, 60) == -1 and pa.workspace_size(d, 60) == 0

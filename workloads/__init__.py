@@ -50,7 +50,8 @@ class Workload:
     kv_dtype: str  # "f32" | "bf16" | "fp8" | "int8"
     in_dtype: str  # dtype of q and of the new K/V handed to the cache write: "f32" | "bf16"
     lens: Tuple  # ("fixed", [..]) | ("uniform", lo, hi) | ("lognormal", median, sigma, lo, hi) | ("const", n)
-    partition_size: int = 0  # split-KV partition in tokens; 0 = one pass per (seq, kv head)
+    # split-KV partition in tokens; 0 = one pass per (seq, kv head); -1 = the library's choice
+    partition_size: int = 0
     shared_prefix: Optional[Tuple[int, int]] = None  # (prefix tokens, suffix tokens per seq)
 
     @property
@@ -68,11 +69,13 @@ class Workload:
 WORKLOADS: Dict[str, Workload] = {
     # 4 seqs, ctx {5,16,17,40}, 4q/2kv, d 64, fp32, 32-block pool.
     "tiny": Workload("tiny", 0, 4, 4, 2, 64, 16, 32, "f32", "f32", ("fixed", [5, 16, 17, 40])),
-    # 32 seqs, ctx ~ U{1..4096}, 32q/8kv, d 128, bf16, 8192-block pool.
-    "b32": Workload("b32", 1, 32, 32, 8, 128, 16, 8192, "bf16", "bf16", ("uniform", 1, 4096)),
+    # 32 seqs, ctx ~ U{1..4096}, 32q/8kv, d 128, bf16, 8192-block pool; split chosen by the
+    # library (too few (seq, kv head) pairs to keep every SM streaming in one pass).
+    "b32": Workload("b32", 1, 32, 32, 8, 128, 16, 8192, "bf16", "bf16", ("uniform", 1, 4096),
+                    partition_size=-1),
     # 100 seqs sharing a 200-token prefix + 50 private tokens, 32q/8kv, d 128, bf16.
     "shared": Workload("shared", 2, 100, 32, 8, 128, 16, 512, "bf16", "bf16", ("const", 250),
-                       shared_prefix=(200, 50)),
+                       partition_size=-1, shared_prefix=(200, 50)),
     # 256 seqs, ctx lognormal(median 1024, sigma 1) clipped [16, 8192], fp8 KV, bf16 q/out.
     "b256": Workload("b256", 3, 256, 32, 8, 128, 16, 32768, "fp8", "bf16",
                      ("lognormal", 1024, 1.0, 16, 8192), partition_size=512),
