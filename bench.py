@@ -125,6 +125,84 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(inside), "note": note}
 
 
+class NvmlClocks:
+    """SM clock and clock-event reasons read through NVML (read-only queries) every
+    ``period`` seconds on a thread, so that a timed region of a few milliseconds still has
+    samples inside it. Falls back to ``ClockSampler`` (nvidia-smi) when NVML is missing."""
+
+    def __init__(self, torch, device_index: int, period: float = 0.001):
+        self.torch, self.index, self.period = torch, device_index, period
+        self.samples = []
+        self.ok = False
+        self._stop = threading.Event()
+
+    def __enter__(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            uuid = str(self.torch.cuda.get_device_properties(self.index).uuid)
+            try:
+                self.h = nv.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-")
+                                                      else "GPU-" + uuid)
+            except Exception:  # noqa: BLE001
+                self.h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception:  # noqa: BLE001
+            self.fallback = ClockSampler(self.index).__enter__()
+            return self
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
+        time.sleep(0.05)
+        return self
+
+    def _poll(self):
+        nv = self.nv
+        reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.time(), float(nv.nvmlDeviceGetClockInfo(
+                    self.h, nv.NVML_CLOCK_SM)), int(reasons(self.h))))
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        if not self.ok:
+            self.fallback.__exit__(*a)
+            return
+        self._stop.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:  # noqa: BLE001
+            pass
+
+    def summary(self, timed, window=None):
+        """Clocks over the timed region (t0, t1) and a loaded window right after it."""
+        if not self.ok:
+            return self.fallback.summary(*timed)
+        inside = [r for r in self.samples if timed[0] <= r[0] <= timed[1]]
+        win = [r for r in self.samples if window and window[0] <= r[0] <= window[1]]
+        rows = inside + win
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "note": "no NVML samples"}
+        mask = 0
+        for r in rows:
+            mask |= r[2]
+        reasons = [n for b, n in _REASONS.items() if mask & b and n != "gpu_idle"]
+        note = f"inside timed region: {len(inside)} NVML samples (every {self.period * 1e3:g} ms)"
+        if window:
+            note += (f"; plus {len(win)} in a {1e3 * (window[1] - window[0]):.0f} ms loaded "
+                     f"window of the same steps right after it")
+        return {"sm_mhz": float(np.median([r[1] for r in rows])), "sm_max_mhz": self.max_mhz,
+                "sm_mhz_timed": float(np.median([r[1] for r in inside])) if inside else None,
+                "reasons": reasons, "samples": len(rows), "note": note}
+
+
 # ---------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------
@@ -222,9 +300,42 @@ def _host_bookkeeping(pa, steps: int = 100):
     return out
 
 
-def _cpu_baseline(draw, seconds: float = 12.0):
+# the benchmark spec's bars on the decode output (max-abs) per KV storage type, with the relative-L2
+# and lse bars of the GPU parity tests
+PARITY_BARS = {"f32": (1e-4, 1e-5, 1e-3), "bf16": (2e-2, 1e-2, 1e-3), "fp8": (3e-2, 3e-2, 1e-3),
+               "int8": (3e-2, 3e-2, 1e-3)}
+
+
+def oracle_sample(wl, n: int = 8):
+    """The sequences the CPU-baseline leg recomputes (their K/V come from the seeded draw in
+    the GPU run too)."""
+    rng = np.random.default_rng(0)
+    return sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, n), replace=False).tolist())
+
+
+def parity_stats(got_out, got_lse, ref_out, ref_lse, kv_dtype, seqs):
+    """Errors of the GPU's decode output against the oracle's on the sampled sequences."""
+    o, ro = got_out[seqs], ref_out[seqs]
+    err = np.abs(o - ro)
+    rel = np.sqrt((err ** 2).sum(-1)) / np.maximum(np.sqrt((ro ** 2).sum(-1)), 1e-30)
+    fin = np.isfinite(ref_lse[seqs])
+    lse = np.abs(got_lse[seqs][fin] - ref_lse[seqs][fin])
+    bars = PARITY_BARS[kv_dtype]
+    res = {"max_abs": float(err.max()), "rel_l2": float(rel.max()),
+           "lse": float(lse.max()) if lse.size else 0.0, "seqs": [int(s) for s in seqs],
+           "bars": {"max_abs": bars[0], "rel_l2": bars[1], "lse": bars[2]}}
+    res["ok"] = bool(res["max_abs"] <= bars[0] and res["rel_l2"] <= bars[1]
+                     and res["lse"] <= bars[2]
+                     and np.array_equal(np.isfinite(got_lse[seqs]), np.isfinite(ref_lse[seqs])))
+    return res
+
+
+def _cpu_baseline(draw, seconds: float = 12.0, gpu=None):
     """The oracle, as it stands, on the host cores: this step's cache write plus decode for a
-    bounded sample of the workload's sequences (cycled until ~`seconds` elapse)."""
+    bounded sample of the workload's sequences (cycled until ~`seconds` elapse). ``gpu``:
+    (out, lse) of the GPU's last step as float64 arrays; the oracle's outputs for the
+    sampled sequences (whose K/V the GPU run took from the same draw) are compared with
+    them after the timing."""
     from oracle import flows, paged as opaged, attention
     try:
         from threadpoolctl import threadpool_info
@@ -232,12 +343,12 @@ def _cpu_baseline(draw, seconds: float = 12.0):
     except Exception:  # noqa: BLE001
         cores = os.cpu_count()
     wl = draw.wl
-    rng = np.random.default_rng(0)
-    sample = sorted(rng.choice(wl.num_seqs, size=min(wl.num_seqs, 8), replace=False).tolist())
+    sample = oracle_sample(wl)
     st = flows.build_state(draw, write_seqs=sample)
     sc = float(np.float32(1.0 / math.sqrt(wl.head_dim)))
     es = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[wl.kv_dtype]
     done_bytes = 0
+    outs = {}
     t0 = time.perf_counter()
     i = 0
     while True:
@@ -246,18 +357,27 @@ def _cpu_baseline(draw, seconds: float = 12.0):
         opaged.ref_reshape_and_cache(k[-1:], v[-1:], st.k_cache, st.v_cache, st.step_slots[s],
                                      wl.in_dtype, wl.kv_dtype, st.k_scales, st.v_scales,
                                      st.k_zeros, st.v_zeros)
-        attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables, st.context_lens,
-                             sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype, st.k_scales,
-                             st.v_scales, seqs=[s], k_zeros=st.k_zeros, v_zeros=st.v_zeros)
+        r = attention.ref_decode(draw.q, st.k_cache, st.v_cache, st.block_tables,
+                                 st.context_lens, sc, wl.num_kv_heads, wl.in_dtype, wl.kv_dtype,
+                                 st.k_scales, st.v_scales, seqs=[s], k_zeros=st.k_zeros,
+                                 v_zeros=st.v_zeros)
+        outs.setdefault(s, r)
         done_bytes += int(draw.context_lens[s]) * 2 * wl.num_kv_heads * wl.head_dim * es
         i += 1
         el = time.perf_counter() - t0
         if el >= seconds and i >= len(sample):
             break
-    return {"value": done_bytes / el / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
-            "sample": f"{i} (seq, all heads) decode steps cycling over {len(sample)} of "
-                      f"{wl.num_seqs} sequences of the same workload, float64 NumPy, "
-                      f"{el:.1f} s"}
+    res = {"value": done_bytes / el / 1e9, "unit": UNIT, "cores": int(cores), "kind": "oracle",
+           "sample": f"{i} (seq, all heads) decode steps cycling over {len(sample)} of "
+                     f"{wl.num_seqs} sequences of the same workload, float64 NumPy, "
+                     f"{el:.1f} s"}
+    if gpu is not None:
+        ref_out = np.full(gpu[0].shape, np.nan)
+        ref_lse = np.full(gpu[1].shape, np.nan)
+        for s, (o, l) in outs.items():
+            ref_out[s], ref_lse[s] = o[s], l[s]
+        res["parity"] = parity_stats(gpu[0], gpu[1], ref_out, ref_lse, wl.kv_dtype, sample)
+    return res
 
 
 def slowest_rank_seconds(seconds: float, dist=None, device="cpu") -> float:
@@ -294,7 +414,10 @@ def run_ours(args):
     pa.set_decode_impl(args.decode_impl)
     wl = workloads.WORKLOADS[args.workload]
     draw = workloads.draw(wl)
-    sc = DeviceScenario(draw, draw_seqs=[], partition_size=args.partition)
+    # the sequences the CPU-baseline leg recomputes take their K/V from the seeded draw (the
+    # others get the same distribution drawn on the device)
+    parity_seqs = oracle_sample(wl) if (world == 1 and not args.no_cpu_baseline) else []
+    sc = DeviceScenario(draw, draw_seqs=parity_seqs, partition_size=args.partition)
     l2 = torch.cuda.get_device_properties(local).L2_cache_size
     flush_buf = torch.empty(max(2 * l2, 64 << 20) // 4, dtype=torch.float32, device="cuda")
 
@@ -309,10 +432,18 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with NvmlClocks(torch, local) as clk:
         t_wall0 = time.time()
         total, dec_mean = _time_steps(torch, sc, args.steps, flush)
         t_wall1 = time.time()
+        # untimed: the same steps for a loaded window of ~0.3 s, for the clock record
+        w0 = time.time()
+        while time.time() - w0 < 0.3:
+            for _ in range(50):
+                flush()
+                sc.step()
+            torch.cuda.synchronize()
+        w1 = time.time()
     total = slowest_rank_seconds(total, dist, "cuda")
     if dist is not None:
         dist.barrier()
@@ -336,7 +467,7 @@ def run_ours(args):
         "config": {"workload": DESCR[args.workload], "name": args.workload,
                    "num_seqs": wl.num_seqs, "q_heads": wl.num_q_heads,
                    "kv_heads": wl.num_kv_heads, "head_dim": wl.head_dim, "block_size": 16,
-                   "partition_size": sc.partition_size,
+                   "partition_size": sc.resolved_partition(),
                    "tokens_in_cache": int(draw.context_lens.sum()),
                    "kv_bytes_per_step": b["kv"], "step_bytes": b,
                    "parallelism": f"replicas x{world} (no data-path collective)",
@@ -356,13 +487,16 @@ def run_ours(args):
         "e2e": {"value": round(e2e_gbs, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": sc.launches_per_step() * args.steps,
-        "clocks": clk.summary(t_wall0, t_wall1),
+        "clocks": clk.summary((t_wall0, t_wall1), (w0, w1)),
     }
     traffic = _traffic_note(args.workload, pa.version())
     if traffic is not None:
         result["roofline"]["traffic"] = traffic
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = _cpu_baseline(draw, args.cpu_seconds)
+        gpu = (sc.out.to(torch.float64).cpu().numpy(), sc.lse.to(torch.float64).cpu().numpy())
+        cb = _cpu_baseline(draw, args.cpu_seconds, gpu=gpu)
+        result["parity"] = cb.pop("parity")
+        result["cpu_baseline"] = cb
     if rank == 0:
         result["host"] = _host_bookkeeping(pa)
     if rank == 0 and args.extra and world == 1:
@@ -471,7 +605,7 @@ def _extra_workloads(torch, pa, args, flush):
                      "decode_ms": round(dec * 1e3, 5),
                      "decode_gbs": round(b["decode"] / dec / 1e9, 2),
                      "tokens_per_s": round(draw.wl.num_seqs / (total / steps), 1),
-                     "partition_size": sc.partition_size, "block_size": wl.block_size,
+                     "partition_size": sc.resolved_partition(), "block_size": wl.block_size,
                      "last_block_waste": round(_last_block_waste(draw.context_lens,
                                                                  wl.block_size), 6),
                      "steps": steps}

@@ -94,3 +94,34 @@ def test_host_bookkeeping_timing():
     assert h["append_batch_us_per_step"] > 0 and h["append_us_per_step"] > 0
     assert h["add_seq_tokens_us_per_request"] > 0
     assert h["prefix_cached_tokens"] == 99 * 192     # 12 full blocks reused per later request
+
+
+def test_nvml_clock_summary_inside_timed_region_and_window():
+    import numpy as np
+    c = bench.NvmlClocks(None, 0)
+    c.ok, c.max_mhz = True, 1965.0
+    # (time, SM MHz, clock-event reason bits)
+    c.samples = [(0.9, 700.0, 0x1), (1.0, 1965.0, 0x0), (1.002, 1950.0, 0x4), (1.5, 1000.0, 0x1),
+                 (2.0, 1965.0, 0x0), (2.1, 1965.0, 0x0), (3.0, 500.0, 0x1)]
+    s = c.summary((1.0, 1.003), (2.0, 2.2))
+    assert s["samples"] == 4 and s["sm_mhz"] == float(np.median([1965, 1950, 1965, 1965]))
+    assert s["sm_mhz_timed"] == float(np.median([1965, 1950]))
+    assert s["reasons"] == ["sw_power_cap"] and s["sm_max_mhz"] == 1965.0
+    assert s["note"].startswith("inside timed region: 2 NVML samples")
+
+
+def test_parity_stats_pass_and_catch_a_dropped_term():
+    import numpy as np
+    rng = np.random.default_rng(0)
+    ref = rng.standard_normal((5, 4, 8)) * 0.1
+    lse = rng.standard_normal((5, 4))
+    got = ref + 1e-4
+    p = bench.parity_stats(got, lse + 1e-4, ref, lse, "bf16", [1, 3])
+    assert p["ok"] and p["seqs"] == [1, 3] and abs(p["max_abs"] - 1e-4) < 1e-12
+    bad = got.copy()
+    bad[3, 2] = 0.0                       # one head's output lost
+    assert not bench.parity_stats(bad, lse, ref, lse, "bf16", [1, 3])["ok"]
+    assert not bench.parity_stats(got, lse + 1e-2, ref, lse, "bf16", [1, 3])["ok"]
+    lse_inf = lse.copy()
+    lse_inf[1, 0] = -np.inf               # an empty row must stay empty
+    assert not bench.parity_stats(got, lse, ref, lse_inf, "bf16", [1, 3])["ok"]
