@@ -396,6 +396,38 @@ def job_throughput(bytes_per_rank_step: int, steps: int, world: int, slowest_s: 
     return world * bytes_per_rank_step * steps / slowest_s / 1e9
 
 
+def run_profile(args):
+    """Warm-up and timed steps of one workload only (decode or prefill), nothing else: the
+    command the ncu summaries under profiles/ capture. Prints one short JSON line."""
+    import torch
+    import paged_kv_cache_465_b200 as pa
+    from paged_kv_cache_465_b200.scenario import DeviceScenario, PrefillScenario
+    torch.cuda.set_device(0)
+    pa.set_decode_impl(args.decode_impl)
+    kw = {"num_seqs": args.seqs} if args.seqs else {}
+    if args.workload in workloads.PREFILL_WORKLOADS:
+        wl = workloads.PREFILL_WORKLOADS[args.workload].scaled(**kw)
+        sc = PrefillScenario(workloads.draw_prefill(wl), draw_seqs=[])
+    else:
+        wl = workloads.WORKLOADS[args.workload].scaled(**kw)
+        sc = DeviceScenario(workloads.draw(wl), draw_seqs=[], partition_size=args.partition)
+    l2 = torch.cuda.get_device_properties(0).L2_cache_size
+    flush_buf = torch.empty(max(2 * l2, 64 << 20) // 4, dtype=torch.float32, device="cuda")
+    for i in range(args.warmup + args.steps):
+        flush_buf.fill_(1.0)
+        if i == args.warmup:
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+        sc.step()
+    torch.cuda.synchronize()
+    err = pa.device_error()
+    print(json.dumps({"profile": args.workload, "steps": args.steps, "warmup": args.warmup,
+                      "wall_ms_per_step": round((time.perf_counter() - t0) / args.steps * 1e3, 4),
+                      "device_error": err}), flush=True)
+    if err:
+        raise SystemExit(1)
+
+
 def run_ours(args):
     import torch
     from paged_kv_cache_465_b200.scenario import DeviceScenario
@@ -677,7 +709,13 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="b256", choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--workload", default="b256",
+                    choices=sorted(workloads.WORKLOADS) + sorted(workloads.PREFILL_WORKLOADS),
+                    help="decode workload (prefill workloads with --profile only)")
+    ap.add_argument("--profile", action="store_true",
+                    help="only the warm-up and timed steps of --workload (for ncu captures)")
+    ap.add_argument("--seqs", type=int, default=0,
+                    help="with --profile: the workload's first N sequences only")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--decode-impl", default="auto",
                     choices=["auto", "simt", "tc", "tc-grid", "tc-cta", "tc-warps"])
@@ -690,7 +728,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    if args.impl == "reference":
+    if args.workload in workloads.PREFILL_WORKLOADS and not args.profile:
+        ap.error("prefill workloads run with --profile only")
+    if args.profile:
+        run_profile(args)
+    elif args.impl == "reference":
         run_reference(args)
     else:
         run_ours(args)

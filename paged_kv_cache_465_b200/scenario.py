@@ -331,38 +331,3 @@ class PrefillScenario(DeviceScenario):
         keys = int(np.sum(qn * (lens - qn) + qn * (qn + 1) // 2))
         return 4 * wl.head_dim * wl.num_q_heads * keys
 
-
-def _main(argv=None):
-    """Runs a few steps of a named workload on cuda:0 (for profilers):
-
-        python -m paged_kv_cache_465_b200.scenario prefill --seqs 2 --steps 3
-    """
-    import argparse
-    import workloads
-    ap = argparse.ArgumentParser(description="run steps of a synthetic workload")
-    ap.add_argument("workload")
-    ap.add_argument("--seqs", type=int, default=0, help="override the number of sequences")
-    ap.add_argument("--steps", type=int, default=3)
-    args = ap.parse_args(argv)
-    import torch
-    from . import device_error
-    if args.workload in workloads.PREFILL_WORKLOADS:
-        wl = workloads.PREFILL_WORKLOADS[args.workload]
-        if args.seqs:
-            wl = wl.scaled(num_seqs=args.seqs)
-        sc = PrefillScenario(workloads.draw_prefill(wl), draw_seqs=[])
-    else:
-        wl = workloads.WORKLOADS[args.workload]
-        if args.seqs:
-            wl = wl.scaled(num_seqs=args.seqs)
-        sc = DeviceScenario(workloads.draw(wl), draw_seqs=[])
-    for _ in range(args.steps):
-        sc.step()
-    torch.cuda.synchronize()
-    err = device_error()
-    print(f"{args.workload}: {args.steps} steps, device error word {err}")
-    return 0 if err == 0 else 1
-
-
-if __name__ == "__main__":
-    raise SystemExit(_main())
