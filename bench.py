@@ -16,6 +16,7 @@ bytes of all ranks over the slowest rank's time ("weak" scaling).
 from __future__ import annotations
 
 import argparse
+import hashlib
 import json
 import math
 import os
@@ -521,7 +522,7 @@ def run_ours(args):
         "gpu_launches": sc.launches_per_step() * args.steps,
         "clocks": clk.summary((t_wall0, t_wall1), (w0, w1)),
     }
-    traffic = _traffic_note(args.workload, pa.version())
+    traffic = _traffic_note(args.workload)
     if traffic is not None:
         result["roofline"]["traffic"] = traffic
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -540,16 +541,29 @@ def run_ours(args):
         print(json.dumps(result), flush=True)
 
 
-def _traffic_note(name, version):
+# the sources the decode call's kernels are compiled from
+DECODE_SOURCES = ("common.cuh", "decode_simt.cuh", "decode_tc.cuh", "pagedattn.cu")
+
+
+def decode_sources_hash() -> str:
+    """First 16 hex digits of the SHA-256 of the decode kernels' sources, in order."""
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_465_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _traffic_note(name):
     """DRAM bytes of one decode call from the committed ncu summary (profiles/traffic.json)
-    when it was taken on this exact library build; else None."""
+    when it was taken on kernels built from exactly these decode sources; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         j = json.load(f)
     e = j.get(name)
-    if not e or j.get("version") != version:
+    if not e or j.get("sources") != decode_sources_hash():
         return None
     return e.get("bytes_per_launch")
 

@@ -124,6 +124,13 @@ def test_full_size_chunks_sampled(pa, scen):
     _run(pa, scen, d, draw_seqs=[int(np.argmax(d.context_lens)), 3], check_cache=False)
 
 
+def test_full_size_fp8_chunks_sampled(pa, scen):
+    """The fp8 chunked step the bench times, at full size, on sampled sequences."""
+    d = workloads.draw_prefill("chunked_fp8")
+    _run(pa, scen, d, draw_seqs=[int(np.argmax(d.context_lens)), int(np.argmin(d.context_lens))],
+         check_cache=False)
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 def test_causality_and_placement(pa, scen, impl):
     wl = workloads.PREFILL_WORKLOADS["chunked"].scaled(num_seqs=3, lens=("fixed", [700, 260, 900]),
