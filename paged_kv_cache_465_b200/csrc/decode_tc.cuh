@@ -845,36 +845,53 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
 __device__ __forceinline__ void merge_rows(const DecodeArgs& a, int64_t row0, int G, int np,
                                            int lane) {
   static_assert(kD == 128, "one channel quad per lane");
-  for (int g = 0; g < G; ++g) {
-    const int64_t row = row0 + g;
-    const float* pm = a.part_m + row * a.max_parts;
-    const float* pl = a.part_l + row * a.max_parts;
-    const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * kD);
-    const float mp = lane < np ? __ldcg(pm + lane) : -INFINITY;
-    float M = mp;
+  constexpr int R = 4;  // rows merged together: their partial reads are in flight at once
+  for (int g0 = 0; g0 < G; g0 += R) {
+    float M[R], w[R], lsum[R];
+    float4 acc[R];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    const float w = (lane < np && M != -INFINITY) ? fast_exp2(mp - M) : 0.f;
-    float lsum = 0.f;
-    if (lane < np) lsum = fmaf(w, __ldcg(pl + lane), lsum);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 4
+    for (int r = 0; r < R; ++r) {
+      const bool live = g0 + r < G && lane < np;
+      const int64_t row = row0 + g0 + r;
+      const float mp = live ? __ldcg(a.part_m + row * a.max_parts + lane) : -INFINITY;
+      const float lp = live ? __ldcg(a.part_l + row * a.max_parts + lane) : 0.f;
+      float m = mp;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      M[r] = m;
+      w[r] = (live && m != -INFINITY) ? fast_exp2(mp - m) : 0.f;
+      lsum[r] = live ? w[r] * lp : 0.f;
+      acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll 2
     for (int k = 0; k < np; ++k) {
-      const float wk = __shfl_sync(0xffffffffu, w, k);
-      const float4 v = __ldcg(pacc + (int64_t)k * (kD / 4) + lane);
-      acc.x = fmaf(wk, v.x, acc.x); acc.y = fmaf(wk, v.y, acc.y);
-      acc.z = fmaf(wk, v.z, acc.z); acc.w = fmaf(wk, v.w, acc.w);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        if (g0 + r >= G) continue;  // warp-uniform
+        const float wk = __shfl_sync(0xffffffffu, w[r], k);
+        const float4 v = __ldcg(reinterpret_cast<const float4*>(
+                                    a.part_acc + (row0 + g0 + r) * a.max_parts * kD) +
+                                (int64_t)k * (kD / 4) + lane);
+        acc[r].x = fmaf(wk, v.x, acc[r].x); acc[r].y = fmaf(wk, v.y, acc[r].y);
+        acc[r].z = fmaf(wk, v.z, acc[r].z); acc[r].w = fmaf(wk, v.w, acc[r].w);
+      }
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-    const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
-    const int64_t o = row * kD + 4 * lane;
-    store_out(a.out, a.out_dtype, o, acc.x * inv);
-    store_out(a.out, a.out_dtype, o + 1, acc.y * inv);
-    store_out(a.out, a.out_dtype, o + 2, acc.z * inv);
-    store_out(a.out, a.out_dtype, o + 3, acc.w * inv);
-    if (lane == 0 && a.lse_out != nullptr)
-      a.lse_out[row] = lsum > 0.f ? (M + __log2f(lsum)) * kLn2 : -INFINITY;
+    for (int r = 0; r < R; ++r) {
+      if (g0 + r >= G) continue;
+      float l = lsum[r];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      const int64_t row = row0 + g0 + r;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const int64_t o = row * kD + 4 * lane;
+      store_out(a.out, a.out_dtype, o, acc[r].x * inv);
+      store_out(a.out, a.out_dtype, o + 1, acc[r].y * inv);
+      store_out(a.out, a.out_dtype, o + 2, acc[r].z * inv);
+      store_out(a.out, a.out_dtype, o + 3, acc[r].w * inv);
+      if (lane == 0 && a.lse_out != nullptr)
+        a.lse_out[row] = l > 0.f ? (M[r] + __log2f(l)) * kLn2 : -INFINITY;
+    }
   }
 }
 
