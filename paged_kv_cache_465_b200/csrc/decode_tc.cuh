@@ -1127,8 +1127,8 @@ constexpr int kWW = PA_TCW_WARPS;
 #ifndef PA_TCW_MIN_WARPS
 #define PA_TCW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
 #endif
-#ifndef PA_TCW_STAGED_FETCH
-#define PA_TCW_STAGED_FETCH 0  // 1: the next item is fetched in steps behind the current one
+#ifndef PA_TCW_LOOKAHEAD
+#define PA_TCW_LOOKAHEAD 1  // 1: the item after the next one is fetched in steps (below)
 #endif
 
 template <pa_dtype KV>
@@ -1137,10 +1137,16 @@ struct TcwCfg {
   static constexpr int kQBytes = 8 * kD * 2;  // one group's q, <= 8 heads
   static constexpr int kSmem =
       kWW * kNStage * TcCfg<KV>::kStage + kWW * kQBytes + kWW * (kNStage + 1) * 8 + 1024;
+  // CTAs per SM that shared memory allows (228 KB per SM, 1 KB reserved per CTA): the
+  // register budget is sized for that many (fp8 / int8: 14, bf16: 8), at most
+  // PA_TCW_MIN_WARPS warps
+  static constexpr int kResident = 233472 / (kSmem + 1024) < PA_TCW_MIN_WARPS / kWW
+                                       ? 233472 / (kSmem + 1024)
+                                       : PA_TCW_MIN_WARPS / kWW;
 };
 
 template <pa_dtype KV, int BS>
-__global__ void __launch_bounds__(kWW * 32, PA_TCW_MIN_WARPS / kWW)
+__global__ void __launch_bounds__(kWW * 32, TcwCfg<KV>::kResident)
 decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap) {
   using C = TcCfg<KV>;
@@ -1224,65 +1230,53 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   int pslot = 0, pk = 0;
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
-  // From the second item on, the item after the current one is fetched in kFetchDone
-  // steps, one per consumed sub-tile. Each step uses only values that a global read issued
-  // one step earlier returns (work ticket, list entry, context length, block ids), so the
-  // reads overlap the current item's tiles instead of stalling the warp between items.
-  // An item shorter than that finishes the fetch at its end.
-  constexpr int kFetchDone = 5;
-  // int8 caches with 8-token blocks keep the fetch in one piece at the item boundary: the
-  // staged form would make that variant spill
-  constexpr bool kStaged = PA_TCW_STAGED_FETCH && !(KV == PA_INT8 && BS == 8);
-  int nstage = kFetchDone;  // nxt and nxt_w are resolved
-  bool nxt_q = false;       // nxt's q copy is issued
-  uint32_t tk = 0;          // work ticket (lane 0 until broadcast)
-  int2 sp = make_int2(0, 0);
-  int sp_ctx = 0;
-  auto fetch_step = [&]() {
-    if (nstage == 0) {
-      if (lane == 0) tk = atomicAdd(&pl.counters[0], 1u);
-    } else if (nstage == 1) {
-      tk = __shfl_sync(0xffffffffu, tk, 0);
-      if (tk < total) sp = pl.list[tk / Hkv];
-    } else if (nstage == 2) {
-      if (tk < total) sp_ctx = a.context_lens[sp.x];
-    } else if (nstage == 3) {
-      nxt = Item{0, 0, 0, 0, 0, 0, 0, 0};
-      if (tk < total) {
-        int ctx = sp_ctx;  // clamped and flagged as checked_ctx does
-        if (ctx < 0 || ctx > a.max_context_len) {
-          if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
-          ctx = ctx < 0 ? 0 : a.max_context_len;
-        }
-        const int t0 = sp.y * P;
-        nxt.valid = 1;
-        nxt.s = sp.x;
-        nxt.kvh = (int)(tk % Hkv);
-        nxt.part = sp.y;
-        nxt.t1 = min(ctx, t0 + P);
-        nxt.c_begin = t0 / kSub;
-        nxt.nsub = (nxt.t1 + kSub - 1) / kSub - nxt.c_begin;
-        nxt.np = (ctx + P - 1) / P;
-      }
-      if (nxt.valid && lane < nxt.nsub)
-        load_sub_ids<BS>(a.block_tables + (int64_t)nxt.s * a.max_blocks_per_seq,
-                         nxt.c_begin + lane, nxt.t1, nxt_w);
-      else
-        empty_sub(nxt_w);
-    } else if (nstage == 4) {
-      if (nxt.valid && lane < nxt.nsub)
-        load_sub_params<KV, BS>(a, nxt.c_begin + lane, nxt.t1, nxt.kvh, nxt_w);
-      if (!dead) {  // the q buffer is free: the current item's fragments are in registers
-        copy_q(nxt);
-        nxt_q = true;
-      }
+  // Look-ahead: the item after `nxt` is fetched in three steps while the current item runs
+  // (work ticket at its start, list entry after its first consumed sub-tile, context
+  // length after its second), each step using what the previous step's read returned; at
+  // the item boundary only its block-table window is still read. `nxt` itself is always
+  // resolved, so the producer streams into it without waiting.
+  constexpr bool kLookahead = PA_TCW_LOOKAHEAD != 0;
+  uint32_t la_tk = 0;  // work ticket (lane 0 until broadcast)
+  int2 la_sp = make_int2(0, 0);
+  int la_ctx = 0;
+  int la_stage = kLookahead ? 0 : 3;
+  auto la_step = [&]() {
+    if (la_stage == 0) {
+      if (lane == 0) la_tk = atomicAdd(&pl.counters[0], 1u);
+    } else if (la_stage == 1) {
+      la_tk = __shfl_sync(0xffffffffu, la_tk, 0);
+      if (la_tk < total) la_sp = pl.list[la_tk / Hkv];
+    } else if (la_stage == 2) {
+      if (la_tk < total) la_ctx = a.context_lens[la_sp.x];
     }
-    ++nstage;
+    ++la_stage;
+  };
+  // the looked-ahead item (after its three steps); else the plain fetch
+  auto next_item = [&]() {
+    if constexpr (!kLookahead) return fetch();
+    Item v{0, 0, 0, 0, 0, 0, 0, 0};
+    if (la_tk < total) {
+      int ctx = la_ctx;  // clamped and flagged as checked_ctx does
+      if (ctx < 0 || ctx > a.max_context_len) {
+        if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
+        ctx = ctx < 0 ? 0 : a.max_context_len;
+      }
+      const int t0 = la_sp.y * P;
+      v.valid = 1;
+      v.s = la_sp.x;
+      v.kvh = (int)(la_tk % Hkv);
+      v.part = la_sp.y;
+      v.t1 = min(ctx, t0 + P);
+      v.c_begin = t0 / kSub;
+      v.nsub = (v.t1 + kSub - 1) / kSub - v.c_begin;
+      v.np = (ctx + P - 1) / P;
+    }
+    return v;
   };
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
-      if (pslot == 1 && (nstage < kFetchDone || !nxt.valid || pk >= nxt.nsub)) break;
+      if (pslot == 1 && (!nxt.valid || pk >= nxt.nsub)) break;
       const Item& v = pslot == 0 ? cur : nxt;
       const SubWin sw = shfl_sub<BS>(pslot == 0 ? cur_w : nxt_w, pk);
       const int stage = g_iss % NST;
@@ -1310,12 +1304,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf), G, lane,
                                            a.scale_log2, qf);
     __syncwarp();
-    // the buffer is free once every lane holds its fragments (first item: nxt is resolved
-    // already; later ones issue it in the last fetch step)
-    if (!dead && nstage == kFetchDone && !nxt_q) {
-      copy_q(nxt);
-      nxt_q = true;
-    }
+    if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
+    if (la_stage == 0) la_step();  // the work ticket of the item after nxt
     w.reset();
     for (int i = 0; i < cur.nsub; ++i) {
       const SubWin sw = shfl_sub<BS>(cur_w, i);
@@ -1332,7 +1322,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       __syncwarp();
       ++g_cons;
       produce();
-      if (kStaged && nstage < kFetchDone) fetch_step();
+      if (la_stage < 3) la_step();
     }
     // ---- item done: its output (single partition) or its partial ----
 #pragma unroll
@@ -1403,19 +1393,12 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       }
     }
     // ---- advance ----
-    if constexpr (kStaged) {
-      while (nstage < kFetchDone) fetch_step();  // a short item: finish the fetch here
-      cur = nxt;
-      cur_w = nxt_w;
-      nstage = 0;
-      fetch_step();  // the work ticket of the item after it
-    } else {
-      cur = nxt;
-      cur_w = nxt_w;
-      nxt = fetch();
-      load_window(nxt, nxt_w);
-    }
-    nxt_q = false;
+    while (la_stage < 3) la_step();  // a short item: finish the look-ahead here
+    cur = nxt;
+    cur_w = nxt_w;
+    nxt = next_item();
+    load_window(nxt, nxt_w);
+    if (kLookahead) la_stage = 0;
     pslot = 0;
     produce();
   }
