@@ -775,27 +775,21 @@ struct PlanView {
   int2* list;
 };
 
-// One CTA of 1024 threads builds the work list: the partitions of a sequence are
-// consecutive, sequences with more partitions come first and, among one-partition
-// sequences, longer ones first (a counting sort over 256 buckets: one-partition sequences
-// by sub-tile count 1 .. P/16, the others by partition count above that). So the
-// partitions of a long sequence are taken together and merged (warp workers) while other
-// work still streams, and the last items of the launch are short ones. It also zeroes the
-// fetch counter (and the arrival counters of the merging warp workers) and writes out = 0
-// / lse = -inf for empty sequences. The order affects scheduling only: every item's
-// result, and the merge order, depend on logical positions alone.
+// One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
+// largest first (full partitions, then partial ones by size; a counting sort), writes the
+// list, zeroes the fetch counter (and the arrival counters of the merging warp workers),
+// and writes out = 0 / lse = -inf for empty sequences. Largest first keeps the launch's
+// tail short: the last items taken are the smallest. (Keeping a sequence's partitions
+// together instead, so that merges happen early, measured 12 % slower on the batch-256
+// workload: full partitions then land in the tail.) The order affects scheduling only:
+// every item's result, and the merge order, depend on logical positions alone.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
-  constexpr int kBuckets = 256;
-  __shared__ int cnt[kBuckets], off[kBuckets];
+  __shared__ int cnt[130], off[130];
   pdl_wait();
   pdl_trigger();
   const int P = a.part_tokens;
   const int nbk = P / kSub;  // sub-tiles of a full partition (<= 128)
-  auto bucket = [&](int ctx, int& np) {
-    np = (ctx + P - 1) / P;
-    return np == 1 ? (ctx + kSub - 1) / kSub : nbk + min(np - 1, kBuckets - 1 - nbk);
-  };
-  for (int i = threadIdx.x; i < kBuckets; i += blockDim.x) cnt[i] = 0;
+  for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
   if (a.fused_merge)
     for (int64_t i = threadIdx.x; i < (int64_t)a.num_seqs * a.num_kv_heads; i += blockDim.x)
       a.arrive[i] = 0u;
@@ -810,14 +804,14 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       }
       continue;
     }
-    int np;
-    const int b = bucket(ctx, np);
-    atomicAdd(&cnt[b], np);
+    const int full = ctx / P, rem = ctx % P;
+    if (full) atomicAdd(&cnt[nbk], full);
+    if (rem) atomicAdd(&cnt[(rem + kSub - 1) / kSub], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
     int acc = 0;
-    for (int b = kBuckets - 1; b >= 1; --b) {
+    for (int b = nbk; b >= 1; --b) {
       off[b] = acc;
       acc += cnt[b];
     }
@@ -827,11 +821,12 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int ctx = checked_ctx(a, s);
-    if (ctx == 0) continue;
-    int np;
-    const int b = bucket(ctx, np);
-    const int base = atomicAdd(&off[b], np);
-    for (int j = 0; j < np; ++j) pl.list[base + j] = make_int2(s, j);
+    const int full = ctx / P, rem = ctx % P;
+    if (full) {
+      const int base = atomicAdd(&off[nbk], full);
+      for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
+    }
+    if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
   }
 }
 

@@ -92,7 +92,7 @@ WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
 int pad_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
 
 #ifndef PA_TCW_FUSED_MERGE
-#define PA_TCW_FUSED_MERGE 1  // 1: warp workers merge rows of up to 32 partitions in place
+#define PA_TCW_FUSED_MERGE 0  // 1: warp workers merge rows of up to 32 partitions in place
 #endif
 
 // Which kernels a decode call runs: the tensor-core family (and which of its kernels) or

@@ -69,7 +69,10 @@ constexpr int kOffV = kOffK + kKSt * kKVBytes;
 // stages from them) and the tile's per-block scales and zero points. The staging buffer is
 // a ring of four quarters of 32 keys: the codes of a quarter of the next tile are loaded
 // as soon as the converters have read that quarter of the current one.
-constexpr int kQuarters = 4, kQKeys = kBN / kQuarters;
+#ifndef PA_PF_QUARTERS
+#define PA_PF_QUARTERS 4
+#endif
+constexpr int kQuarters = PA_PF_QUARTERS, kQKeys = kBN / kQuarters;  // 1, 2 or 4
 template <bool QUANT>
 struct PfLayout {
   static constexpr int kThreads = QUANT ? 384 : 320;
@@ -101,13 +104,13 @@ constexpr int kBarP = kBarSF + kQT;        // [query tile], kBM arrivals
 constexpr int kBarO = kBarP + kQT;         // [query tile][ring]
 constexpr int kBarFin = kBarO + kQT * kORing;
 constexpr int kBarK8F = kBarFin + 1;       // quantised: [quarter] codes staged (TMA)
-constexpr int kBarK8E = kBarK8F + 4;       // quantised: [quarter] staging read by the converters
-constexpr int kBarV8F = kBarK8E + 4;
-constexpr int kBarV8E = kBarV8F + 4;
-constexpr int kBarSC = kBarV8E + 4;        // quantised: [4] a tile's K / V scales for the softmax
+constexpr int kBarK8E = kBarK8F + kQuarters;  // quantised: [quarter] staging read by converters
+constexpr int kBarV8F = kBarK8E + kQuarters;
+constexpr int kBarV8E = kBarV8F + kQuarters;
+constexpr int kBarSC = kBarV8E + kQuarters;   // quantised: [4] a tile's K / V scales for softmax
 constexpr int kSideRing = 4;
 constexpr int kNumBars = kBarSC + kSideRing;
-static_assert(kQuarters == 4, "four staging barriers per K / V");
+static_assert(kQuarters == 1 || kQuarters == 2 || kQuarters == 4, "staging ring");
 static_assert(kNumBars * 8 + 8 <= PfLayout<true>::kBarArea, "barrier area");
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
