@@ -123,11 +123,6 @@ struct DecodeArgs {
   int max_context_len;
   int final_pass;    // 1: one item covers the whole context, write out directly
   int skip_single;   // split path: single-partition sequences were written directly
-  // split path, warp workers: the warp that stores the last partial of a (sequence, kv
-  // head) merges its partitions itself (no reduce launch). arrive[s * Hkv + kvh] counts
-  // the partials stored so far; the plan kernel zeroes it.
-  int fused_merge;
-  uint32_t* arrive;  // [S][Hkv]
   pa_dtype q_dtype, out_dtype;
   // prefill rows (CUDA-core kernel only): work row s is new token s; the tokens of
   // sequence q are rows query_start[q] .. query_start[q+1]-1, the last ones of its context
@@ -405,8 +400,11 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
   const float* pl = a.part_l + row * a.max_parts;
   const float4* pacc = reinterpret_cast<const float4*>(a.part_acc + row * a.max_parts * D);
 
-  float M = -INFINITY;
-  for (int p = lane; p < np; p += 32) M = fmaxf(M, pm[p]);
+  // the first 32 partitions' maxima and sums are read together (one round trip)
+  const float m0 = lane < np ? pm[lane] : -INFINITY;
+  const float l0 = lane < np ? pl[lane] : 0.f;
+  float M = m0;
+  for (int p = lane + 32; p < np; p += 32) M = fmaxf(M, pm[p]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
 
@@ -417,10 +415,12 @@ __global__ void __launch_bounds__(128) lse_reduce_kernel(const DecodeArgs a) {
   float lsum = 0.f;
   for (int c0 = 0; c0 < np; c0 += 32) {
     const int p = c0 + lane;
-    const float w = (p < np && M != -INFINITY) ? fast_exp2(pm[p] - M) : 0.f;
-    if (p < np) lsum = fmaf(w, pl[p], lsum);
+    const float mp = c0 == 0 ? m0 : (p < np ? pm[p] : -INFINITY);
+    const float lp = c0 == 0 ? l0 : (p < np ? pl[p] : 0.f);
+    const float w = (p < np && M != -INFINITY) ? fast_exp2(mp - M) : 0.f;
+    if (p < np) lsum = fmaf(w, lp, lsum);
     const int n = min(32, np - c0);
-#pragma unroll 4
+#pragma unroll 8
     for (int k = 0; k < n; ++k) {
       const float wk = __shfl_sync(0xffffffffu, w, k);
       const float4* src = pacc + (int64_t)(c0 + k) * QUADS;

@@ -511,23 +511,11 @@ struct SubWin {
   uint32_t z0, z1;     // int8: packed (K, V) zero points
 };
 
-// Sub-tile c's window entry in two steps, so that a caller can issue the block-table reads
-// and use them later: load_sub_ids reads the raw block ids, load_sub_params checks them and
-// reads the blocks' scales (and zero points). Both steps together are load_sub.
-template <int BS>
-__device__ __forceinline__ void load_sub_ids(const int32_t* btrow, int c, int t1, SubWin& w) {
-  if constexpr (BS == 8) {
-    w.p0 = btrow[2 * c];
-    w.p1 = c * kSub + 8 < t1 ? btrow[2 * c + 1] : -3;  // -3: second half absent
-  } else {
-    w.p0 = btrow[c * kSub / BS];
-  }
-}
-
 template <pa_dtype KV, int BS>
-__device__ __forceinline__ void load_sub_params(const DecodeArgs& a, int c, int t1, int kvh,
-                                                SubWin& w) {
-  auto one = [&](int& p, float& ks, float& vs, uint32_t& z) {
+__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
+                                         int t1, int kvh, SubWin& w) {
+  auto one = [&](int blk, int& p, float& ks, float& vs, uint32_t& z) {
+    p = btrow[blk];
     ks = 1.f;
     vs = 1.f;
     z = 0;
@@ -552,23 +540,16 @@ __device__ __forceinline__ void load_sub_params(const DecodeArgs& a, int c, int 
     }
   };
   if constexpr (BS == 8) {
-    one(w.p0, w.ks0, w.vs0, w.z0);
+    one(2 * c, w.p0, w.ks0, w.vs0, w.z0);
     if (c * kSub + 8 < t1) {
-      one(w.p1, w.ks1, w.vs1, w.z1);
+      one(2 * c + 1, w.p1, w.ks1, w.vs1, w.z1);
     } else {
       w.p1 = -3; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
     }
   } else {
-    one(w.p0, w.ks0, w.vs0, w.z0);
+    one(c * kSub / BS, w.p0, w.ks0, w.vs0, w.z0);
     w.p1 = w.p0; w.ks1 = w.ks0; w.vs1 = w.vs0; w.z1 = w.z0;
   }
-}
-
-template <pa_dtype KV, int BS>
-__device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
-                                         int t1, int kvh, SubWin& w) {
-  load_sub_ids<BS>(btrow, c, t1, w);
-  load_sub_params<KV, BS>(a, c, t1, kvh, w);
 }
 
 __device__ __forceinline__ void empty_sub(SubWin& w) {
@@ -759,17 +740,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
 }
 
 // =======================================================================================
-// Split path: plan kernel + persistent kernels; the partitions are merged by the warp
-// workers themselves (rows of up to 32 partitions) or by lse_reduce_kernel afterwards.
+// Split path: plan kernel + persistent kernels; lse_reduce_kernel merges the partitions.
 // =======================================================================================
 // Workspace of the split path (offsets in bytes, each region 256-aligned):
 //   [0]     uint32 fetch counter, uint32 total items
 //   list    int2 (seq, partition) per partition item, largest items first
 //   m, l    float [S][Hq][P];  acc float [S][Hq][P][kD]   (partials, as the CUDA-core path)
-//   arrive  uint32 [S][Hkv]: partials stored so far (warp workers merging in place)
-// Sequences with a single partition are written to `out` directly. The others are merged
-// by the warp that stores their last partial (warp workers, P <= 32), else by
-// lse_reduce_kernel afterwards (spread over every (seq, q head)).
+// Sequences with a single partition are written to `out` directly; the others are merged
+// by lse_reduce_kernel afterwards (spread over every (seq, q head)).
 struct PlanView {
   uint32_t* counters;  // [0] fetch, [1] total
   int2* list;
@@ -777,12 +755,9 @@ struct PlanView {
 
 // One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
 // largest first (full partitions, then partial ones by size; a counting sort), writes the
-// list, zeroes the fetch counter (and the arrival counters of the merging warp workers),
-// and writes out = 0 / lse = -inf for empty sequences. Largest first keeps the launch's
-// tail short: the last items taken are the smallest. (Keeping a sequence's partitions
-// together instead, so that merges happen early, measured 12 % slower on the batch-256
-// workload: full partitions then land in the tail.) The order affects scheduling only:
-// every item's result, and the merge order, depend on logical positions alone.
+// list, zeroes the fetch counter, and writes out = 0 / lse = -inf for empty sequences.
+// Largest first keeps the launch's tail short: the last items taken are the smallest.
+// The order affects scheduling only: every item's result depends on logical positions.
 __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const PlanView pl) {
   __shared__ int cnt[130], off[130];
   pdl_wait();
@@ -790,9 +765,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   const int P = a.part_tokens;
   const int nbk = P / kSub;  // sub-tiles of a full partition (<= 128)
   for (int i = threadIdx.x; i < 130; i += blockDim.x) cnt[i] = 0;
-  if (a.fused_merge)
-    for (int64_t i = threadIdx.x; i < (int64_t)a.num_seqs * a.num_kv_heads; i += blockDim.x)
-      a.arrive[i] = 0u;
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int ctx = checked_ctx(a, s);
@@ -827,66 +799,6 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
     }
     if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
-  }
-}
-
-// Merge of the partitions of the G query rows row0 .. row0+G-1 (one (sequence, kv head)),
-// run by the warp that stored the last of their partials; np <= 32. Lane p holds
-// partition p's running max and sum, lane k owns channel quad k (4 k .. 4 k + 3):
-// M = max_p m_p, L = sum_p 2^(m_p - M) l_p, out = sum_p 2^(m_p - M) acc_p / L. The
-// arithmetic and its order are those of lse_reduce_kernel, so the result does not depend
-// on which warp merges. Partials are read through L2 (ld.global.cg): other SMs wrote them
-// during this launch.
-__device__ __forceinline__ void merge_rows(const DecodeArgs& a, int64_t row0, int G, int np,
-                                           int lane) {
-  static_assert(kD == 128, "one channel quad per lane");
-  constexpr int R = 4;  // rows merged together: their partial reads are in flight at once
-  for (int g0 = 0; g0 < G; g0 += R) {
-    float M[R], w[R], lsum[R];
-    float4 acc[R];
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const bool live = g0 + r < G && lane < np;
-      const int64_t row = row0 + g0 + r;
-      const float mp = live ? __ldcg(a.part_m + row * a.max_parts + lane) : -INFINITY;
-      const float lp = live ? __ldcg(a.part_l + row * a.max_parts + lane) : 0.f;
-      float m = mp;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      M[r] = m;
-      w[r] = (live && m != -INFINITY) ? fast_exp2(mp - m) : 0.f;
-      lsum[r] = live ? w[r] * lp : 0.f;
-      acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
-    }
-#pragma unroll 2
-    for (int k = 0; k < np; ++k) {
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        if (g0 + r >= G) continue;  // warp-uniform
-        const float wk = __shfl_sync(0xffffffffu, w[r], k);
-        const float4 v = __ldcg(reinterpret_cast<const float4*>(
-                                    a.part_acc + (row0 + g0 + r) * a.max_parts * kD) +
-                                (int64_t)k * (kD / 4) + lane);
-        acc[r].x = fmaf(wk, v.x, acc[r].x); acc[r].y = fmaf(wk, v.y, acc[r].y);
-        acc[r].z = fmaf(wk, v.z, acc[r].z); acc[r].w = fmaf(wk, v.w, acc[r].w);
-      }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      if (g0 + r >= G) continue;
-      float l = lsum[r];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-      const int64_t row = row0 + g0 + r;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      const int64_t o = row * kD + 4 * lane;
-      store_out(a.out, a.out_dtype, o, acc[r].x * inv);
-      store_out(a.out, a.out_dtype, o + 1, acc[r].y * inv);
-      store_out(a.out, a.out_dtype, o + 2, acc[r].z * inv);
-      store_out(a.out, a.out_dtype, o + 3, acc[r].w * inv);
-      if (lane == 0 && a.lse_out != nullptr)
-        a.lse_out[row] = l > 0.f ? (M[r] + __log2f(l)) * kLn2 : -INFINITY;
-    }
   }
 }
 
@@ -1122,9 +1034,6 @@ constexpr int kWW = PA_TCW_WARPS;
 #ifndef PA_TCW_MIN_WARPS
 #define PA_TCW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
 #endif
-#ifndef PA_TCW_LOOKAHEAD
-#define PA_TCW_LOOKAHEAD 1  // 1: the item after the next one is fetched in steps (below)
-#endif
 
 template <pa_dtype KV>
 struct TcwCfg {
@@ -1132,16 +1041,11 @@ struct TcwCfg {
   static constexpr int kQBytes = 8 * kD * 2;  // one group's q, <= 8 heads
   static constexpr int kSmem =
       kWW * kNStage * TcCfg<KV>::kStage + kWW * kQBytes + kWW * (kNStage + 1) * 8 + 1024;
-  // CTAs per SM that shared memory allows (228 KB per SM, 1 KB reserved per CTA): the
-  // register budget is sized for that many (fp8 / int8: 14, bf16: 8), at most
-  // PA_TCW_MIN_WARPS warps
-  static constexpr int kResident = 233472 / (kSmem + 1024) < PA_TCW_MIN_WARPS / kWW
-                                       ? 233472 / (kSmem + 1024)
-                                       : PA_TCW_MIN_WARPS / kWW;
 };
 
+
 template <pa_dtype KV, int BS>
-__global__ void __launch_bounds__(kWW * 32, TcwCfg<KV>::kResident)
+__global__ void __launch_bounds__(kWW * 32, PA_TCW_MIN_WARPS / kWW)
 decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ CUtensorMap kmap,
                 const __grid_constant__ CUtensorMap vmap) {
   using C = TcCfg<KV>;
@@ -1215,59 +1119,23 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     }
   };
 
-  Item cur = fetch();
-  Item nxt = fetch();
-  SubWin cur_w, nxt_w;
-  load_window(cur, cur_w);
-  load_window(nxt, nxt_w);
-  copy_q(cur);
-
   int pslot = 0, pk = 0;
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
-  // Look-ahead: the item after `nxt` is fetched in three steps while the current item runs
-  // (work ticket at its start, list entry after its first consumed sub-tile, context
-  // length after its second), each step using what the previous step's read returned; at
-  // the item boundary only its block-table window is still read. `nxt` itself is always
-  // resolved, so the producer streams into it without waiting.
-  constexpr bool kLookahead = PA_TCW_LOOKAHEAD != 0;
-  uint32_t la_tk = 0;  // work ticket (lane 0 until broadcast)
-  int2 la_sp = make_int2(0, 0);
-  int la_ctx = 0;
-  int la_stage = kLookahead ? 0 : 3;
-  auto la_step = [&]() {
-    if (la_stage == 0) {
-      if (lane == 0) la_tk = atomicAdd(&pl.counters[0], 1u);
-    } else if (la_stage == 1) {
-      la_tk = __shfl_sync(0xffffffffu, la_tk, 0);
-      if (la_tk < total) la_sp = pl.list[la_tk / Hkv];
-    } else if (la_stage == 2) {
-      if (la_tk < total) la_ctx = a.context_lens[la_sp.x];
-    }
-    ++la_stage;
-  };
-  // the looked-ahead item (after its three steps); else the plain fetch
-  auto next_item = [&]() {
-    if constexpr (!kLookahead) return fetch();
-    Item v{0, 0, 0, 0, 0, 0, 0, 0};
-    if (la_tk < total) {
-      int ctx = la_ctx;  // clamped and flagged as checked_ctx does
-      if (ctx < 0 || ctx > a.max_context_len) {
-        if (threadIdx.x == 0) flag_error(PA_DEVERR_CONTEXT);
-        ctx = ctx < 0 ? 0 : a.max_context_len;
-      }
-      const int t0 = la_sp.y * P;
-      v.valid = 1;
-      v.s = la_sp.x;
-      v.kvh = (int)(la_tk % Hkv);
-      v.part = la_sp.y;
-      v.t1 = min(ctx, t0 + P);
-      v.c_begin = t0 / kSub;
-      v.nsub = (v.t1 + kSub - 1) / kSub - v.c_begin;
-      v.np = (ctx + P - 1) / P;
-    }
-    return v;
-  };
+  // The first item streams before the second is fetched (the producer stops at the end of
+  // an item whose successor is not resolved yet). Not with 8-token blocks, where the extra
+  // live state would spill.
+  constexpr bool kRamp = BS != 8;
+  Item cur = fetch(), nxt{0, 0, 0, 0, 0, 0, 0, 0};
+  SubWin cur_w, nxt_w;
+  load_window(cur, cur_w);
+  if constexpr (kRamp) {
+    empty_sub(nxt_w);
+  } else {
+    nxt = fetch();
+    load_window(nxt, nxt_w);
+  }
+  copy_q(cur);
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
@@ -1283,6 +1151,11 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     }
   };
   produce();
+  if constexpr (kRamp) {
+    nxt = fetch();
+    load_window(nxt, nxt_w);
+    produce();
+  }
 
   uint32_t qf[8][2];
   WarpAcc w;
@@ -1300,7 +1173,6 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
                                            a.scale_log2, qf);
     __syncwarp();
     if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
-    if (la_stage == 0) la_step();  // the work ticket of the item after nxt
     w.reset();
     for (int i = 0; i < cur.nsub; ++i) {
       const SubWin sw = shfl_sub<BS>(cur_w, i);
@@ -1317,7 +1189,6 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       __syncwarp();
       ++g_cons;
       produce();
-      if (la_stage < 3) la_step();
     }
     // ---- item done: its output (single partition) or its partial ----
 #pragma unroll
@@ -1371,29 +1242,11 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
         }
       }
     }
-    // ---- the last partial of a (sequence, kv head) to be stored merges them all ----
-    if (cur.np > 1 && a.fused_merge) {
-      __threadfence();  // this lane's partial stores, before the arrival below
-      __syncwarp();
-      uint32_t prev = 0;
-      if (lane == 0) {
-        __threadfence();
-        prev = atomicAdd(a.arrive + (int64_t)cur.s * Hkv + cur.kvh, 1u);
-      }
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev == (uint32_t)cur.np - 1) {
-        __threadfence();  // the other partials, stored before their arrivals, are visible
-        __syncwarp();
-        merge_rows(a, row0, G, cur.np, lane);
-      }
-    }
     // ---- advance ----
-    while (la_stage < 3) la_step();  // a short item: finish the look-ahead here
     cur = nxt;
     cur_w = nxt_w;
-    nxt = next_item();
+    nxt = fetch();
     load_window(nxt, nxt_w);
-    if (kLookahead) la_stage = 0;
     pslot = 0;
     produce();
   }

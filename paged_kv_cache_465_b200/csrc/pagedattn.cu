@@ -22,7 +22,7 @@ inline size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // Split-path workspace: plan area (counters, item list) followed by the partials
 // (m, l, acc) of every (seq, q head, partition).
 struct WorkspaceLayout {
-  size_t cnt_off, list_off, m_off, l_off, acc_off, arr_off, total;
+  size_t cnt_off, list_off, m_off, l_off, acc_off, total;
   int parts;
 };
 
@@ -75,7 +75,7 @@ bool desc_supported(const pa_decode_desc* d) {
 }
 
 WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
-  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0, 0};
+  WorkspaceLayout w{0, 0, 0, 0, 0, 0, 0};
   if (d->partition_size == 0 || max_context_len <= 0) return w;
   w.parts = (max_context_len + d->partition_size - 1) / d->partition_size;
   const size_t rows = (size_t)d->num_seqs * d->num_q_heads * w.parts;
@@ -84,33 +84,27 @@ WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
   w.m_off = w.list_off + round_up((size_t)d->num_seqs * w.parts * 8, 256);
   w.l_off = w.m_off + round_up(rows * sizeof(float), 256);
   w.acc_off = w.l_off + round_up(rows * sizeof(float), 256);
-  w.arr_off = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
-  w.total = w.arr_off + round_up((size_t)d->num_seqs * d->num_kv_heads * sizeof(uint32_t), 256);
+  w.total = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
   return w;
 }
 
 int pad_group(int G) { return G <= 1 ? 1 : G <= 2 ? 2 : G <= 4 ? 4 : G <= 8 ? 8 : 16; }
 
-#ifndef PA_TCW_FUSED_MERGE
-#define PA_TCW_FUSED_MERGE 0  // 1: warp workers merge rows of up to 32 partitions in place
-#endif
-
-// Which kernels a decode call runs: the tensor-core family (and which of its kernels) or
-// the CUDA-core path; whether the split path's partitions are merged in place by the warp
-// workers (rows of up to 32 partitions) or by a reduce launch afterwards.
+// Which kernels a decode call runs: the tensor-core family (and which of its kernels, the
+// persistent ones after a plan kernel) or the CUDA-core path; a split call ends with the
+// log-sum-exp reduce.
 struct DecodeRoute {
-  bool split, tc, fused_merge;
+  bool split, tc;
   tc::TcKind kind;
   int launches;  // kernel launches of the call
 };
 
 DecodeRoute route_for(const pa_decode_desc* d, const WorkspaceLayout& wl, int impl) {
-  DecodeRoute r{wl.total > 0, false, false, tc::kTcGrid, 1};
+  DecodeRoute r{wl.total > 0, false, tc::kTcGrid, 1};
   if (impl != 1 && tc_supported(d)) {
     r.tc = true;
     r.kind = tc_kind(d, r.split, impl);
-    r.fused_merge = PA_TCW_FUSED_MERGE && r.kind == tc::kTcWarps && wl.parts <= 32;
-    r.launches = (r.kind != tc::kTcGrid ? 2 : 1) + (r.split && !r.fused_merge ? 1 : 0);
+    r.launches = (r.kind != tc::kTcGrid ? 2 : 1) + (r.split ? 1 : 0);
   } else {
     r.launches = r.split ? 2 : 1;
   }
@@ -264,10 +258,6 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
       pl.counters = reinterpret_cast<uint32_t*>(ws + wl.cnt_off);
       pl.list = reinterpret_cast<int2*>(ws + wl.list_off);
       a.skip_single = 1;  // single-partition sequences are written by the kernel itself
-      if (r.fused_merge) {
-        a.fused_merge = 1;
-        a.arrive = reinterpret_cast<uint32_t*>(ws + wl.arr_off);
-      }
     }
     e = launch_tc(a, desc, grid, r.kind == tc::kTcGrid ? nullptr : &pl, r.kind, st);
   } else {
@@ -279,7 +269,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     }
   }
   if (e != cudaSuccess) return PA_ERR_CUDA;
-  if (split && !a.fused_merge && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
+  if (split && launch_reduce(a, D, st) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
 
