@@ -88,12 +88,10 @@ typedef enum {
 #define PA_DEVERR_ZERO 0x40      /* int8 zero point outside [-128, 127]                 */
 
 /*
- * partition_size value that lets the library choose the split for a decode call: the
- * largest of 512, 256, 128 and 64 tokens that gives at least two work items per resident
- * warp worker of the device (2 x SMs x 16) if every sequence were max_context_len long,
- * else 64; one pass (0) when max_context_len <= 64. The choice depends only on num_seqs,
- * num_kv_heads, max_context_len and the SM count, so results stay independent of where
- * blocks sit; paged_attn_partition_size() reports it.
+ * partition_size value that lets the library choose the split for a decode call: 512
+ * tokens when max_context_len > 512, else one pass (0). The choice depends only on
+ * max_context_len, so results stay independent of where blocks sit;
+ * paged_attn_partition_size() reports it.
  */
 #define PA_PARTITION_AUTO (-1)
 

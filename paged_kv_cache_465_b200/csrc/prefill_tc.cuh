@@ -66,13 +66,7 @@ constexpr int kOffK = kOffQ + kQT * kQBytes;
 constexpr int kOffV = kOffK + kKSt * kKVBytes;
 // Shared-memory map per cache type: a quantised cache adds a staging buffer for the codes
 // of one K tile and one V tile (TMA lands them there, the converter warps write the bf16
-// stages from them) and the tile's per-block scales and zero points. The staging buffer is
-// a ring of four quarters of 32 keys: the codes of a quarter of the next tile are loaded
-// as soon as the converters have read that quarter of the current one.
-#ifndef PA_PF_QUARTERS
-#define PA_PF_QUARTERS 4
-#endif
-constexpr int kQuarters = PA_PF_QUARTERS, kQKeys = kBN / kQuarters;  // 1, 2 or 4
+// stages from them) and the tile's per-block scales and zero points.
 template <bool QUANT>
 struct PfLayout {
   static constexpr int kThreads = QUANT ? 384 : 320;
@@ -82,9 +76,7 @@ struct PfLayout {
   static constexpr int kOffScale = kOffV8 + kStage8;            // float [2][32], int [2][32]
   static constexpr int kOffSide = kOffScale + (QUANT ? 512 : 0);  // float [4][2][32]
   static constexpr int kOffBar = kOffSide + (QUANT ? 1024 : 0);
-  static constexpr int kBarArea = 512;                          // barriers, tmem slot, flag
-  static constexpr int kSmem = kOffBar + kBarArea + 1024;       // + alignment slack
-  static_assert(kSmem <= 232448, "227 KB of shared memory per CTA");
+  static constexpr int kSmem = kOffBar + 256 + 1024;            // + barriers, + alignment slack
 };
 constexpr uint32_t kTileCols = 256;       // tensor memory of a query tile: S (P over its
 constexpr uint32_t kOCol = 128;           // first 64 columns) at column 0, O at 128
@@ -103,15 +95,14 @@ constexpr int kBarSF = kBarVE + kVSt;      // [query tile]
 constexpr int kBarP = kBarSF + kQT;        // [query tile], kBM arrivals
 constexpr int kBarO = kBarP + kQT;         // [query tile][ring]
 constexpr int kBarFin = kBarO + kQT * kORing;
-constexpr int kBarK8F = kBarFin + 1;       // quantised: [quarter] codes staged (TMA)
-constexpr int kBarK8E = kBarK8F + kQuarters;  // quantised: [quarter] staging read by converters
-constexpr int kBarV8F = kBarK8E + kQuarters;
-constexpr int kBarV8E = kBarV8F + kQuarters;
-constexpr int kBarSC = kBarV8E + kQuarters;   // quantised: [4] a tile's K / V scales for softmax
+constexpr int kBarK8F = kBarFin + 1;       // quantised: codes of the tile staged (TMA)
+constexpr int kBarK8E = kBarK8F + 1;       // quantised: staging read by the converters
+constexpr int kBarV8F = kBarK8E + 1;
+constexpr int kBarV8E = kBarV8F + 1;
+constexpr int kBarSC = kBarV8E + 1;        // quantised: [4] a tile's K / V scales for the softmax
 constexpr int kSideRing = 4;
 constexpr int kNumBars = kBarSC + kSideRing;
-static_assert(kQuarters == 1 || kQuarters == 2 || kQuarters == 4, "staging ring");
-static_assert(kNumBars * 8 + 8 <= PfLayout<true>::kBarArea, "barrier area");
+static_assert(kNumBars * 8 + 8 <= 256, "barrier area");
 
 // Instruction descriptors (kind::f16): f32 accumulator, bf16 A and B, M = 128.
 // S = Q K^T: A and B K-major, N = 128 keys. O += P V: A (P) from tensor memory, B (V)
@@ -348,9 +339,7 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       if (i >= kBarP && i < kBarP + kQT) count = kBM;
       // quantised: the bf16 stages are filled, and the staging read, by the converters
       if (QUANT && ((i >= kBarKF && i < kBarKF + kKSt) || (i >= kBarVF && i < kBarVF + kVSt) ||
-                    (i >= kBarK8E && i < kBarK8E + kQuarters) ||
-                    (i >= kBarV8E && i < kBarV8E + kQuarters) ||
-                    (i >= kBarSC && i < kBarSC + kSideRing)))
+                    i == kBarK8E || i == kBarV8E || (i >= kBarSC && i < kBarSC + kSideRing)))
         count = kConvThreads;
       mbar_init(bar(i), count);
     }
@@ -402,9 +391,6 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     int last_k[kKSt], last_v[kVSt];
     for (int i = 0; i < kKSt; ++i) last_k[i] = -1;
     for (int i = 0; i < kVSt; ++i) last_v[i] = -1;
-    int last_q[2][kQuarters];  // quantised: last tile whose codes each quarter received
-    for (int i = 0; i < kQuarters; ++i) last_q[0][i] = last_q[1][i] = -1;
-    constexpr int NBQ = NB_T / kQuarters;  // blocks per quarter
     int p_cur = fetch(0);
     bool ok = true;
     for (int j = 0; j < ntiles; ++j) {
@@ -414,36 +400,31 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
           (uint32_t)__popc(__ballot_sync(0xffffffffu, p_cur >= 0)) * 2u * BS * 128u;
       const int pb = __shfl_sync(0xffffffffu, p_cur, (lane >> 1) & 31);
 #pragma unroll
-      for (int kv = 0; kv < 2 && QUANT && ok; ++kv) {
-        // quantised: each quarter of the tile's codes goes to its staging quarter once the
-        // converters have read that quarter of the previous tile, with its blocks' scales
-        // (and zero points) beside them
-        for (int qq = 0; qq < kQuarters; ++qq) {
-          bool w = true;
-          if (lane == 0 && j >= 1) w = mbar_wait(bar((kv ? kBarV8E : kBarK8E) + qq), (j - 1) & 1);
-          if (!__shfl_sync(0xffffffffu, w, 0)) {
-            ok = false;
-            break;
-          }
-          const bool mine = lane >= qq * NBQ && lane < (qq + 1) * NBQ;  // this quarter's blocks
-          if (mine) {
-            float* sc = reinterpret_cast<float*>(smem + L::kOffScale) + kv * 32;
-            int* zp = reinterpret_cast<int*>(smem + L::kOffScale + 256) + kv * 32;
-            const int64_t bh = (int64_t)(p_cur >= 0 ? p_cur : 0) * a.num_kv_heads + kvh;
-            sc[lane] = p_cur >= 0 ? (kv ? a.v_scales : a.k_scales)[bh] : 1.f;  // absent: masked
-            zp[lane] = (KV == PA_INT8 && p_cur >= 0) ? (kv ? a.v_zeros : a.k_zeros)[bh] : 0;
-          }
-          __syncwarp();  // the scales before the quarter's arrival below
-          const uint32_t qbytes =
-              (uint32_t)__popc(__ballot_sync(0xffffffffu, mine && p_cur >= 0)) * BS * 128u;
-          const uint32_t fb = bar((kv ? kBarV8F : kBarK8F) + qq);
-          if (lane == 0) mbar_arrive_tx(fb, qbytes);  // one byte per element
-          __syncwarp();
-          if (mine && p_cur >= 0)
-            tma_load_2d(smem_u32(smem + (kv ? L::kOffV8 : L::kOffK8)) + lane * BS * 128,
-                        kv ? &vmap : &kmap, 0, (p_cur * a.num_kv_heads + kvh) * BS, fb);
-          last_q[kv][qq] = j;
+      for (int kv = 0; kv < 2 && QUANT; ++kv) {
+        // quantised: the tile's codes go to the staging buffer once the converters have
+        // read the previous tile, with the blocks' scales (and zero points) beside them
+        bool w = true;
+        if (lane == 0 && j >= 1) w = mbar_wait(bar(kv ? kBarV8E : kBarK8E), (j - 1) & 1);
+        if (!__shfl_sync(0xffffffffu, w, 0)) {
+          ok = false;
+          break;
         }
+        if (lane < NB_T) {
+          float* sc = reinterpret_cast<float*>(smem + L::kOffScale) + kv * 32;
+          int* zp = reinterpret_cast<int*>(smem + L::kOffScale + 256) + kv * 32;
+          const int64_t bh = (int64_t)(p_cur >= 0 ? p_cur : 0) * a.num_kv_heads + kvh;
+          sc[lane] = p_cur >= 0 ? (kv ? a.v_scales : a.k_scales)[bh] : 1.f;  // absent: masked
+          zp[lane] = (KV == PA_INT8 && p_cur >= 0) ? (kv ? a.v_zeros : a.k_zeros)[bh] : 0;
+        }
+        __syncwarp();
+        const uint32_t fb = bar(kv ? kBarV8F : kBarK8F);
+        if (lane == 0) mbar_arrive_tx(fb, bytes / 2);  // one byte per element
+        __syncwarp();
+        if (lane < NB_T && p_cur >= 0)
+          tma_load_2d(smem_u32(smem + (kv ? L::kOffV8 : L::kOffK8)) + lane * BS * 128,
+                      kv ? &vmap : &kmap, 0, (p_cur * a.num_kv_heads + kvh) * BS, fb);
+        if (kv) last_v[0] = j;
+        else last_k[0] = j;
       }
 #pragma unroll
       for (int kv = 0; kv < 2 && !QUANT; ++kv) {
@@ -479,10 +460,8 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
     if (lane == 0 && *dead) {
       // copies still in flight complete before the CTA's shared memory is released
       if (QUANT) {
-        for (int kv = 0; kv < 2; ++kv)
-          for (int qq = 0; qq < kQuarters; ++qq)
-            if (last_q[kv][qq] >= 0)
-              mbar_wait(bar((kv ? kBarV8F : kBarK8F) + qq), last_q[kv][qq] & 1);
+        if (last_k[0] >= 0) mbar_wait(bar(kBarK8F), last_k[0] & 1);
+        if (last_v[0] >= 0) mbar_wait(bar(kBarV8F), last_v[0] & 1);
       } else {
         for (int i = 0; i < kKSt; ++i)
           if (last_k[i] >= 0) mbar_wait(bar(kBarKF + i), (last_k[i] / kKSt) & 1);
@@ -578,61 +557,55 @@ prefill_tc_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap qmap,
       for (int kv = 0; kv < 2; ++kv) {
         const int nst = kv ? kVSt : kKSt;
         const int st = j % nst;
-        bool w = !*dead;
+        bool w = !*dead && mbar_wait(bar(kv ? kBarV8F : kBarK8F), j & 1);
         if (w && j >= nst) w = mbar_wait(bar((kv ? kBarVE : kBarKE) + st), ((j / nst) - 1) & 1);
-        const uint8_t* src = smem + (kv ? L::kOffV8 : L::kOffK8);
-        const float* sc = reinterpret_cast<const float*>(smem + L::kOffScale) + kv * 32;
-        const int* zp = reinterpret_cast<const int*>(smem + L::kOffScale + 256) + kv * 32;
-        const uint32_t dst = (kv ? sV : sK) + st * kKVBytes;
-        constexpr int NBQ = NB_T / kQuarters;  // blocks per quarter
-        for (int qq = 0; qq < kQuarters && w; ++qq) {
-          w = !*dead && mbar_wait(bar((kv ? kBarV8F : kBarK8F) + qq), j & 1);
-          if (!w) break;
-#pragma unroll
-          for (int it = 0; it < kQKeys * 8 / kConvThreads; ++it) {
-            const int chunk = ct + kConvThreads * it;
-            const int t = qq * kQKeys + (chunk >> 3), q8 = chunk & 7;
-            const uint4 raw = *reinterpret_cast<const uint4*>(src + t * 128 + q8 * 16);
-            const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
-            uint32_t o[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              float f[4];
-              if constexpr (KV == PA_INT8) {
-                const float z = (float)zp[t / BS];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) f[e] = (float)(int8_t)(wd[k] >> (8 * e)) - z;
-              } else {  // E4M3 -> f16 -> f32, both exact
-                f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] & 0xffffu)), f[0], f[1]);
-                f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] >> 16)), f[2], f[3]);
-              }
-              o[2 * k] = pack_bf16x2(f[0], f[1]);
-              o[2 * k + 1] = pack_bf16x2(f[2], f[3]);
-            }
-            // channels 16 q8 .. 16 q8 + 15: half q8 / 4 of the channels, 16-byte chunks
-            // 2 (q8 % 4) and 2 (q8 % 4) + 1 of the key's 128-byte row, swizzled by row % 8
-            const uint32_t row = dst + (q8 >> 2) * kKVSlab + t * 128;
-            const int c0 = 2 * (q8 & 3);
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         ::"r"(row + ((c0 ^ (t & 7)) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]),
-                           "r"(o[3]) : "memory");
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
-                         ::"r"(row + (((c0 + 1) ^ (t & 7)) << 4)), "r"(o[4]), "r"(o[5]), "r"(o[6]),
-                           "r"(o[7]) : "memory");
-          }
-          // the quarter's block scales for the softmax (slot j % 4 is free: the softmax of
-          // tile j - 4 finished before the S products of tile j - 2, which freed this
-          // stage), read before the producer may overwrite them
-          if (ct < NBQ)
-            reinterpret_cast<float*>(smem + L::kOffSide)[((j % kSideRing) * 2 + kv) * 32 +
-                                                         qq * NBQ + ct] = sc[qq * NBQ + ct];
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          mbar_arrive(bar((kv ? kBarV8E : kBarK8E) + qq));  // staging quarter read
-        }
         if (!w) {
           ok = false;
           break;
         }
+        const uint8_t* src = smem + (kv ? L::kOffV8 : L::kOffK8);
+        const float* sc = reinterpret_cast<const float*>(smem + L::kOffScale) + kv * 32;
+        const int* zp = reinterpret_cast<const int*>(smem + L::kOffScale + 256) + kv * 32;
+        const uint32_t dst = (kv ? sV : sK) + st * kKVBytes;
+#pragma unroll 4
+        for (int it = 0; it < kBN * 8 / kConvThreads; ++it) {
+          const int chunk = ct + kConvThreads * it;
+          const int t = chunk >> 3, q8 = chunk & 7;
+          const uint4 raw = *reinterpret_cast<const uint4*>(src + t * 128 + q8 * 16);
+          const uint32_t wd[4] = {raw.x, raw.y, raw.z, raw.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float f[4];
+            if constexpr (KV == PA_INT8) {
+              const float z = (float)zp[t / BS];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) f[e] = (float)(int8_t)(wd[k] >> (8 * e)) - z;
+            } else {  // E4M3 -> f16 -> f32, both exact
+              f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] & 0xffffu)), f[0], f[1]);
+              f16x2_to_f32(e4m3x2_to_f16x2((uint16_t)(wd[k] >> 16)), f[2], f[3]);
+            }
+            o[2 * k] = pack_bf16x2(f[0], f[1]);
+            o[2 * k + 1] = pack_bf16x2(f[2], f[3]);
+          }
+          // channels 16 q8 .. 16 q8 + 15: half q8 / 4 of the channels, 16-byte chunks
+          // 2 (q8 % 4) and 2 (q8 % 4) + 1 of the key's 128-byte row, swizzled by row % 8
+          const uint32_t row = dst + (q8 >> 2) * kKVSlab + t * 128;
+          const int c0 = 2 * (q8 & 3);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(row + ((c0 ^ (t & 7)) << 4)), "r"(o[0]), "r"(o[1]), "r"(o[2]),
+                         "r"(o[3]) : "memory");
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};"
+                       ::"r"(row + (((c0 + 1) ^ (t & 7)) << 4)), "r"(o[4]), "r"(o[5]), "r"(o[6]),
+                         "r"(o[7]) : "memory");
+        }
+        // the tile's block scales for the softmax (slot j % 4 is free: the softmax of tile
+        // j - 4 finished before the S products of tile j - 2, which freed this stage)
+        if (ct < NB_T)
+          reinterpret_cast<float*>(smem + L::kOffSide)[((j % kSideRing) * 2 + kv) * 32 + ct] =
+              sc[ct];
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        mbar_arrive(bar(kv ? kBarV8E : kBarK8E));           // staging read
         mbar_arrive(bar((kv ? kBarVF : kBarKF) + st));       // bf16 stage written
       }
       if (ok) mbar_arrive(bar(kBarSC + j % kSideRing));     // K and V scales of tile j

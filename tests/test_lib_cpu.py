@@ -258,27 +258,15 @@ def test_prefill_host_validation_without_device(pa):
 
 
 def test_library_chosen_partition(pa):
-    """PA_PARTITION_AUTO: the largest of 512/256/128/64 tokens giving at least two items per
-    resident warp worker (2 x SMs x 16; 148 SMs when no device answers) for contexts of
-    max_context_len, else 64; one pass up to 64 tokens. The workspace and launch count
-    follow the chosen partition."""
-    target = 2 * 148 * 16
-
-    def rule(S, Hkv, L):
-        if L <= 64:
-            return 0
-        for p in (512, 256, 128):
-            if S * Hkv * -(-L // p) >= target:
-                return p
-        return 64
-
-    for S, Hkv, L, B in [(32, 8, 4096, 16), (256, 8, 8192, 16), (100, 8, 250, 16), (8, 8, 131072, 16),
-                         (1, 1, 64, 16), (1, 1, 65, 8), (3, 2, 40, 32), (4096, 8, 600, 32),
-                         (64, 8, 1000, 8)]:
+    """PA_PARTITION_AUTO: 512-token partitions when a context may be longer than 512 tokens,
+    else one pass; the workspace and the launch count follow the chosen partition."""
+    for S, Hkv, L, B in [(32, 8, 4096, 16), (256, 8, 8192, 16), (100, 8, 250, 16),
+                         (8, 8, 131072, 16), (1, 1, 512, 16), (1, 1, 513, 8), (3, 2, 40, 32),
+                         (4096, 8, 600, 32), (64, 8, 1000, 8)]:
         d = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, pa.PARTITION_AUTO, pa.PA_BF16,
                          pa.PA_BF16, pa.PA_BF16, block_size=B)
         p = pa.partition_size_for(d, L)
-        assert p == rule(S, Hkv, L), (S, Hkv, L, p)
+        assert p == (512 if L > 512 else 0), (S, Hkv, L, p)
         e = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, p, pa.PA_BF16, pa.PA_BF16,
                          pa.PA_BF16, block_size=B)
         assert pa.workspace_size(d, L) == pa.workspace_size(e, L)
