@@ -123,6 +123,9 @@ struct DecodeArgs {
   int max_context_len;
   int final_pass;    // 1: one item covers the whole context, write out directly
   int skip_single;   // split path: single-partition sequences were written directly
+  // split path, warp workers: warp w < static_seqs * Hkv takes partition 0 of (sequence
+  // w / Hkv, kv head w % Hkv) as its first item, without the plan; the plan lists the rest
+  int static_seqs;
   pa_dtype q_dtype, out_dtype;
   // prefill rows (CUDA-core kernel only): work row s is new token s; the tokens of
   // sequence q are rows query_start[q] .. query_start[q+1]-1, the last ones of its context

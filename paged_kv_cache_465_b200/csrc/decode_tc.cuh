@@ -511,11 +511,13 @@ struct SubWin {
   uint32_t z0, z1;     // int8: packed (K, V) zero points
 };
 
+// Block ids, scales and zero points are read through L2 (ld.global.cg): each is read once
+// per item, and a warp worker reads its first item's before the plan kernel has finished.
 template <pa_dtype KV, int BS>
 __device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btrow, int c,
                                          int t1, int kvh, SubWin& w) {
   auto one = [&](int blk, int& p, float& ks, float& vs, uint32_t& z) {
-    p = btrow[blk];
+    p = __ldcg(btrow + blk);
     ks = 1.f;
     vs = 1.f;
     z = 0;
@@ -526,10 +528,10 @@ __device__ __forceinline__ void load_sub(const DecodeArgs& a, const int32_t* btr
     }
     if constexpr (KV != PA_BF16) {
       const int64_t bh = (int64_t)p * a.num_kv_heads + kvh;
-      ks = a.k_scales[bh];
-      vs = a.v_scales[bh];
+      ks = __ldcg(a.k_scales + bh);
+      vs = __ldcg(a.v_scales + bh);
       if constexpr (KV == PA_INT8) {
-        const int kz = a.k_zeros[bh], vz = a.v_zeros[bh];
+        const int kz = __ldcg(a.k_zeros + bh), vz = __ldcg(a.v_zeros + bh);
         if (!zero_in_range(kz) || !zero_in_range(vz)) {
           flag_error(PA_DEVERR_ZERO);
           p = -1;
@@ -744,13 +746,14 @@ decode_tc_kernel(const DecodeArgs a, const __grid_constant__ CUtensorMap kmap,
 // =======================================================================================
 // Workspace of the split path (offsets in bytes, each region 256-aligned):
 //   [0]     uint32 fetch counter, uint32 total items
-//   list    int2 (seq, partition) per partition item, largest items first
+//   list    int4 (seq, partition, context length, 0) per partition item, largest first
+//           (the context length rides along so that a worker's fetch needs one read less)
 //   m, l    float [S][Hq][P];  acc float [S][Hq][P][kD]   (partials, as the CUDA-core path)
 // Sequences with a single partition are written to `out` directly; the others are merged
 // by lse_reduce_kernel afterwards (spread over every (seq, q head)).
 struct PlanView {
   uint32_t* counters;  // [0] fetch, [1] total
-  int2* list;
+  int4* list;
 };
 
 // One CTA of 1024 threads: counts partitions per size (sub-tiles per item), orders them
@@ -776,9 +779,11 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
       }
       continue;
     }
+    // partition 0 of the first static_seqs sequences is a warp's first item already
+    const int skip = s < a.static_seqs ? 1 : 0;
     const int full = ctx / P, rem = ctx % P;
-    if (full) atomicAdd(&cnt[nbk], full);
-    if (rem) atomicAdd(&cnt[(rem + kSub - 1) / kSub], 1);
+    if (full > skip) atomicAdd(&cnt[nbk], full - skip);
+    if (rem && (full > 0 || !skip)) atomicAdd(&cnt[(rem + kSub - 1) / kSub], 1);
   }
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -793,18 +798,20 @@ __global__ void __launch_bounds__(1024) plan_kernel(const DecodeArgs a, const Pl
   __syncthreads();
   for (int s = threadIdx.x; s < a.num_seqs; s += blockDim.x) {
     const int ctx = checked_ctx(a, s);
+    const int skip = s < a.static_seqs ? 1 : 0;
     const int full = ctx / P, rem = ctx % P;
-    if (full) {
-      const int base = atomicAdd(&off[nbk], full);
-      for (int j = 0; j < full; ++j) pl.list[base + j] = make_int2(s, j);
+    if (full > skip) {
+      const int base = atomicAdd(&off[nbk], full - skip);
+      for (int j = skip; j < full; ++j) pl.list[base + j - skip] = make_int4(s, j, ctx, 0);
     }
-    if (rem) pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int2(s, full);
+    if (rem && (full > 0 || !skip))
+      pl.list[atomicAdd(&off[(rem + kSub - 1) / kSub], 1)] = make_int4(s, full, ctx, 0);
   }
 }
 
 // Work item slot shared by the CTA (written by thread 0 between barriers).
 struct ItemSlot {
-  int valid, s, part, kvh;
+  int valid, s, part, kvh, ctx;
 };
 
 // Persistent CTAs: 16-token blocks only (a block is one sub-tile).
@@ -838,10 +845,10 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
   // thread 0: take the next item from the shared counter into slot `sl`, start its q copy
   auto fetch = [&](int sl) {
     const uint32_t it = atomicAdd(&pl.counters[0], 1u);
-    ItemSlot x{0, 0, 0, 0};
+    ItemSlot x{0, 0, 0, 0, 0};
     if (it < total) {
-      const int2 sp = pl.list[it / Hkv];
-      x = ItemSlot{1, sp.x, sp.y, (int)(it % Hkv)};
+      const int4 sp = pl.list[it / Hkv];
+      x = ItemSlot{1, sp.x, sp.y, (int)(it % Hkv), sp.z};
       const uint32_t qb = qbars + 8 * sl;
       mbar_arrive_tx(qb, (uint32_t)(G * kD * 2));
       bulk_load_1d(smem_u32(qbuf + sl * C::kQBytes),
@@ -868,7 +875,7 @@ decode_tc_persistent(const DecodeArgs a, const PlanView pl,
     const ItemSlot x = slots[sl];
     WarpItem v{x.valid, x.s, x.kvh, x.part, 0, 0, 0, 0};
     if (x.valid) {
-      const int ctx = checked_ctx(a, x.s);
+      const int ctx = x.ctx;  // checked by the plan kernel
       const int t0 = x.part * P;
       v.t1 = min(ctx, t0 + P);
       v.b_begin = t0 / kSub;
@@ -1069,13 +1076,38 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
   __syncwarp();
-  pdl_wait();  // the plan kernel's list and counters
-  const uint32_t total = pl.counters[1];
+  uint32_t total = 0;  // items in the plan's list, read once the plan has finished
   const uint64_t policy = evict_first_policy();
 
   // an item's sub-tiles are c_begin + k, k < nsub (<= 32)
   struct Item {
     int valid, s, kvh, part, t1, c_begin, nsub, np;
+  };
+  // This warp's first item: partition 0 of (sequence gw / Hkv, kv head gw % Hkv) for
+  // gw < static_seqs * Hkv. It needs no plan, so it is read and starts streaming before the
+  // plan kernel has finished; its inputs were written before the plan kernel started (that
+  // kernel waits for its predecessors before it lets this one launch), and they are read
+  // through L2.
+  auto static_item = [&]() {
+    Item v{0, 0, 0, 0, 0, 0, 0, 0};
+    const int gw = blockIdx.x * kWW + warp;
+    if (gw < a.static_seqs * Hkv) {
+      const int s = gw / Hkv;
+      int ctx = __ldcg(a.context_lens + s);  // clamped and flagged as checked_ctx does
+      if (ctx < 0 || ctx > a.max_context_len) {
+        if (lane == 0) flag_error(PA_DEVERR_CONTEXT);
+        ctx = ctx < 0 ? 0 : a.max_context_len;
+      }
+      if (ctx > 0) {
+        v.valid = 1;
+        v.s = s;
+        v.kvh = gw % Hkv;
+        v.t1 = min(ctx, P);
+        v.nsub = (v.t1 + kSub - 1) / kSub;
+        v.np = (ctx + P - 1) / P;
+      }
+    }
+    return v;
   };
   auto fetch = [&]() {
     uint32_t it = 0;
@@ -1083,8 +1115,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     it = __shfl_sync(0xffffffffu, it, 0);
     Item v{0, 0, 0, 0, 0, 0, 0, 0};
     if (it < total) {
-      const int2 sp = pl.list[it / Hkv];
-      const int ctx = checked_ctx(a, sp.x);
+      const int4 sp = pl.list[it / Hkv];
+      const int ctx = sp.z;  // checked by the plan kernel
       const int t0 = sp.y * P;
       v.valid = 1;
       v.s = sp.x;
@@ -1123,19 +1155,13 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
   // The first item streams before the second is fetched (the producer stops at the end of
-  // an item whose successor is not resolved yet). Not with 8-token blocks, where the extra
-  // live state would spill.
+  // an item whose successor is not resolved yet), and before the plan has finished. Not
+  // with 8-token blocks, where the extra live state would spill: there both items are
+  // resolved first.
   constexpr bool kRamp = BS != 8;
-  Item cur = fetch(), nxt{0, 0, 0, 0, 0, 0, 0, 0};
+  Item cur = static_item(), nxt{0, 0, 0, 0, 0, 0, 0, 0};
   SubWin cur_w, nxt_w;
-  load_window(cur, cur_w);
-  if constexpr (kRamp) {
-    empty_sub(nxt_w);
-  } else {
-    nxt = fetch();
-    load_window(nxt, nxt_w);
-  }
-  copy_q(cur);
+  empty_sub(nxt_w);
   auto produce = [&]() {
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
@@ -1150,11 +1176,29 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       ++pk;
     }
   };
-  produce();
+  auto start = [&]() {
+    load_window(cur, cur_w);
+    copy_q(cur);
+    produce();
+  };
   if constexpr (kRamp) {
+    if (cur.valid) start();
+    pdl_wait();  // the plan kernel's list and counters
+    total = pl.counters[1];
+    if (!cur.valid) {  // no static item: the first comes from the list
+      cur = fetch();
+      if (cur.valid) start();
+    }
     nxt = fetch();
     load_window(nxt, nxt_w);
     produce();
+  } else {
+    pdl_wait();
+    total = pl.counters[1];
+    if (!cur.valid) cur = fetch();
+    nxt = fetch();
+    load_window(nxt, nxt_w);
+    start();
   }
 
   uint32_t qf[8][2];
@@ -1363,7 +1407,23 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   }
   const int sms = sm_count();
   if (sms <= 0 || pl == nullptr) return cudaErrorInvalidValue;
-  cudaError_t e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, a, *pl);
+  cudaError_t e;
+  if (kind == kTcWarps) {
+    static DeviceCache slots;
+    int per_sm = 0;
+    e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, slots, &per_sm);
+    if (e != cudaSuccess) return e;
+    const int warps = sms * per_sm * kWW;
+    DecodeArgs w = a;
+    w.static_seqs = min(warps / a.num_kv_heads, a.num_seqs);  // whole sequences only
+    e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, w, *pl);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32),
+                   TcwCfg<KV>::kSmem, st, w, *pl, km, vm);
+    if (e != cudaSuccess) return e;
+    return cudaGetLastError();
+  }
+  e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, a, *pl);
   if (e != cudaSuccess) return e;
   if (kind == kTcCta) {
     if constexpr (BS != kSub) return cudaErrorInvalidValue;
@@ -1373,14 +1433,6 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
     if (e != cudaSuccess) return e;
     e = launch_pdl(decode_tc_persistent<KV>, dim3(sms * per_sm), dim3(kNW * 32), C::kPSmem, st,
                    a, *pl, km, vm);
-    if (e != cudaSuccess) return e;
-  } else {
-    static DeviceCache slots;
-    int per_sm = 0;
-    e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, slots, &per_sm);
-    if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32),
-                   TcwCfg<KV>::kSmem, st, a, *pl, km, vm);
     if (e != cudaSuccess) return e;
   }
   return cudaGetLastError();

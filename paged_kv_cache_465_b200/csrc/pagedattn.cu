@@ -77,7 +77,7 @@ WorkspaceLayout layout_for(const pa_decode_desc* d, int max_context_len) {
   const size_t rows = (size_t)d->num_seqs * d->num_q_heads * w.parts;
   w.cnt_off = 0;
   w.list_off = 256;
-  w.m_off = w.list_off + round_up((size_t)d->num_seqs * w.parts * 8, 256);
+  w.m_off = w.list_off + round_up((size_t)d->num_seqs * w.parts * 16, 256);
   w.l_off = w.m_off + round_up(rows * sizeof(float), 256);
   w.acc_off = w.l_off + round_up(rows * sizeof(float), 256);
   w.total = w.acc_off + round_up(rows * (size_t)d->head_dim * sizeof(float), 256);
@@ -252,7 +252,7 @@ pa_status paged_attn_decode(const void* q, const void* k_cache, const void* v_ca
     if (r.kind != tc::kTcGrid) {
       char* ws = static_cast<char*>(workspace);
       pl.counters = reinterpret_cast<uint32_t*>(ws + wl.cnt_off);
-      pl.list = reinterpret_cast<int2*>(ws + wl.list_off);
+      pl.list = reinterpret_cast<int4*>(ws + wl.list_off);
       a.skip_single = 1;  // single-partition sequences are written by the kernel itself
     }
     e = launch_tc(a, desc, grid, r.kind == tc::kTcGrid ? nullptr : &pl, r.kind, st);
