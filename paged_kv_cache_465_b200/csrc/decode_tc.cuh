@@ -1042,12 +1042,20 @@ constexpr int kWW = PA_TCW_WARPS;
 #define PA_TCW_MIN_WARPS 16  // resident warps per SM the register budget is sized for
 #endif
 
+// Shared memory of one CTA of kWW warp workers: their TMA rings (1024-byte aligned, the
+// 128-byte swizzle's period), then one q buffer per warp sized for the call's group (G
+// heads of kD bf16), then each warp's barriers, plus alignment slack. Sizing the q buffers
+// by G lets more workers, hence more bytes in flight, fit in an SM's shared memory (fp8
+// with four query heads per kv head: 15 warps per SM instead of 14). (Two workers per CTA
+// sharing the slack would fit 16, but made ptxas spill.)
 template <pa_dtype KV>
 struct TcwCfg {
   static constexpr int kNStage = KV == PA_FP8_E4M3 ? PA_TCW_STAGE_FP8 : PA_TCW_STAGE_BF16;
-  static constexpr int kQBytes = 8 * kD * 2;  // one group's q, <= 8 heads
-  static constexpr int kSmem =
-      kWW * kNStage * TcCfg<KV>::kStage + kWW * kQBytes + kWW * (kNStage + 1) * 8 + 1024;
+  __host__ __device__ static constexpr int qbytes(int G) { return G * kD * 2; }
+  __host__ __device__ static constexpr int smem(int G) {
+    return kWW * kNStage * TcCfg<KV>::kStage + kWW * qbytes(G) + kWW * (kNStage + 1) * 8 + 1024;
+  }
+  static constexpr int kMaxSmem = smem(8);
 };
 
 
@@ -1065,8 +1073,9 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   const int gq = lane >> 2, tq = lane & 3;
   const int G = a.group, Hkv = a.num_kv_heads, P = a.part_tokens;
   const uint32_t wtiles = smem_u32(smem + warp * NST * STAGE);
-  uint8_t* qbuf = smem + kWW * NST * STAGE + warp * TcwCfg<KV>::kQBytes;
-  const uint32_t bars = smem_u32(smem + kWW * NST * STAGE + kWW * TcwCfg<KV>::kQBytes) +
+  const int qbytes = TcwCfg<KV>::qbytes(a.group);
+  uint8_t* qbuf = smem + kWW * NST * STAGE + warp * qbytes;
+  const uint32_t bars = smem_u32(smem + kWW * NST * STAGE + kWW * qbytes) +
                         warp * (NST + 1) * 8;
   const uint32_t qbar = bars + NST * 8;
   if (lane == 0) {
@@ -1360,9 +1369,12 @@ inline int sm_count() {
 // persistent warp workers.
 enum TcKind { kTcGrid = 0, kTcCta = 1, kTcWarps = 2 };
 
+// `smem_limit`: the kernel's dynamic shared-memory limit (the largest any launch uses);
+// `smem`: this launch's size, for the occupancy.
 template <typename K>
-inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm, int smem_limit = 0) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       smem_limit > smem ? smem_limit : smem);
   if (e != cudaSuccess) return e;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, kernel, threads, smem);
   if (e == cudaSuccess && *per_sm <= 0) e = cudaErrorInvalidConfiguration;
@@ -1374,14 +1386,14 @@ inline cudaError_t occupancy(K kernel, int threads, int smem, int* per_sm) {
 // is the kernel's per-device cache; concurrent first calls store the same values).
 template <typename K>
 inline cudaError_t resident_per_sm(K kernel, int threads, int smem, DeviceCache& slots,
-                                   int* per_sm) {
+                                   int* per_sm, int smem_limit = 0) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   int n = slots[dev].load(std::memory_order_relaxed);
   if (n == 0) {
-    e = occupancy(kernel, threads, smem, &n);
+    e = occupancy(kernel, threads, smem, &n, smem_limit);
     if (e != cudaSuccess) return e;
     slots[dev].store(n, std::memory_order_relaxed);
   }
@@ -1409,17 +1421,21 @@ inline cudaError_t launch_tc_kv(const DecodeArgs& a, const pa_decode_desc* d, di
   if (sms <= 0 || pl == nullptr) return cudaErrorInvalidValue;
   cudaError_t e;
   if (kind == kTcWarps) {
-    static DeviceCache slots;
+    // occupancy depends on the group's q buffers: measured (and cached) per group size; the
+    // kernel's shared-memory limit is set for the largest group
+    static DeviceCache slots_g[8];
     int per_sm = 0;
-    e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, TcwCfg<KV>::kSmem, slots, &per_sm);
+    const int gsz = TcwCfg<KV>::smem(a.group);
+    e = resident_per_sm(decode_tc_warps<KV, BS>, kWW * 32, gsz, slots_g[a.group - 1], &per_sm,
+                        TcwCfg<KV>::kMaxSmem);
     if (e != cudaSuccess) return e;
     const int warps = sms * per_sm * kWW;
     DecodeArgs w = a;
     w.static_seqs = min(warps / a.num_kv_heads, a.num_seqs);  // whole sequences only
     e = launch_pdl(plan_kernel, dim3(1), dim3(1024), 0, st, w, *pl);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32),
-                   TcwCfg<KV>::kSmem, st, w, *pl, km, vm);
+    e = launch_pdl(decode_tc_warps<KV, BS>, dim3(sms * per_sm), dim3(kWW * 32), gsz, st, w,
+                   *pl, km, vm);
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
   }
