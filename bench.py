@@ -669,13 +669,16 @@ def _extra_workloads(torch, pa, args, flush):
     base = workloads.WORKLOADS["b256"]
     runs += [(f"b256_bs{B}", base.scaled(block_size=B, num_blocks=base.num_blocks * 16 // B))
              for B in (8, 32)]
+    # the long-context workload with the library's own split (PA_PARTITION_AUTO) instead of
+    # the configured 512 tokens
+    runs += [("long_auto", workloads.WORKLOADS["long"].scaled(partition_size=-1))]
     for name, wl in runs:
         draw = workloads.draw(wl)
         sc = DeviceScenario(draw, draw_seqs=[] if name not in ("tiny", "shared") else None)
         for _ in range(3):
             flush()
             sc.step()
-        steps = 50 if name == "long" else 200
+        steps = 50 if name.startswith("long") else 200
         total, dec = _time_steps(torch, sc, steps, flush)
         b = sc.step_bytes()
         gbs = b["kv"] * steps / total / 1e9

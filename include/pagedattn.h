@@ -88,10 +88,10 @@ typedef enum {
 #define PA_DEVERR_ZERO 0x40      /* int8 zero point outside [-128, 127]                 */
 
 /*
- * partition_size value that lets the library choose the split for a decode call: 512
- * tokens when max_context_len > 512, else one pass (0). The choice depends only on
- * max_context_len, so results stay independent of where blocks sit;
- * paged_attn_partition_size() reports it.
+ * partition_size value that lets the library choose the split for a decode call: one
+ * pass (0) when max_context_len <= 512; else 512 tokens when num_seqs * num_kv_heads >=
+ * 1024, else 1024. The choice depends only on the descriptor and max_context_len, so
+ * results stay independent of where blocks sit; paged_attn_partition_size() reports it.
  */
 #define PA_PARTITION_AUTO (-1)
 
@@ -285,11 +285,12 @@ pa_status pa_device_error(int* bits_out, void* stream);
 
 /*
  * Selects the decode kernels used by later paged_attn_decode calls in this process:
- * 0 = automatic (tensor cores for bf16 / fp8 caches where the shape is supported, else the
- * CUDA-core fp32 path), 1 = CUDA-core path only, 2 = same as 0, 3 / 4 / 5 = tensor cores
- * with a fixed kernel where the call allows it: 3 one CTA per work item, 4 persistent CTAs
- * that share each work item (split path, partitions <= 2048 tokens), 5 persistent warp
- * workers, one work item per warp (split path, partitions <= 512 tokens). All compute the
+ * 0 = automatic (tensor cores for bf16 / fp8 / int8 caches where the shape is supported:
+ * persistent warp workers for partitions <= 512 tokens, else one CTA per work item; else
+ * the CUDA-core fp32 path), 1 = CUDA-core path only, 2 = same as 0, 3 / 4 / 5 = tensor
+ * cores with a fixed kernel where the call allows it: 3 one CTA per work item, 4
+ * persistent CTAs that share each work item (split path, partitions <= 2048 tokens), 5
+ * persistent warp workers, one work item per warp (split path, partitions <= 512 tokens). All compute the
  * same function; they differ in how work is scheduled and how q.K and P.V are multiplied.
  * Returns PA_ERR_INVALID for any other value. Not thread-safe.
  */

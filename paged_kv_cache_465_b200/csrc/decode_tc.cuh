@@ -1471,7 +1471,9 @@ inline bool tc_supported(const pa_decode_desc* d) {
 // CTAs, 5 = persistent warps. The persistent kernels need the split path (a workspace for
 // the plan) and keep one partition's 16-token sub-tiles per warp in 32-entry register
 // windows: persistent CTAs (16-token blocks only) up to 32 * 4 sub-tiles (2048 tokens),
-// warp workers up to 32 sub-tiles (512 tokens).
+// warp workers up to 32 sub-tiles (512 tokens). Automatic: warp workers where they fit,
+// else one CTA per item (faster than the persistent CTAs wherever both were measured on
+// a B200: 1024-token partitions of 32 sequences, 512-token ones of 8 x 131072 tokens).
 inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
   const int P = d->partition_size;
   const bool cta_ok = split && d->block_size == kSub && P <= 32 * tc::kNW * kSub;
@@ -1479,8 +1481,7 @@ inline tc::TcKind tc_kind(const pa_decode_desc* d, bool split, int impl) {
   if (impl == 3) return tc::kTcGrid;
   if (impl == 4) return cta_ok ? tc::kTcCta : tc::kTcGrid;
   if (impl == 5) return warps_ok ? tc::kTcWarps : (cta_ok ? tc::kTcCta : tc::kTcGrid);
-  if (warps_ok) return tc::kTcWarps;
-  return cta_ok ? tc::kTcCta : tc::kTcGrid;
+  return warps_ok ? tc::kTcWarps : tc::kTcGrid;
 }
 
 inline cudaError_t launch_tc(const DecodeArgs& a, const pa_decode_desc* d, dim3 grid,

@@ -38,17 +38,19 @@ bool desc_ok(const pa_decode_desc* d) {
   return true;
 }
 
-// The partition the library takes for PA_PARTITION_AUTO: 512 tokens when a context may be
-// longer than that, else one pass (0). Measured on a B200 over 64 .. 512-token partitions
-// and both persistent kernel families: 32 sequences of up to 4096 tokens decode fastest
-// split at 512 (0.059 ms, against 0.065 at 128 or 256 and 0.070 in one pass); 100
-// sequences of 250 tokens in one pass (0.027 ms, against 0.032 at 256). Fewer, longer
-// items win because every item costs a fetch, a partial and its share of the reduce. It
-// depends on max_context_len only, never on the context lengths themselves (device data)
-// or on where blocks sit, so results stay independent of the physical placement.
+// The partition the library takes for PA_PARTITION_AUTO: one pass (0) when no context can
+// exceed 512 tokens; else 512 tokens when there are at least 1024 (sequence, kv head)
+// pairs, else 1024. Measured on a B200 (decode call, fraction of the measured copy
+// bandwidth): 256 sequences x 8 kv heads up to 8192 tokens, fp8: 0.77 at 512 (warp
+// workers) against 0.73 at 1024 (one CTA per item); 32 x 8 up to 4096 tokens, bf16: 0.63
+// at 1024 against 0.59 at 512 and 0.49 in one pass; 8 x 8 at 131072 tokens, bf16: 1.00 at
+// 1024 against 0.95 at 512; 100 x 8 at 250 tokens: one pass fastest. With few pairs,
+// longer items split over a CTA's four warps finish sooner. It depends on the shape only,
+// never on the context lengths themselves (device data) or on where blocks sit, so
+// results stay independent of the physical placement.
 int auto_partition(const pa_decode_desc* d, int max_context_len) {
-  (void)d;
-  return max_context_len > 512 ? 512 : 0;
+  if (max_context_len <= 512) return 0;
+  return (int64_t)d->num_seqs * d->num_kv_heads >= 1024 ? 512 : 1024;
 }
 
 // desc with PA_PARTITION_AUTO replaced by the partition the library takes.

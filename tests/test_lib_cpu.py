@@ -258,15 +258,17 @@ def test_prefill_host_validation_without_device(pa):
 
 
 def test_library_chosen_partition(pa):
-    """PA_PARTITION_AUTO: 512-token partitions when a context may be longer than 512 tokens,
-    else one pass; the workspace and the launch count follow the chosen partition."""
+    """PA_PARTITION_AUTO: one pass when no context exceeds 512 tokens, else 512-token
+    partitions for at least 1024 (sequence, kv head) pairs and 1024-token ones for fewer;
+    the workspace and the launch count follow the chosen partition."""
     for S, Hkv, L, B in [(32, 8, 4096, 16), (256, 8, 8192, 16), (100, 8, 250, 16),
                          (8, 8, 131072, 16), (1, 1, 512, 16), (1, 1, 513, 8), (3, 2, 40, 32),
-                         (4096, 8, 600, 32), (64, 8, 1000, 8)]:
+                         (4096, 8, 600, 32), (64, 8, 1000, 8), (128, 8, 1000, 16),
+                         (127, 8, 1000, 16)]:
         d = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, pa.PARTITION_AUTO, pa.PA_BF16,
                          pa.PA_BF16, pa.PA_BF16, block_size=B)
         p = pa.partition_size_for(d, L)
-        assert p == (512 if L > 512 else 0), (S, Hkv, L, p)
+        assert p == (0 if L <= 512 else 512 if S * Hkv >= 1024 else 1024), (S, Hkv, L, p)
         e = pa.make_desc(S, 4 * Hkv, Hkv, 128, -(-L // B), 1 << 16, p, pa.PA_BF16, pa.PA_BF16,
                          pa.PA_BF16, block_size=B)
         assert pa.workspace_size(d, L) == pa.workspace_size(e, L)
