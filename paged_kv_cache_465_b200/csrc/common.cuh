@@ -65,6 +65,13 @@ __device__ __forceinline__ float2 f16x2_to_float2(uint32_t h) {
   return make_float2(lo, hi);
 }
 
+// 1/x on the special-function unit (PTX rcp.approx, subnormals kept; about one ulp).
+__device__ __forceinline__ float fast_rcp(float x) {
+  float y;
+  asm("rcp.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // 2^x on the special-function unit (PTX ex2.approx; relative error ~2^-22).
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;

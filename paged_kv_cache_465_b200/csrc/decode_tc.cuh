@@ -287,6 +287,10 @@ __device__ __forceinline__ float load_q_frags(const uint16_t* qp, int G, int lan
 // before the softmax, so a warp has independent work in flight at every step.
 // Per-half dequantisation parameters of a 16-token sub-tile: tokens 0-7 come from one
 // block and 8-15 from another when blocks hold 8 tokens; otherwise both halves are equal.
+// Growth of a score over its head's reference maximum (log2 units) that P may absorb
+// before the reference is raised (P <= 2^kSlack).
+constexpr float kSlack = 8.f;
+
 struct HalfParams {
   float zs0, zs1;              // log2-domain score scale (x K scale) of each half
   float vs0, vs1;              // V scale of each half
@@ -305,9 +309,12 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid,
   float pv0 = 1.f, pv1 = 1.f, beta = 1.f;
   if constexpr (FP8) {
     const float vnew = fmaxf(w.vref, fmaxf(hp.vs0, hp.vs1));
-    beta = w.vref > 0.f ? w.vref / vnew : 1.f;
-    pv0 = vnew > 0.f ? hp.vs0 / vnew : 0.f;
-    pv1 = vnew > 0.f ? hp.vs1 / vnew : 0.f;
+    // one approximate reciprocal rather than three divisions (P is rounded to f16 next);
+    // beta stays exactly 1 while the reference does not grow
+    const float rv = vnew > 0.f ? fast_rcp(vnew) : 0.f;
+    beta = (w.vref > 0.f && vnew != w.vref) ? w.vref * rv : 1.f;
+    pv0 = hp.vs0 * rv;
+    pv1 = hp.vs1 * rv;
     w.vref = vnew;
   }
   // rows of tokens past the item may hold anything (even NaN): zero them before P.V reads
@@ -384,18 +391,27 @@ __device__ __forceinline__ void tc_block(uint32_t kt, uint32_t vt, int nvalid,
   const float z1 = va ? (sa[1] + sb[1]) * hp.zs0 : -INFINITY;
   const float z2 = vb ? (sa[2] + sb[2]) * hp.zs1 : -INFINITY;
   const float z3 = vb ? (sa[3] + sb[3]) * hp.zs1 : -INFINITY;
+  // The reference m of a head is raised (to the running maximum, found across the 8 lanes
+  // of the head) only when a score exceeds it by more than kSlack; otherwise P is taken
+  // against the stale m and may reach 2^kSlack (f16 holds it exactly as well as a value
+  // below 1), so most sub-tiles skip the cross-lane maximum and the rescale. The outcome
+  // depends only on the scores, never on where the blocks sit.
   float bm0 = fmaxf(z0, z2), bm1 = fmaxf(z1, z3);
+  float al0 = 1.f, al1 = 1.f;
+  if (__any_sync(0xffffffffu, bm0 > w.m0 + kSlack || bm1 > w.m1 + kSlack)) {
 #pragma unroll
-  for (int o = 4; o < 32; o <<= 1) {
-    bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
-    bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
+    for (int o = 4; o < 32; o <<= 1) {
+      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, o));
+      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, o));
+    }
+    const float mn0 = fmaxf(w.m0, bm0), mn1 = fmaxf(w.m1, bm1);
+    al0 = fast_exp2(w.m0 - mn0);
+    al1 = fast_exp2(w.m1 - mn1);
+    w.m0 = mn0;
+    w.m1 = mn1;
   }
-  const float mn0 = fmaxf(w.m0, bm0), mn1 = fmaxf(w.m1, bm1);
-  const float al0 = fast_exp2(w.m0 - mn0), al1 = fast_exp2(w.m1 - mn1);
-  w.m0 = mn0;
-  w.m1 = mn1;
-  const float p0 = fast_exp2(z0 - mn0), p1 = fast_exp2(z1 - mn1);
-  const float p2 = fast_exp2(z2 - mn0), p3 = fast_exp2(z3 - mn1);
+  const float p0 = fast_exp2(z0 - w.m0), p1 = fast_exp2(z1 - w.m1);
+  const float p2 = fast_exp2(z2 - w.m0), p3 = fast_exp2(z3 - w.m1);
   w.l0 = w.l0 * al0 + (p0 + p2);
   w.l1 = w.l1 * al1 + (p1 + p3);
   if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f || beta != 1.f)) {
@@ -574,6 +590,19 @@ __device__ __forceinline__ SubWin shfl_sub(const SubWin& w, int k) {
   } else {
     r.p1 = r.p0; r.ks1 = r.ks0; r.vs1 = r.vs0; r.z1 = r.z0;
   }
+  return r;
+}
+
+__device__ __forceinline__ SubWin select_sub(bool first, const SubWin& a, const SubWin& b) {
+  SubWin r;
+  r.p0 = first ? a.p0 : b.p0;
+  r.p1 = first ? a.p1 : b.p1;
+  r.ks0 = first ? a.ks0 : b.ks0;
+  r.vs0 = first ? a.vs0 : b.vs0;
+  r.ks1 = first ? a.ks1 : b.ks1;
+  r.vs1 = first ? a.vs1 : b.vs1;
+  r.z0 = first ? a.z0 : b.z0;
+  r.z1 = first ? a.z1 : b.z1;
   return r;
 }
 
@@ -1175,12 +1204,15 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     while (!dead && g_iss - g_cons < (uint32_t)NST) {
       if (pslot == 0 && pk >= cur.nsub) { pslot = 1; pk = 0; }
       if (pslot == 1 && (!nxt.valid || pk >= nxt.nsub)) break;
-      const Item& v = pslot == 0 ? cur : nxt;
-      const SubWin sw = shfl_sub<BS>(pslot == 0 ? cur_w : nxt_w, pk);
+      // field-wise selects: a reference to one of the two items would put both in local
+      // memory
+      const bool first = pslot == 0;
+      const int c_begin = first ? cur.c_begin : nxt.c_begin, kvh = first ? cur.kvh : nxt.kvh;
+      const SubWin sw = shfl_sub<BS>(select_sub(first, cur_w, nxt_w), pk);
       const int stage = g_iss % NST;
       if (lane == 0)
         issue_sub<KV, BS>(wtiles + stage * STAGE, &kmap, &vmap, bars + 8 * stage, policy, sw,
-                          v.c_begin + pk, v.kvh, Hkv);
+                          c_begin + pk, kvh, Hkv);
       ++g_iss;
       ++pk;
     }

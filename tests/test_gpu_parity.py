@@ -341,6 +341,26 @@ def test_ragged_lengths_and_needles(pa, scen, impl, name, part, lens):
         _run_and_compare(pa, scen, d, impl, partition_size=part)
 
 
+@pytest.mark.parametrize("impl", SPLIT_IMPLS)
+@pytest.mark.parametrize("part", [512, 0])
+def test_fp8_query_dynamic_range(pa, scen, impl, part):
+    """fp8 cache, q with a wide range of magnitudes: the heads of a group 2^-8, 2^-4, 1 and
+    2 apart and every channel scaled by 2^u, u uniform in [-12, 3] (bf16 inputs), with and
+    without a needle. The tensor-core kernels take the K codes into 8-bit products against
+    q split into two E4M3 codes per element under a power of two per head; this is the
+    case where one power of two per group, or one E4M3 code per element, would fail."""
+    lens = [16, 17, 500, 700, 1500, 2049]
+    wl = workloads.WORKLOADS["b256"].scaled(num_seqs=len(lens))
+    assert wl.kv_dtype == "fp8" and wl.group == 4
+    rng = np.random.default_rng(465)
+    head = 2.0 ** np.array([-8, -4, 0, 1] * (wl.num_q_heads // 4))
+    chan = 2.0 ** rng.uniform(-12.0, 3.0, size=(len(lens), wl.num_q_heads, wl.head_dim))
+    scale = (head[None, :, None] * chan).astype(np.float32)
+    for needle in (False, True):
+        d = workloads.draw(wl, lens_override=lens, needle=needle, q_scale=scale)
+        _run_and_compare(pa, scen, d, impl, partition_size=part)
+
+
 @pytest.mark.parametrize("impl", ["simt", "auto"])
 def test_zero_query_is_mean_of_values(pa, scen, impl):
     wl = workloads.WORKLOADS["b32"].scaled(num_seqs=3)

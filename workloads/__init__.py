@@ -118,7 +118,8 @@ class Draw:
     """
 
     def __init__(self, wl: Workload, needle: bool = False, q_zero: bool = False,
-                 lens_override: Optional[List[int]] = None):
+                 lens_override: Optional[List[int]] = None,
+                 q_scale: Optional[np.ndarray] = None):
         self.wl = wl
         self.needle = needle
         ss = np.random.SeedSequence(wl.seed)
@@ -148,6 +149,8 @@ class Draw:
         qf = qrng.standard_normal((S, wl.num_q_heads, wl.head_dim), dtype=np.float32)
         if q_zero:
             qf[:] = 0.0
+        if q_scale is not None:     # per-(seq, head, channel) factors, broadcast over q
+            qf = (qf * np.asarray(q_scale, dtype=np.float32)).astype(np.float32)
         self.q = self._typed(qf)
         # Needle: one token per (seq, kv head) whose key is c * (mean query of the group),
         # so that its logit dominates; its position is drawn uniformly over the context.
