@@ -1192,11 +1192,13 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
   int pslot = 0, pk = 0;
   uint32_t g_iss = 0, g_cons = 0;
   bool dead = false;
-  // The first item streams before the second is fetched (the producer stops at the end of
-  // an item whose successor is not resolved yet), and before the plan has finished. Not
-  // with 8-token blocks, where the extra live state would spill: there both items are
-  // resolved first.
+  // The first item streams, and is consumed, before the plan has finished: the second is
+  // fetched (which waits for the plan kernel) only NST + 1 sub-tiles before the end of the
+  // first, and the producer stops at the end of an item whose successor is not resolved
+  // yet. Not with 8-token blocks, where the extra live state would spill: there both items
+  // are resolved first.
   constexpr bool kRamp = BS != 8;
+  bool listed = false;  // the plan has finished and the second item is resolved
   Item cur = static_item(), nxt{0, 0, 0, 0, 0, 0, 0, 0};
   SubWin cur_w, nxt_w;
   empty_sub(nxt_w);
@@ -1222,20 +1224,25 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     copy_q(cur);
     produce();
   };
-  if constexpr (kRamp) {
-    if (cur.valid) start();
+  auto take_list = [&]() {
     pdl_wait();  // the plan kernel's list and counters
     total = pl.counters[1];
-    if (!cur.valid) {  // no static item: the first comes from the list
-      cur = fetch();
-      if (cur.valid) start();
+    listed = true;
+  };
+  if constexpr (kRamp) {
+    if (cur.valid) start();
+    if (!cur.valid || cur.nsub <= NST + 1) {
+      take_list();
+      if (!cur.valid) {  // no static item: the first comes from the list
+        cur = fetch();
+        if (cur.valid) start();
+      }
+      nxt = fetch();
+      load_window(nxt, nxt_w);
+      produce();
     }
-    nxt = fetch();
-    load_window(nxt, nxt_w);
-    produce();
   } else {
-    pdl_wait();
-    total = pl.counters[1];
+    take_list();
     if (!cur.valid) cur = fetch();
     nxt = fetch();
     load_window(nxt, nxt_w);
@@ -1257,7 +1264,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     const float zscale = load_q_frags<FP8>(reinterpret_cast<const uint16_t*>(qbuf), G, lane,
                                            a.scale_log2, qf);
     __syncwarp();
-    if (!dead) copy_q(nxt);  // the buffer is free once every lane holds its fragments
+    if (!dead && listed) copy_q(nxt);  // the buffer is free once every lane holds its fragments
     w.reset();
     for (int i = 0; i < cur.nsub; ++i) {
       const SubWin sw = shfl_sub<BS>(cur_w, i);
@@ -1273,6 +1280,12 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
       }
       __syncwarp();
       ++g_cons;
+      if (kRamp && !listed && i + 1 >= cur.nsub - NST - 1) {  // the first item's successor
+        take_list();
+        nxt = fetch();
+        load_window(nxt, nxt_w);
+        if (!dead) copy_q(nxt);
+      }
       produce();
     }
     // ---- item done: its output (single partition) or its partial ----
