@@ -101,6 +101,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     if (global_ns() - t0 > kWaitNs) return false;
   }
 }
+// Store with an L2 eviction-priority policy (the split partials: kept in L2 for the reduce
+// launch that reads them right after, while the K/V stream passes through evict-first).
+__device__ __forceinline__ void st_hint(float* p, float v, uint64_t policy) {
+  asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy)
+               : "memory");
+}
+__device__ __forceinline__ uint64_t evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -1299,6 +1310,7 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
     const int g0 = 2 * tq, g1 = 2 * tq + 1;
     const bool live0 = g0 < G, live1 = g1 < G;
     const float ms[2] = {w.m0, w.m1}, ls[2] = {w.l0, w.l1};
+    const uint64_t keep = evict_last_policy();
 #pragma unroll
     for (int t = 0; t < 8; ++t) {
       int dA, dB;
@@ -1320,8 +1332,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
           store_out(a.out, a.out_dtype, row * kD + dB, x1 * inv);
         } else {
           const int64_t pr = (row * a.max_parts + cur.part) * kD;
-          a.part_acc[pr + dA] = x0;
-          a.part_acc[pr + dB] = x1;
+          st_hint(a.part_acc + pr + dA, x0, keep);
+          st_hint(a.part_acc + pr + dB, x1, keep);
         }
       }
     }
@@ -1335,8 +1347,8 @@ decode_tc_warps(const DecodeArgs a, const PlanView pl, const __grid_constant__ C
             a.lse_out[row] = ls[h] > 0.f ? (ms[h] + __log2f(ls[h])) * kLn2 : -INFINITY;
         } else {
           const int64_t pr = row * a.max_parts + cur.part;
-          a.part_m[pr] = ms[h];
-          a.part_l[pr] = ls[h];
+          st_hint(a.part_m + pr, ms[h], keep);
+          st_hint(a.part_l + pr, ls[h], keep);
         }
       }
     }
