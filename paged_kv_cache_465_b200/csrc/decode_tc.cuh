@@ -26,8 +26,8 @@
 // q is scaled by a power of two into f16 range (undone exactly in the score scale). The
 // per-(block, kv head) K scale folds into the score scale; the V scale folds into P as
 // P * v_scale[b] / v_ref, where v_ref is the running maximum V scale of the warp (the
-// accumulator is rescaled when it grows, like the running softmax maximum), so P stays
-// within [0, 1].
+// accumulator is rescaled when it grows, like the running softmax maximum), so the weight
+// never exceeds P itself (at most 2^8 with the lazy softmax maximum of tc_block).
 //
 // Every wait on an mbarrier is bounded (about one second of %globaltimer); on expiry the
 // warp records PA_DEVERR_TIMEOUT, stops consuming, waits (bounded) for the copies it
