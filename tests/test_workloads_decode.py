@@ -23,6 +23,21 @@ def test_draws_are_reproducible():
     assert not np.array_equal(workloads.draw("b32").q[:4], workloads.draw("b256").q[:4])
 
 
+def test_query_scale_option_scales_before_bf16_rounding():
+    # the q dynamic-range parity case: per-element factors applied to the float32 draw,
+    # then rounded to bf16 like every bf16 input; K/V and lengths are untouched
+    wl = workloads.WORKLOADS["b256"].scaled(num_seqs=3)
+    base = workloads.draw(wl, lens_override=[5, 40, 700])
+    f = np.full((3, wl.num_q_heads, wl.head_dim), 2.0 ** -6, dtype=np.float32)
+    f[:, 1::4] = 2.0 ** 3
+    d = workloads.draw(wl, lens_override=[5, 40, 700], q_scale=f)
+    # power-of-two factors commute with bf16 rounding (no under- or overflow here)
+    expect = codecs.bf16_decode(base.q).astype(np.float64) * f
+    assert np.array_equal(codecs.bf16_decode(d.q).astype(np.float64), expect)
+    assert np.array_equal(d.kv(2)[0], base.kv(2)[0])
+    assert np.array_equal(d.context_lens, base.context_lens)
+
+
 def test_length_distributions():
     W = workloads.WORKLOADS
     assert workloads.draw("tiny").context_lens.tolist() == [5, 16, 17, 40]
